@@ -1,0 +1,44 @@
+"""Closed-form work and byte counts for the roofline figures.
+
+Prefill FLOPs count only visible (query, key) pairs: 2*d for q.k plus 2*d for
+p*v per pair, so 4 * d per pair per query head. Visible pairs per head:
+full N^2, causal N(N+1)/2, window sum_i min(i+1, w).
+
+Decode bytes count the K and V bytes a step must read from HBM:
+sum_b seq_len_b * Hkv * d * 2 (K and V) * 2 (bf16).
+"""
+
+from __future__ import annotations
+
+MASK_IDS = {"full": 0, "causal": 1, "window": 2}
+
+
+def visible_pairs(n: int, mask: str, window: int = 0) -> int:
+    if mask == "full":
+        return n * n
+    if mask == "causal":
+        return n * (n + 1) // 2
+    if mask == "window":
+        w = min(int(window), n)
+        # rows 0..w-1 see i+1 keys, the remaining n-w rows see w keys
+        return w * (w + 1) // 2 + (n - w) * w
+    raise ValueError(mask)
+
+
+def prefill_flops(B: int, Hq: int, N: int, d: int, mask: str, window: int = 0) -> int:
+    return 4 * B * Hq * d * visible_pairs(N, mask, window)
+
+
+def prefill_io_bytes(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:
+    """Compulsory HBM bytes of one prefill: Q, K, V read, O (bf16) and LSE (fp32) written."""
+    return 2 * B * N * d * (2 * Hq + 2 * Hkv) + 4 * B * Hq * N
+
+
+def decode_kv_bytes(seq_lens, Hkv: int, d: int) -> int:
+    return sum(int(n) for n in seq_lens) * Hkv * d * 2 * 2
+
+
+def decode_io_bytes(seq_lens, B: int, Hq: int, Hkv: int, d: int, block_size: int) -> int:
+    """KV bytes plus q, o, lse, block-table and seq_len bytes."""
+    tables = sum(-(-int(n) // block_size) for n in seq_lens) * 4 + 4 * B
+    return decode_kv_bytes(seq_lens, Hkv, d) + B * Hq * d * 2 * 2 + B * Hq * 4 + tables
