@@ -1,3 +1,148 @@
-"""Exact softmax attention (causal / sliding-window / full GQA prefill and
-paged decode) for NVIDIA B200, behind a C-ABI library of hand-written sm_100a
-CUDA kernels. This module is the thin Python binding over that library."""
+"""Exact softmax attention for NVIDIA B200 (sm_100a).
+
+Causal / sliding-window / full grouped-query prefill and paged single-token
+decode, computed by hand-written CUDA kernels behind the C ABI of
+``include/attn.h``. This module is the thin Python binding: it checks tensor
+dtypes, shapes and devices, allocates outputs with PyTorch (device memory
+plumbing only) and passes raw pointers and the current CUDA stream to the
+library. Every step of the computation runs in the library's kernels; there
+is no CPU or PyTorch fallback, and calls raise if the library is not built.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from . import _lib
+from ._lib import AttnError, STATUS_BIT_DEVICE_CHECK, STATUS_BIT_TIMEOUT  # noqa: F401
+
+MASKS = {"full": 0, "causal": 1, "window": 2, "sliding_window": 2}
+
+__all__ = ["prefill", "decode_paged", "paged_gather", "decode_plan", "decode_workspace_bytes", "AttnError",
+           "version"]
+
+
+def version() -> int:
+    return int(_lib.lib().attn_version())
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got {t.dim()}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def prefill(q, k, v, mask: str = "causal", window: int = 0, scale: float | None = None, out=None, lse=None,
+            status=None, stream=None, return_lse: bool = True):
+    """O = softmax(scale * Q K^T + M) V for every query row; returns (O, LSE).
+
+    q [B, Hq, N, d], k/v [B, Hkv, N, d], bf16 CUDA tensors; O bf16 like q,
+    LSE fp32 [B, Hq, N] (natural log). mask: "full", "causal" or "window"
+    (keys i - window < j <= i).
+    """
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    _need(v, "v", torch.bfloat16, 4)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, N, d] matching q")
+    if mask not in MASKS:
+        raise ValueError(f"mask must be one of {sorted(MASKS)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    rc = _lib.lib().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d, MASKS[mask],
+                                 int(window), float(scale), _ptr(status), _stream_handle(stream))
+    _lib.check(rc, "attn_prefill")
+    return out, lse
+
+
+def decode_plan(B: int, Hq: int, Hkv: int, max_seq_len: int, num_sms: int):
+    """(chunk_tokens, num_splits) of the split-KV decode plan; host only."""
+    chunk, splits = ctypes.c_int(0), ctypes.c_int(0)
+    rc = _lib.lib().attn_decode_plan(B, Hq, Hkv, max_seq_len, num_sms, ctypes.byref(chunk), ctypes.byref(splits))
+    _lib.check(rc, "attn_decode_plan")
+    return chunk.value, splits.value
+
+
+def decode_workspace_bytes(B: int, Hq: int, Hkv: int, d: int, max_seq_len: int, block_size: int) -> int:
+    n = int(_lib.lib().attn_decode_workspace_bytes(B, Hq, Hkv, d, max_seq_len, block_size))
+    if n == 0:
+        raise AttnError(_lib.ATTN_ERR_INVALID_ARG, "attn_decode_workspace_bytes")
+    return n
+
+
+def decode_paged(q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int, scale: float | None = None,
+                 out=None, lse=None, workspace=None, status=None, stream=None, return_lse: bool = True):
+    """One query token per sequence against its paged cache; returns (O, LSE).
+
+    q [B, Hq, d] bf16; caches [num_blocks, block_size, Hkv, d] bf16;
+    block_table [B, max_blocks] int32; seq_lens [B] int32.
+    """
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hq, d = q.shape
+    num_blocks, block_size, Hkv, d2 = k_cache.shape
+    if d2 != d or v_cache.shape != k_cache.shape:
+        raise ValueError("caches must be [num_blocks, block_size, Hkv, d] matching q")
+    if block_table.shape[0] != B or seq_lens.shape[0] != B:
+        raise ValueError("block_table and seq_lens need one row per sequence")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if workspace is None:
+        nbytes = decode_workspace_bytes(B, Hq, Hkv, d, max_seq_len, block_size)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    rc = _lib.lib().attn_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+                                      _ptr(out), _ptr(lse), B, Hq, Hkv, d, num_blocks, block_size,
+                                      block_table.shape[1], int(max_seq_len), float(scale), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _ptr(status),
+                                      _stream_handle(stream))
+    _lib.check(rc, "attn_decode_paged")
+    return out, lse
+
+
+def paged_gather(cache, block_table, seq_lens, max_seq_len: int, out=None, status=None, stream=None):
+    """Contiguous [B, Hkv, max_seq_len, d] copy of a paged cache (zeros past seq_len)."""
+    _need(cache, "cache", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    num_blocks, block_size, Hkv, d = cache.shape
+    B = block_table.shape[0]
+    if out is None:
+        out = torch.empty((B, Hkv, max_seq_len, d), dtype=cache.dtype, device=cache.device)
+    rc = _lib.lib().attn_paged_gather(_ptr(cache), _ptr(block_table), _ptr(seq_lens), _ptr(out), B, Hkv, d,
+                                      num_blocks, block_size, block_table.shape[1], int(max_seq_len), _ptr(status),
+                                      _stream_handle(stream))
+    _lib.check(rc, "attn_paged_gather")
+    return out

@@ -1,0 +1,523 @@
+// Paged single-token decode: split-KV partials + log-sum-exp merge, and the
+// bit-exact block-table gather.
+//
+// What it computes ("Module 09: Efficient Attention", "Code: A Paged KV Cache
+// from Scratch"; "USAAIO Lesson 90", part 2): for every sequence b and query
+// head h, softmax(scale * q_{b,h} . K_b^T) V_b over all seq_lens[b] cached
+// tokens, where token t of sequence b lives in slot t % block_size of physical
+// block block_table[b][t / block_size] of the pool
+// [num_blocks, block_size, Hkv, d].
+//
+// How ("Inference attention" post, "FlashDecoding"): the sequence is cut into
+// chunks of `chunk` tokens. One CTA handles one (chunk, K/V head, query-head
+// chunk of <= 16, sequence). Its 4 warps each stream 16-token sub-blocks of
+// K and V through a private 3-stage cp.async ring in shared memory (16-byte
+// loads of whole 256-byte head rows), score the <= 16 query heads of the
+// group against them with mma.sync m16n8k16 (bf16 in, fp32 accumulate), and
+// keep FlashAttention's running (max, sum, output) per query head. The warps
+// combine in shared memory and write one normalised partial output and its
+// log-sum-exp per (sequence, head, chunk). The merge kernel combines the
+// chunks with the online softmax's rescaling.
+//
+// The kernel is HBM-bound: each K/V byte of a (sequence, K/V head) is read
+// once and shared by the whole query-head group.
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace attn {
+namespace {
+
+constexpr int kDecWarps = 4;
+constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kStages = 3;  // per-warp ring depth
+constexpr int kSub = 16;    // tokens per sub-block
+
+struct DecodeParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k_cache;
+  const __nv_bfloat16* v_cache;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  float* o_part;    // [B, Hq, splits, D]
+  float* lse_part;  // [B, Hq, splits]
+  int32_t* status;
+  int B, Hq, Hkv, group, hchunks;
+  int num_blocks, block_size, max_blocks_per_seq, max_seq_len;
+  int chunk, splits;
+  float scale_log2;  // scale * log2(e): scores live in the base-2 domain
+};
+
+__device__ __forceinline__ void flag_status(int32_t* status, int bit) {
+  if (status != nullptr) atomicOr(status, bit);
+}
+
+// Shared memory: Q tile [16][D] then, per warp, kStages x (K [16][D], V [16][D]).
+// Rows are 16-byte-chunk swizzled: chunk c of row r lives at chunk c ^ (r & 7),
+// which makes every ldmatrix phase hit 8 distinct bank groups.
+template <int D>
+struct DecSmem {
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kChunks = kRowBytes / 16;
+  static constexpr int kTile = kSub * kRowBytes;
+  static constexpr int kRing = kDecWarps * kStages * 2 * kTile;
+  static constexpr int kTotal = kTile + kRing + 64;
+};
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk, int row_bytes) {
+  return static_cast<uint32_t>(row * row_bytes + ((chunk ^ (row & 7)) << 4));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeParams p) {
+  using L = DecSmem<D>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* q_s = smem;
+  uint8_t* ring = smem + L::kTile;
+  int* cta_bad = reinterpret_cast<int*>(smem + L::kTile + L::kRing);
+
+  const int split = blockIdx.x;
+  const int kvh = blockIdx.y / p.hchunks;
+  const int hc = blockIdx.y % p.hchunks;
+  const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int seq_len = p.seq_lens[b];
+  if (seq_len < 1 || seq_len > p.max_seq_len) return;  // the merge kernel flags this row
+  const int t0 = split * p.chunk;
+  if (t0 >= seq_len) return;  // chunk past the end: the merge never reads it
+  const int t1 = min(t0 + p.chunk, seq_len);
+  const int nsub = (t1 - t0 + kSub - 1) / kSub;
+  const int h0 = kvh * p.group + hc * 16;
+  const int rows = min(16, p.group - hc * 16);
+
+  if (threadIdx.x == 0) *cta_bad = 0;
+  // Q rows of this head chunk -> swizzled shared tile; padding rows are zero.
+  for (int i = threadIdx.x; i < 16 * L::kChunks; i += kDecThreads) {
+    const int r = i / L::kChunks, c = i % L::kChunks;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (r < rows)
+      val = *reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.Hq + h0 + r) * D + c * 8);
+    *reinterpret_cast<uint4*>(q_s + swz(r, c, L::kRowBytes)) = val;
+  }
+  __syncthreads();
+
+  // A fragments of Q for every 16-wide k step (rows = query heads).
+  uint32_t qf[D / 16][4];
+  {
+    const uint32_t qb = smem_u32(q_s);
+    const int r = lane & 15;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int c = kk * 2 + (lane >> 4);
+      ldmatrix_x4(qb + swz(r, c, L::kRowBytes), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+    }
+  }
+
+  // Per-warp streaming over sub-blocks warp, warp + 4, ...
+  uint8_t* my_ring = ring + warp * kStages * 2 * L::kTile;
+  const int n_my = (nsub > warp) ? (nsub - warp + kDecWarps - 1) / kDecWarps : 0;
+  bool bad = false;
+
+  auto issue = [&](int j, int stage) {
+    const int t = t0 + (warp + j * kDecWarps) * kSub;  // first token of the sub-block
+    const int lblk = t / p.block_size;
+    const int off = t - lblk * p.block_size;  // multiple of 16, off + 15 < block_size
+    const int phys = __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks_per_seq + lblk);
+    const bool ok = (phys >= 0) && (phys < p.num_blocks);
+    bad |= !ok;
+    const uint32_t kdst = smem_u32(my_ring + stage * 2 * L::kTile);
+#pragma unroll
+    for (int x = lane; x < kSub * L::kChunks; x += 32) {
+      const int r = x / L::kChunks, c = x % L::kChunks;
+      const bool valid = ok && (t + r < t1);  // slots past seq_len are zero-filled, never read
+      const size_t src = valid ? ((static_cast<size_t>(phys) * p.block_size + off + r) * p.Hkv + kvh) * D + c * 8
+                               : 0;
+      const uint32_t dst = kdst + swz(r, c, L::kRowBytes);
+      cp_async_16(dst, p.k_cache + src, valid ? 16u : 0u);
+      cp_async_16(dst + L::kTile, p.v_cache + src, valid ? 16u : 0u);
+    }
+  };
+
+  const float neg_inf = -INFINITY;
+  float m_run[2] = {neg_inf, neg_inf};  // rows g and g + 8 of this lane (base-2 domain)
+  float l_run[2] = {0.f, 0.f};          // per-lane partial sums; reduced over the quad at the end
+  float o_acc[D / 8][4];
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) o_acc[n][0] = o_acc[n][1] = o_acc[n][2] = o_acc[n][3] = 0.f;
+
+  const int g = lane >> 2, tq = lane & 3;
+
+#pragma unroll
+  for (int j = 0; j < kStages - 1; ++j) {
+    if (j < n_my) issue(j, j);
+    cp_async_commit();
+  }
+  for (int j = 0; j < n_my; ++j) {
+    const int jn = j + kStages - 1;
+    if (jn < n_my) issue(jn, jn % kStages);
+    cp_async_commit();
+    cp_async_wait<kStages - 1>();
+    __syncwarp();
+
+    const uint32_t kb = smem_u32(my_ring + (j % kStages) * 2 * L::kTile);
+    const uint32_t vb = kb + L::kTile;
+    const int tok0 = t0 + (warp + j * kDecWarps) * kSub;
+
+    // S = Q K^T for 16 tokens: two n-tiles of 8 tokens.
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int r = ((lane >> 4) << 3) + (lane & 7);
+      const int c = kk * 2 + ((lane >> 3) & 1);
+      uint32_t b00, b01, b10, b11;
+      ldmatrix_x4(kb + swz(r, c, L::kRowBytes), b00, b01, b10, b11);
+      mma_bf16_16816(s[0], qf[kk], b00, b01);
+      mma_bf16_16816(s[1], qf[kk], b10, b11);
+    }
+    // scale into base 2, mask slots past the sequence end
+    float mx[2] = {neg_inf, neg_inf};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tok = tok0 + nt * 8 + 2 * tq + (e & 1);
+        const float x = (tok < t1) ? s[nt][e] * p.scale_log2 : neg_inf;
+        s[nt][e] = x;
+        mx[e >> 1] = fmaxf(mx[e >> 1], x);
+      }
+    }
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
+      mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
+    }
+    // the first token of a sub-block is always < t1, so mx is finite
+    float alpha[2];
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const float m_new = fmaxf(m_run[rr], mx[rr]);
+      alpha[rr] = fast_exp2(m_run[rr] - m_new);  // 0 on the first sub-block (m_run = -inf)
+      m_run[rr] = m_new;
+      l_run[rr] *= alpha[rr];
+    }
+    float pr[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        pr[nt][e] = fast_exp2(s[nt][e] - m_run[e >> 1]);
+        l_run[e >> 1] += pr[nt][e];
+      }
+    uint32_t pa[4];
+    pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
+    pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
+    pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
+    pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      o_acc[n][0] *= alpha[0];
+      o_acc[n][1] *= alpha[0];
+      o_acc[n][2] *= alpha[1];
+      o_acc[n][3] *= alpha[1];
+    }
+    // O += P V: V rows are tokens (k), columns are the head dim (n) -> trans loads.
+#pragma unroll
+    for (int n = 0; n < D / 8; n += 2) {
+      const int r = (lane & 7) + (((lane >> 3) & 1) << 3);
+      const int c = n + (lane >> 4);
+      uint32_t b0a, b1a, b0b, b1b;
+      ldmatrix_x4_trans(vb + swz(r, c, L::kRowBytes), b0a, b1a, b0b, b1b);
+      mma_bf16_16816(o_acc[n], pa, b0a, b1a);
+      mma_bf16_16816(o_acc[n + 1], pa, b0b, b1b);
+    }
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 1);
+    l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 2);
+  }
+  if (bad) atomicOr(cta_bad, 1);
+  __syncthreads();  // every warp is done with its ring: reuse it for the combine
+
+  // Combine the 4 warps: per warp m[16], l[16], O[16][D] (unnormalised, fp32).
+  float* wm = reinterpret_cast<float*>(ring);
+  float* wl = wm + kDecWarps * 16;
+  float* wo = wl + kDecWarps * 16;
+  if (tq == 0) {
+    wm[warp * 16 + g] = m_run[0];
+    wm[warp * 16 + g + 8] = m_run[1];
+    wl[warp * 16 + g] = l_run[0];
+    wl[warp * 16 + g + 8] = l_run[1];
+  }
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) {
+    const int col = n * 8 + 2 * tq;
+    float* w0 = wo + (warp * 16 + g) * D + col;
+    float* w1 = wo + (warp * 16 + g + 8) * D + col;
+    w0[0] = o_acc[n][0];
+    w0[1] = o_acc[n][1];
+    w1[0] = o_acc[n][2];
+    w1[1] = o_acc[n][3];
+  }
+  __syncthreads();
+
+  const bool cta_is_bad = (*cta_bad != 0);
+  if (cta_is_bad && threadIdx.x == 0) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
+  // 128 threads: thread -> (row = tid / 8, 8 threads per row, D / 8 columns each)
+  {
+    const int r = threadIdx.x >> 3;
+    const int part = threadIdx.x & 7;
+    if (r < rows) {
+      float M = neg_inf;
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, wm[w * 16 + r]);
+      float wsc[kDecWarps];
+      float Lsum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) {
+        wsc[w] = (wm[w * 16 + r] == neg_inf) ? 0.f : fast_exp2(wm[w * 16 + r] - M);
+        Lsum += wsc[w] * wl[w * 16 + r];
+      }
+      const float inv = 1.f / Lsum;
+      const size_t prow = (static_cast<size_t>(b) * p.Hq + h0 + r) * p.splits + split;
+      float* dst = p.o_part + prow * D;
+      for (int c = part * (D / 8); c < (part + 1) * (D / 8); c += 4) {
+        float4 acc;
+        float* a = &acc.x;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float v = 0.f;
+#pragma unroll
+          for (int w = 0; w < kDecWarps; ++w) v += wsc[w] * wo[(w * 16 + r) * D + c + e];
+          a[e] = cta_is_bad ? NAN : v * inv;
+        }
+        *reinterpret_cast<float4*>(dst + c) = acc;
+      }
+      if (part == 0) p.lse_part[prow] = cta_is_bad ? NAN : (M + __log2f(Lsum)) * kLn2;
+    }
+  }
+}
+
+struct MergeParams {
+  const float* o_part;
+  const float* lse_part;
+  const int32_t* seq_lens;
+  __nv_bfloat16* o;
+  float* lse;
+  int32_t* status;
+  int B, Hq, splits, chunk, max_seq_len;
+};
+
+// One warp per (sequence, query head): lse = log sum_s exp(lse_s),
+// O = sum_s exp(lse_s - lse) O_s, over the chunks that hold tokens.
+template <int D>
+__global__ void __launch_bounds__(128) decode_merge_kernel(const MergeParams p) {
+  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= p.B * p.Hq) return;
+  const int b = wid / p.Hq;
+  const size_t row = static_cast<size_t>(wid);
+  const int seq_len = p.seq_lens[b];
+  constexpr int PER = D / 32;  // columns per lane
+  __nv_bfloat16* orow = p.o + row * D + lane * PER;
+  if (seq_len < 1 || seq_len > p.max_seq_len) {
+    if (lane == 0) {
+      flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
+      if (p.lse) p.lse[row] = NAN;
+    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) orow[e] = __float2bfloat16_rn(NAN);
+    return;
+  }
+  const int ns = (seq_len + p.chunk - 1) / p.chunk;
+  const float* lrow = p.lse_part + row * p.splits;
+  float M = -INFINITY;
+  bool nan_seen = false;
+  for (int s = lane; s < ns; s += 32) {
+    const float x = lrow[s];
+    nan_seen |= (x != x);
+    M = fmaxf(M, x);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  nan_seen = __any_sync(0xffffffffu, nan_seen);
+  float total = 0.f;
+  for (int s = lane; s < ns; s += 32) total += fast_exp2((lrow[s] - M) * kLog2e);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+  const float lse = M + __logf(total);
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  const float* obase = p.o_part + row * p.splits * D + lane * PER;
+  for (int s = 0; s < ns; ++s) {
+    const float w = fast_exp2((lrow[s] - lse) * kLog2e);
+    const float* src = obase + static_cast<size_t>(s) * D;
+#pragma unroll
+    for (int e = 0; e < PER; e += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(src + e);
+      acc[e] += w * v.x;
+      acc[e + 1] += w * v.y;
+      acc[e + 2] += w * v.z;
+      acc[e + 3] += w * v.w;
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < PER; e += 2) {
+    const float a0 = nan_seen ? NAN : acc[e];
+    const float a1 = nan_seen ? NAN : acc[e + 1];
+    *reinterpret_cast<__nv_bfloat162*>(orow + e) = __floats2bfloat162_rn(a0, a1);
+  }
+  if (lane == 0 && p.lse) p.lse[row] = nan_seen ? NAN : lse;
+}
+
+// Gather: out[b][h][t][:] = cache[block_table[b][t / bs]][t % bs][h][:] for
+// t < seq_lens[b], zero for the rest of [0, max_seq_len). One thread per
+// 16-byte chunk; consecutive threads walk (head, chunk) of one token, which
+// is contiguous in the pool.
+__global__ void paged_gather_kernel(const uint4* __restrict__ cache, const int32_t* __restrict__ table,
+                                    const int32_t* __restrict__ seq_lens, uint4* __restrict__ out, int B, int Hkv,
+                                    int chunks_per_row, int num_blocks, int block_size, int max_blocks_per_seq,
+                                    int max_seq_len, int32_t* status) {
+  const size_t per_seq = static_cast<size_t>(max_seq_len) * Hkv * chunks_per_row;
+  const size_t total = per_seq * B;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int b = static_cast<int>(i / per_seq);
+    size_t rem = i - static_cast<size_t>(b) * per_seq;
+    const int t = static_cast<int>(rem / (static_cast<size_t>(Hkv) * chunks_per_row));
+    rem -= static_cast<size_t>(t) * Hkv * chunks_per_row;
+    const int h = static_cast<int>(rem / chunks_per_row);
+    const int c = static_cast<int>(rem - static_cast<size_t>(h) * chunks_per_row);
+    const int n = seq_lens[b];
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    const uint4 nan4 = make_uint4(0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u);  // bf16 NaN pairs
+    if (n < 0 || n > max_seq_len) {
+      val = nan4;
+      if (t == 0 && h == 0 && c == 0 && status) atomicOr(status, ATTN_STATUS_BIT_DEVICE_CHECK);
+    } else if (t < n) {
+      const int lblk = t / block_size;
+      const int phys = table[static_cast<size_t>(b) * max_blocks_per_seq + lblk];
+      if (phys < 0 || phys >= num_blocks) {
+        val = nan4;
+        if (h == 0 && c == 0 && status) atomicOr(status, ATTN_STATUS_BIT_DEVICE_CHECK);
+      } else {
+        val = cache[((static_cast<size_t>(phys) * block_size + (t - lblk * block_size)) * Hkv + h) * chunks_per_row +
+                    c];
+      }
+    }
+    out[((static_cast<size_t>(b) * Hkv + h) * max_seq_len + t) * chunks_per_row + c] = val;
+  }
+}
+
+template <int D>
+cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                            const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int num_blocks,
+                            int block_size, int max_blocks_per_seq, int max_seq_len, float scale, void* workspace,
+                            const DecodePlan& plan, int32_t* status, cudaStream_t stream) {
+  DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  p.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.o_part = static_cast<float*>(workspace);
+  p.lse_part = p.o_part + static_cast<size_t>(B) * Hq * plan.splits * D;
+  p.status = status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.group = Hq / Hkv;
+  p.hchunks = plan.hchunks;
+  p.num_blocks = num_blocks;
+  p.block_size = block_size;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.max_seq_len = max_seq_len;
+  p.chunk = plan.chunk;
+  p.splits = plan.splits;
+  p.scale_log2 = scale * kLog2e;
+
+  const int smem = DecSmem<D>::kTotal;
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(plan.splits, Hkv * plan.hchunks, B);
+  decode_split_kernel<D><<<grid, kDecThreads, smem, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  MergeParams m;
+  m.o_part = p.o_part;
+  m.lse_part = p.lse_part;
+  m.seq_lens = seq_lens;
+  m.o = static_cast<__nv_bfloat16*>(o);
+  m.lse = lse;
+  m.status = status;
+  m.B = B;
+  m.Hq = Hq;
+  m.splits = plan.splits;
+  m.chunk = plan.chunk;
+  m.max_seq_len = max_seq_len;
+  const int warps = B * Hq;
+  decode_merge_kernel<D><<<(warps + 3) / 4, 128, 0, stream>>>(m);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t decode_workspace_bytes(int B, int Hq, int d, const DecodePlan& plan) {
+  const size_t rows = static_cast<size_t>(B) * Hq * plan.splits;
+  return rows * d * sizeof(float) + rows * sizeof(float);
+}
+
+int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan* out) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_seq_len <= 0 || num_sms <= 0 || out == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  const int group = Hq / Hkv;
+  const int hchunks = (group + 15) / 16;
+  const long long units = static_cast<long long>(B) * Hkv * hchunks;
+  const long long target = 4LL * num_sms;  // CTAs: enough to fill every SM a few times over
+  int chunk = 2048;
+  while (chunk > 256 && units * ((max_seq_len + chunk - 1) / chunk) < target) chunk >>= 1;
+  out->chunk = chunk;
+  out->splits = (max_seq_len + chunk - 1) / chunk;
+  out->hchunks = hchunks;
+  return ATTN_OK;
+}
+
+cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                          const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int d,
+                          int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, float scale,
+                          void* workspace, const DecodePlan& plan, int32_t* status, cudaStream_t stream) {
+  if (d == 128)
+    return launch_decode_t<128>(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, num_blocks,
+                                block_size, max_blocks_per_seq, max_seq_len, scale, workspace, plan, status, stream);
+  return launch_decode_t<64>(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, num_blocks, block_size,
+                             max_blocks_per_seq, max_seq_len, scale, workspace, plan, status, stream);
+}
+
+cudaError_t launch_paged_gather(const void* cache, const int32_t* block_table, const int32_t* seq_lens, void* out,
+                                int B, int Hkv, int d, int num_blocks, int block_size, int max_blocks_per_seq,
+                                int max_seq_len, int32_t* status, cudaStream_t stream) {
+  const int chunks = d / 8;
+  const size_t total = static_cast<size_t>(B) * max_seq_len * Hkv * chunks;
+  const int threads = 256;
+  const size_t want = (total + threads - 1) / threads;
+  const int blocks = static_cast<int>(want < 65535 * 8 ? want : 65535 * 8);
+  paged_gather_kernel<<<blocks, threads, 0, stream>>>(static_cast<const uint4*>(cache), block_table, seq_lens,
+                                                      static_cast<uint4*>(out), B, Hkv, chunks, num_blocks,
+                                                      block_size, max_blocks_per_seq, max_seq_len, status);
+  return cudaGetLastError();
+}
+
+}  // namespace attn

@@ -1,0 +1,46 @@
+// Library-internal declarations shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "../../include/attn.h"
+
+namespace attn {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Bounded waits: clock64 cycles before a pipeline wait gives up (~0.5 s at
+// the B200's boost clock). Read per call from ATTN_WAIT_BUDGET_CYCLES when set.
+long long wait_budget_cycles();
+// Waits that drain in-flight copies and MMAs before a CTA exits use their own,
+// larger bound, so that a short pipeline budget never cuts a drain short.
+constexpr long long kDrainBudgetCycles = 4000000000LL;
+
+struct DecodePlan {
+  int chunk;       // tokens per split (multiple of 16)
+  int splits;      // ceil(max_seq_len / chunk)
+  int hchunks;     // query-head chunks of <= 16 per K/V head
+};
+
+int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan* out);
+size_t decode_workspace_bytes(int B, int Hq, int d, const DecodePlan& plan);
+
+// Kernel launchers (defined next to their kernels). Return cudaError_t.
+cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                          const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int d,
+                          int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, float scale,
+                          void* workspace, const DecodePlan& plan, int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_paged_gather(const void* cache, const int32_t* block_table, const int32_t* seq_lens, void* out,
+                                int B, int Hkv, int d, int num_blocks, int block_size, int max_blocks_per_seq,
+                                int max_seq_len, int32_t* status, cudaStream_t stream);
+
+// Returns ATTN_OK / ATTN_ERR_CUDA (tensor-map encoding or launch failure).
+int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                   int d, int mask_kind, int window, float scale, int32_t* status, cudaStream_t stream);
+
+}  // namespace attn

@@ -1,0 +1,181 @@
+/*
+ * attn.h - C ABI of the B200 (sm_100a) exact softmax attention library.
+ *
+ * Two operations, both exact scaled-dot-product attention
+ *     O = softmax(Q K^T * scale + M) V
+ * computed with an online softmax so that the score matrix never leaves the
+ * chip ("Module 5. Modern Attention Mechanisms", section 4, the SDPA
+ * definition; section 8, the FlashAttention recurrence):
+ *
+ *   attn_prefill       - every query row of a sequence against its own keys,
+ *                        full / causal / sliding-window mask, grouped-query
+ *                        heads (Hkv divides Hq; Hkv == Hq is MHA, Hkv == 1 MQA).
+ *   attn_decode_paged  - one query token per sequence against a paged K/V
+ *                        cache addressed through a block table
+ *                        ("Module 09: Efficient Attention", "The Block Table"),
+ *                        split along the sequence and merged by log-sum-exp
+ *                        ("Inference attention" post, section "FlashDecoding").
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers named q, k, v, o, lse, k_cache, v_cache, block_table, seq_lens,
+ *     out, workspace and status are DEVICE pointers owned by the caller; the
+ *     library never allocates, frees or retains them.
+ *   - bf16 means IEEE bfloat16 stored in 2 bytes; tensors are dense,
+ *     row-major ("C order") in the layouts stated per call, and every base
+ *     pointer is 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; 0 = legacy default
+ *     stream). A return of ATTN_OK means the work was validated and enqueued.
+ *   - Host-side argument errors return a negative status and launch nothing.
+ *   - Device-side checks (block-table entries, seq_lens, bounded waits) cannot
+ *     be reported by the return value; they OR a status code into *status
+ *     (when status != NULL) and turn the affected output rows into NaN. The
+ *     caller zeroes *status before the call and reads it after synchronising.
+ *   - head dimension d must be 64 or 128 (else ATTN_ERR_UNSUPPORTED).
+ *   - Query head h reads K/V head h / (Hq / Hkv): consecutive groups
+ *     ("Modern Attention Mechanisms", section 6).
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* attn_stream_t; /* the same handle as cudaStream_t */
+
+enum attn_status {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = -1,  /* bad size, null pointer, misalignment, Hq % Hkv != 0, ... */
+  ATTN_ERR_UNSUPPORTED = -2,  /* valid request this build does not implement (e.g. d = 96) */
+  ATTN_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed (launch, tensor map) */
+  ATTN_ERR_DEVICE_CHECK = -4, /* device bit: a block-table entry or seq_len was out of range */
+  ATTN_ERR_TIMEOUT = -5,      /* device bit: a bounded pipeline wait expired */
+  ATTN_ERR_WORKSPACE = -6     /* workspace pointer NULL or smaller than attn_decode_workspace_bytes */
+};
+
+/* Device-side status bits OR-ed into *status. */
+#define ATTN_STATUS_BIT_DEVICE_CHECK 0x1
+#define ATTN_STATUS_BIT_TIMEOUT 0x2
+
+enum attn_mask_kind {
+  ATTN_MASK_FULL = 0,          /* every key visible */
+  ATTN_MASK_CAUSAL = 1,        /* key j visible to query i iff j <= i */
+  ATTN_MASK_SLIDING_WINDOW = 2 /* key j visible iff 0 <= i - j < window (window includes i) */
+};
+
+/*
+ * attn_prefill - exact attention of N query rows against N keys per head.
+ *
+ * Defined by "Modern Attention Mechanisms", section 4: softmax over keys of
+ * Q K^T * scale with an additive mask, causality p_k <= p_q and the window
+ * 0 <= p_q - p_k < W (W positions including the current one); and section 6
+ * for the GQA head map. Query and key positions are aligned (square N).
+ *
+ *   q     [B, Hq,  N, d] bf16      read
+ *   k, v  [B, Hkv, N, d] bf16      read
+ *   o     [B, Hq,  N, d] bf16      written: softmax(...) V, rounded to nearest even
+ *   lse   [B, Hq,  N]    fp32      written when non-NULL: natural-log log-sum-exp
+ *                                  of the scaled scores over the visible keys
+ *   mask_kind  ATTN_MASK_*; window is read only for ATTN_MASK_SLIDING_WINDOW and
+ *              must then be >= 1 (window >= N behaves exactly as CAUSAL).
+ *   scale      the score scale, typically 1/sqrt(d); must be finite and > 0.
+ *   status     device int32 or NULL (bounded-wait timeout bit).
+ *
+ * Every row of every mask kind sees at least its own key, so no row is fully
+ * masked. Errors: ATTN_ERR_INVALID_ARG for non-positive sizes, Hq % Hkv != 0,
+ * NULL q/k/v/o, misaligned pointers, window < 1 with SLIDING_WINDOW, bad scale;
+ * ATTN_ERR_UNSUPPORTED for d not in {64, 128}; ATTN_ERR_CUDA on launch failure.
+ */
+ATTN_API int attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                 int N, int d, int mask_kind, int window, float scale, int32_t* status, attn_stream_t stream);
+
+/*
+ * attn_decode_plan - the split-KV plan attn_decode_paged uses (host only, no
+ * GPU needed). Long sequences are cut into chunks of *chunk_tokens tokens
+ * (a multiple of 16); each (sequence, K/V head, chunk) is one unit of work
+ * ("Inference attention" post, "FlashDecoding": split keys along the
+ * sequence so that small batches fill the GPU). num_sms is the device's SM
+ * count. Returns ATTN_OK or ATTN_ERR_INVALID_ARG.
+ */
+ATTN_API int attn_decode_plan(int B, int Hq, int Hkv, int max_seq_len, int num_sms, int* chunk_tokens, int* num_splits);
+
+/*
+ * attn_decode_workspace_bytes - bytes of device workspace attn_decode_paged
+ * needs for these sizes on the current device (partial outputs fp32
+ * [B, Hq, splits, d] plus partial log-sum-exp fp32 [B, Hq, splits]).
+ * Returns 0 for invalid sizes.
+ */
+ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int max_seq_len, int block_size);
+
+/*
+ * attn_decode_paged - one new query token per sequence against its whole
+ * cached context, read through a block table.
+ *
+ * Defined by "Module 09: Efficient Attention", "Code: A Paged KV Cache from
+ * Scratch": the pool has shape (num_blocks, block_size, num_kv_heads,
+ * head_dim) and token t of sequence b sits in slot t % block_size of physical
+ * block block_table[b][t / block_size]. The query attends to all seq_lens[b]
+ * cached tokens, its own K/V already appended ("USAAIO Lesson 90", part 2), so
+ * no mask applies. Split partials are merged with the online softmax's
+ * rescaling ("Inference attention" post, "FlashDecoding").
+ *
+ *   q            [B, Hq, d] bf16                            read
+ *   k_cache,
+ *   v_cache      [num_blocks, block_size, Hkv, d] bf16      read (only referenced slots)
+ *   block_table  [B, max_blocks_per_seq] int32              read: entries
+ *                0 .. ceil(seq_lens[b] / block_size) - 1 must lie in [0, num_blocks);
+ *                later entries are never read (may hold -1)
+ *   seq_lens     [B] int32, each in [1, max_seq_len]        read
+ *   o            [B, Hq, d] bf16                            written
+ *   lse          [B, Hq] fp32, natural log                  written when non-NULL
+ *   block_size   a multiple of 16 (the pages' default is 16)
+ *   max_seq_len  <= max_blocks_per_seq * block_size
+ *   workspace    device scratch of at least attn_decode_workspace_bytes(...)
+ *                bytes, 16-byte aligned; contents on entry are irrelevant.
+ *   status       device int32 or NULL.
+ *
+ * A referenced block-table entry outside [0, num_blocks) or a seq_len outside
+ * [1, max_seq_len] is never dereferenced: the affected rows of o and lse are
+ * NaN and ATTN_STATUS_BIT_DEVICE_CHECK is OR-ed into *status.
+ */
+ATTN_API int attn_decode_paged(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                      const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int d,
+                      int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, float scale,
+                      void* workspace, size_t workspace_bytes, int32_t* status, attn_stream_t stream);
+
+/*
+ * attn_paged_gather - walk every sequence's block table into a contiguous
+ * cache (the "gather" of "Module 09: Efficient Attention", "Code: A Paged KV
+ * Cache from Scratch"). Bit-exact copy; used to check block-table indexing.
+ *
+ *   cache        [num_blocks, block_size, Hkv, d] bf16       read
+ *   out          [B, Hkv, max_seq_len, d] bf16               written: token t of
+ *                sequence b for t < seq_lens[b], zero for the rest
+ *   block_table, seq_lens as for attn_decode_paged (seq_lens[b] may be 0 here).
+ * Invalid referenced entries: that token's row is NaN and the device-check
+ * bit is set.
+ */
+ATTN_API int attn_paged_gather(const void* cache, const int32_t* block_table, const int32_t* seq_lens, void* out, int B,
+                      int Hkv, int d, int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len,
+                      int32_t* status, attn_stream_t stream);
+
+/* attn_status_string - static English description of a status code. */
+ATTN_API const char* attn_status_string(int status);
+
+/* attn_version - library version, major * 10000 + minor * 100 + patch. */
+ATTN_API int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

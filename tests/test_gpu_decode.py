@@ -1,0 +1,184 @@
+"""GPU parity of attn_decode_paged and attn_paged_gather against the fp64
+oracle (through the C ABI)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_softmax_attention_causal_b200 import decode_paged, paged_gather, prefill, workloads
+from parity import assert_parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _to_cuda(x):
+    return (x.q.cuda(), x.k_cache.cuda(), x.v_cache.cuda(), x.block_table.cuda(), x.seq_lens.cuda())
+
+
+def _poison_unreferenced(x):
+    """NaN into every pool slot no sequence references (whole unreferenced
+    blocks and the slots past seq_len in each last block)."""
+    used = torch.zeros(x.k_cache.shape[:2], dtype=torch.bool)
+    for b, n in enumerate(x.seq_lens.tolist()):
+        for t in range(n):
+            used[int(x.block_table[b, t // x.block_size]), t % x.block_size] = True
+    nan = torch.tensor(float("nan"), dtype=torch.bfloat16)
+    x.k_cache[~used] = nan
+    x.v_cache[~used] = nan
+    return x
+
+
+def _check(x, heads=None, seqs=None, poison=True, what=""):
+    if poison:
+        x = _poison_unreferenced(x)
+    q, kc, vc, bt, sl = _to_cuda(x)
+    d = q.shape[-1]
+    scale = 1.0 / math.sqrt(d)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = decode_paged(q, kc, vc, bt, sl, x.max_seq_len, scale=scale, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    o, lse = o.cpu(), lse.cpu()
+    Hq = q.shape[1]
+    seqs = range(q.shape[0]) if seqs is None else seqs
+    heads = range(Hq) if heads is None else heads
+    for b in seqs:
+        o_ref, l_ref = oracle.decode_rows_ref(x.q, x.k_cache, x.v_cache, x.block_table, x.seq_lens, b, heads, scale)
+        assert_parity(o[b, list(heads)], o_ref, lse[b, list(heads)], l_ref, what=f"{what} seq {b}")
+    return o, lse
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_small_mixed_lengths(d):
+    x = workloads.paged_decode_inputs(4, 8, 2, d, seq_lens=[1, 17, 300, 4096], block_size=16, seed=1,
+                                      extra_blocks=5)
+    _check(x, what=f"d={d}")
+
+
+@pytest.mark.parametrize("hq,hkv", [(32, 32), (32, 1), (20, 1), (4, 4), (48, 2)])
+def test_head_groups(hq, hkv):
+    x = workloads.paged_decode_inputs(2, hq, hkv, 128, seq_lens=[33, 2500], block_size=16, seed=2,
+                                      extra_blocks=3)
+    _check(x, what=f"{hq}/{hkv}")
+
+
+@pytest.mark.parametrize("bs", [32, 64])
+def test_block_sizes(bs):
+    x = workloads.paged_decode_inputs(3, 8, 1, 128, seq_lens=[5, 1000, 777], block_size=bs, seed=3,
+                                      extra_blocks=2)
+    _check(x, what=f"bs={bs}")
+
+
+def test_long_single_sequence_many_splits():
+    x = workloads.paged_decode_inputs(1, 8, 2, 128, seq_lens=[20000], block_size=16, seed=4)
+    _check(x, poison=False)
+
+
+def test_permutation_invariance():
+    x = workloads.paged_decode_inputs(2, 8, 2, 128, seq_lens=[900, 64], block_size=16, seed=5)
+    q, kc, vc, bt, sl = _to_cuda(x)
+    o1, l1 = decode_paged(q, kc, vc, bt, sl, x.max_seq_len)
+    # move every block to a new physical slot and rewrite the table
+    perm = torch.randperm(kc.shape[0], generator=torch.Generator().manual_seed(9)).cuda()
+    kc2 = torch.empty_like(kc)
+    vc2 = torch.empty_like(vc)
+    kc2[perm] = kc
+    vc2[perm] = vc
+    bt2 = torch.where(bt >= 0, perm[bt.clamp(min=0).long()].int(), bt)
+    o2, l2 = decode_paged(q, kc2, vc2, bt2, sl, x.max_seq_len)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_gather_bit_exact():
+    x = workloads.paged_decode_inputs(3, 4, 2, 128, seq_lens=[1, 40, 333], block_size=16, seed=6, extra_blocks=4)
+    out = paged_gather(x.k_cache.cuda(), x.block_table.cuda(), x.seq_lens.cuda(), x.max_seq_len).cpu()
+    ref = oracle.gather_paged_ref(x.k_cache, x.block_table, x.seq_lens, x.max_seq_len)
+    assert torch.equal(out.double(), torch.from_numpy(ref))
+
+
+def test_gather_bit_exact_decode_workload_shape():
+    cfg = workloads.DECODE_WORKLOADS["paged_decode_b64"]
+    x = workloads.paged_decode_inputs(8, 4, 8, 128, len_range=(1, 4096), block_size=16, seed=7)
+    out = paged_gather(x.v_cache.cuda(), x.block_table.cuda(), x.seq_lens.cuda(), x.max_seq_len).cpu()
+    ref = oracle.gather_paged_ref(x.v_cache, x.block_table, x.seq_lens, x.max_seq_len)
+    assert torch.equal(out.double(), torch.from_numpy(ref))
+    assert cfg["block_size"] == 16
+
+
+def test_invalid_block_table_entry_is_flagged_not_read():
+    x = workloads.paged_decode_inputs(3, 8, 2, 128, seq_lens=[100, 200, 50], block_size=16, seed=8)
+    x.block_table[1, 3] = x.k_cache.shape[0] + 1000  # referenced (200 tokens use 13 blocks)
+    q, kc, vc, bt, sl = _to_cuda(x)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = decode_paged(q, kc, vc, bt, sl, x.max_seq_len, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & 0x1
+    assert torch.isnan(o[1].float()).all() and torch.isnan(lse[1]).all()
+    scale = 1 / math.sqrt(128)
+    for b in (0, 2):
+        o_ref, l_ref = oracle.decode_rows_ref(x.q, x.k_cache, x.v_cache, x.block_table, x.seq_lens, b, range(8),
+                                              scale)
+        assert_parity(o[b].cpu(), o_ref, lse[b].cpu(), l_ref)
+    # the gather flags the same entry and NaNs that token's rows
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g = paged_gather(kc, bt, sl, x.max_seq_len, status=st2)
+    torch.cuda.synchronize()
+    assert int(st2.item()) & 0x1
+    assert torch.isnan(g[1, :, 48:64].float()).all() and not torch.isnan(g[0].float()).any()
+
+
+@pytest.mark.parametrize("bad_len", [0, -3, 10 ** 6])
+def test_invalid_seq_len_is_flagged(bad_len):
+    x = workloads.paged_decode_inputs(2, 4, 2, 128, seq_lens=[64, 64], block_size=16, seed=9)
+    x.seq_lens[0] = bad_len
+    q, kc, vc, bt, sl = _to_cuda(x)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = decode_paged(q, kc, vc, bt, sl, 64, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & 0x1
+    assert torch.isnan(o[0].float()).all()
+    assert torch.isfinite(o[1].float()).all()
+
+
+def test_decode_equals_prefill_last_row():
+    """Cached decoding equals the full forward pass ("Module 09", the GQA cache
+    demonstration): decode at context t == row t-1 of causal prefill."""
+    B, Hq, Hkv, N, d = 1, 8, 2, 777, 128
+    xp = workloads.prefill_inputs(B, Hq, Hkv, N, d, 10)
+    q, k, v = (t.cuda() for t in (xp.q, xp.k, xp.v))
+    o_pf, lse_pf = prefill(q, k, v, mask="causal")
+    bs = 16
+    nblk = -(-N // bs)
+    perm = torch.randperm(nblk, generator=torch.Generator().manual_seed(3))
+    kc = torch.zeros((nblk, bs, Hkv, d), dtype=torch.bfloat16)
+    vc = torch.zeros_like(kc)
+    kt = xp.k[0].transpose(0, 1)  # [N, Hkv, d]
+    vt = xp.v[0].transpose(0, 1)
+    for lb in range(nblk):
+        n = min(bs, N - lb * bs)
+        kc[perm[lb], :n] = kt[lb * bs: lb * bs + n]
+        vc[perm[lb], :n] = vt[lb * bs: lb * bs + n]
+    table = perm.int()[None, :].cuda()
+    for t in (1, 16, 17, 500, N):
+        o_d, l_d = decode_paged(q[:, :, t - 1].contiguous(), kc.cuda(), vc.cuda(), table,
+                                torch.tensor([t], dtype=torch.int32, device="cuda"), N)
+        assert_parity(o_d[0].cpu(), o_pf[0, :, t - 1].cpu(), l_d[0].cpu(), lse_pf[0, :, t - 1].cpu(),
+                      what=f"t={t}")
+
+
+# --------------------------------------------------------------------------
+# full-size workloads, sampled sequences and heads
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("name", ["paged_decode_b64", "gqa_dial_decode_mha", "gqa_dial_decode_gqa8",
+                                  "gqa_dial_decode_mqa"])
+def test_full_size_sampled(name):
+    cfg = dict(workloads.DECODE_WORKLOADS[name])
+    B, Hq, Hkv, d = cfg.pop("B"), cfg.pop("Hq"), cfg.pop("Hkv"), cfg.pop("d")
+    x = workloads.paged_decode_inputs(B, Hq, Hkv, d, seed=0, **cfg)
+    rng = np.random.default_rng(1)
+    seqs = sorted(set([0, B - 1] + rng.integers(0, B, 3).tolist()))
+    heads = sorted(set([0, Hq - 1] + rng.integers(0, Hq, 4).tolist()))
+    _check(x, heads=heads, seqs=seqs, poison=False, what=name)
