@@ -1,0 +1,410 @@
+"""Benchmark of the attention hot path on B200: one JSON line on rank 0.
+
+A step is one pass of the hot path over one batch of synthetic inputs:
+causal GQA prefill of the Llama-3-8B-shaped batch (B=4, Hq=32, Hkv=8,
+N=4096, d=128) followed by one paged decode step of 64 sequences (context
+uniform in [1024, 32768], Hq=32, Hkv=8, d=128, 16-token blocks). The headline
+`value` is the prefill's TFLOP/s (causal FLOPs: only visible pairs count);
+the decode's KV GB/s sits under "decode". Inputs are resident in HBM before
+the timed region; L2 is flushed (a 256 MiB write) before every timed kernel.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own
+independent batch (weak scaling, no collective on the data path); the time
+is the max over ranks and `value` counts the work of all ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_softmax_attention_causal_b200 import accounting, workloads  # noqa: E402
+
+METRIC = "prefill causal-GQA TFLOP/s & paged-decode KV GB/s, % of B200 peak"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------
+# environment
+# ----------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return {"hbm_gbs": float(m["hbm_gbs"]), "bf16_tflops": float(m["bf16_tflops"]),
+                "bf16_tflops_sustained": float(m.get("bf16_tflops_sustained", m["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        loaded = [s for s in sm if mx is None or s >= 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def kernel_source_hash(name: str) -> str:
+    path = os.path.join(ROOT, "exact_softmax_attention_causal_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, source: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_sha256_16") != kernel_source_hash(source):
+        return None
+    return rec.get("bytes_per_launch")
+
+
+def oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+# ----------------------------------------------------------------------------
+# the fp64 CPU oracle, timed on the host cores (cpu_baseline and --impl reference)
+# ----------------------------------------------------------------------------
+def oracle_prefill_heads(x, cfg, heads, budget_s=None):
+    """Run the oracle over whole (batch, head) slices of the prefill workload.
+
+    Returns (flops, seconds, heads_done). Stops early once budget_s is spent
+    (at least one head always runs).
+    """
+    import oracle  # the oracle is only ever loaded by the baseline legs
+
+    B, Hq, N, d = cfg["B"], cfg["Hq"], cfg["N"], cfg["d"]
+    kind = accounting.MASK_IDS[cfg["mask"]]
+    per_head = 4 * d * accounting.visible_pairs(N, cfg["mask"], cfg["window"])
+    scale = workloads.default_scale(d)
+    rows = range(N)
+    done = 0
+    t0 = time.perf_counter()
+    for i in range(heads):
+        bh = (i * 37) % (B * Hq)  # spread the sample over batches and heads
+        oracle.prefill_rows_ref(x.q, x.k, x.v, bh // Hq, bh % Hq, rows, kind, cfg["window"], scale)
+        done += 1
+        if budget_s is not None and time.perf_counter() - t0 >= budget_s:
+            break
+    return per_head * done, time.perf_counter() - t0, done
+
+
+def cpu_baseline(x, cfg, budget_s):
+    flops, secs, done = oracle_prefill_heads(x, cfg, heads=cfg["B"] * cfg["Hq"], budget_s=budget_s)
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{done} of {cfg['B'] * cfg['Hq']} (batch, head) slices of the {cfg['name']} prefill, "
+                      f"all {cfg['N']} rows each, fp64 NumPy, {secs:.1f} s"}
+
+
+def run_reference(args, cfg):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0  # the oracle arm runs once, on rank 0
+    x = workloads.prefill_inputs(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["N"], cfg["d"], args.seed)
+    heads_per_step = args.reference_heads
+    for _ in range(args.warmup):
+        oracle_prefill_heads(x, cfg, heads_per_step)
+    flops = 0
+    secs = 0.0
+    for _ in range(args.steps):
+        f, s, _ = oracle_prefill_heads(x, cfg, heads_per_step)
+        flops += f
+        secs += s
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(cfg, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+                         "sample": f"{heads_per_step} (batch, head) slices of the {cfg['name']} prefill per step, "
+                                   f"all {cfg['N']} rows each"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(cfg, n_gpus):
+    return {"workload": cfg["name"], "B": cfg["B"], "Hq": cfg["Hq"], "Hkv": cfg["Hkv"], "N": cfg["N"],
+            "d": cfg["d"], "mask": cfg["mask"], "window": cfg["window"], "global_batch": cfg["B"] * n_gpus,
+            "seq_len": cfg["N"], "parallelism": f"independent batch per GPU x{n_gpus}",
+            "l2": "flushed (256 MiB write) before every timed kernel"}
+
+# ----------------------------------------------------------------------------
+# the CUDA path
+# ----------------------------------------------------------------------------
+def run_ours(args, pcfg, dcfg):
+    import exact_softmax_attention_causal_b200 as attn
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+    seed = args.seed + 1000 * rank  # every rank owns an independent batch
+
+    B, Hq, Hkv, N, d = pcfg["B"], pcfg["Hq"], pcfg["Hkv"], pcfg["N"], pcfg["d"]
+    xp = workloads.prefill_inputs(B, Hq, Hkv, N, d, seed)
+    q, k, v = xp.q.to(dev), xp.k.to(dev), xp.v.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    p_flops = accounting.prefill_flops(B, Hq, N, d, pcfg["mask"], pcfg["window"])
+
+    dB, dHq, dHkv, dd = dcfg["B"], dcfg["Hq"], dcfg["Hkv"], dcfg["d"]
+    xd = workloads.paged_decode_inputs(dB, dHq, dHkv, dd, len_range=dcfg.get("len_range"),
+                                       seq_lens=dcfg.get("seq_lens"), block_size=dcfg["block_size"], seed=seed)
+    dq, kc, vc = xd.q.to(dev), xd.k_cache.to(dev), xd.v_cache.to(dev)
+    bt, sl = xd.block_table.to(dev), xd.seq_lens.to(dev)
+    dout = torch.empty_like(dq)
+    dlse = torch.empty((dB, dHq), dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.decode_workspace_bytes(dB, dHq, dHkv, dd, xd.max_seq_len, xd.block_size),
+                     dtype=torch.uint8, device=dev)
+    kv_bytes = accounting.decode_kv_bytes(xd.seq_lens.tolist(), dHkv, dd)
+    del xd
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        flush.fill_(1)
+        if ev:
+            ev[0].record()
+        attn.prefill(q, k, v, mask=pcfg["mask"], window=pcfg["window"], out=o, lse=lse)
+        if ev:
+            ev[1].record()
+        flush.fill_(2)
+        if ev:
+            ev[2].record()
+        attn.decode_paged(dq, kc, vc, bt, sl, dcfg_max_len(dcfg), out=dout, lse=dlse, workspace=ws)
+        if ev:
+            ev[3].record()
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    region = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    with ClockSampler(local) as clk:
+        for _ in range(args.warmup):
+            step()
+        barrier()
+        region[0].record()
+        for i in range(args.steps):
+            step(events[i])
+        region[1].record()
+        barrier()
+    p_ms = sum(e[0].elapsed_time(e[1]) for e in events)
+    d_ms = sum(e[2].elapsed_time(e[3]) for e in events)
+    region_ms = region[0].elapsed_time(region[1])
+
+    # end to end through the public API: pinned host inputs in, O and LSE back out, every step
+    hq, hk, hv = xp.q.pin_memory(), xp.k.pin_memory(), xp.v.pin_memory()
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    e2e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    barrier()
+    e2e_ev[0].record()
+    for _ in range(args.steps):
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        attn.prefill(q, k, v, mask=pcfg["mask"], window=pcfg["window"], out=o, lse=lse)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+    e2e_ev[1].record()
+    barrier()
+    e2e_ms = e2e_ev[0].elapsed_time(e2e_ev[1])
+
+    times = torch.tensor([p_ms, d_ms, region_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    p_ms, d_ms, region_ms, e2e_ms = times.tolist()
+
+    result = None
+    if rank == 0:
+        K = args.steps
+        peaks = measured_peaks()
+        tag = "of measured" if peaks["source"] == "measured" else "of fallback"
+        p_avg_s = p_ms / K / 1e3
+        d_avg_s = d_ms / K / 1e3
+        p_tflops_launch = p_flops / p_avg_s / 1e12
+        d_gbs_launch = kv_bytes / d_avg_s / 1e9
+        result = {
+            "metric": METRIC,
+            "value": p_flops * K * world / (p_ms / 1e3) / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": (p_ms + d_ms) / K,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": config_block(pcfg, world),
+            "roofline": {"bound": "tensor", "achieved": p_tflops_launch, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": p_tflops_launch / peaks["bf16_tflops"],
+                         "traffic": recorded_traffic("prefill_fwd_kernel", "prefill_sm100.cu"),
+                         "peak_source": f"bf16_tflops (burst) {tag}",
+                         "kernel": "prefill_fwd_kernel<128>", "flops_per_launch": p_flops},
+            "e2e": {"value": p_flops * K * world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 3 * K,
+            "clocks": clk.summary(),
+            "decode": {
+                "metric": "paged-decode KV GB/s", "value": kv_bytes * K * world / (d_ms / 1e3) / 1e9,
+                "unit": "GB/s", "workload": dcfg["name"], "kv_bytes_per_step": kv_bytes, "ms_per_step": d_ms / K,
+                "roofline": {"bound": "hbm", "achieved": d_gbs_launch, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": d_gbs_launch / peaks["hbm_gbs"],
+                             "traffic": recorded_traffic("decode_split_kernel", "decode_sm100.cu"),
+                             "peak_source": f"hbm_gbs {tag}",
+                             "kernel": "decode_split_kernel<128> + decode_merge_kernel<128>"},
+            },
+            "region_ms": region_ms,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(xp, pcfg, args.cpu_seconds)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if result is not None:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def dcfg_max_len(dcfg):
+    if dcfg.get("len_range") is not None:
+        return int(dcfg["len_range"][1])
+    return int(max(dcfg["seq_lens"]))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama3_8b_causal_gqa", choices=sorted(workloads.PREFILL_WORKLOADS))
+    ap.add_argument("--decode-workload", default="paged_decode_b64", choices=sorted(workloads.DECODE_WORKLOADS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--reference-heads", type=int, default=2, help="oracle (batch, head) slices per step")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    pcfg = dict(workloads.PREFILL_WORKLOADS[args.workload], name=args.workload)
+    dcfg = dict(workloads.DECODE_WORKLOADS[args.decode_workload], name=args.decode_workload)
+    world, _, _ = dist_env()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.impl == "reference":
+        return run_reference(args, pcfg)
+    return run_ours(args, pcfg, dcfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
