@@ -18,6 +18,7 @@ SYMBOLS = (
     "attn_decode_plan",
     "attn_decode_workspace_bytes",
     "attn_decode_paged",
+    "attn_decode_paged_noalloc",
     "attn_paged_gather",
     "attn_status_string",
     "attn_version",
@@ -30,6 +31,7 @@ ATTN_ERR_CUDA = -3
 ATTN_ERR_DEVICE_CHECK = -4
 ATTN_ERR_TIMEOUT = -5
 ATTN_ERR_WORKSPACE = -6
+DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
 STATUS_BIT_DEVICE_CHECK = 0x1
 STATUS_BIT_TIMEOUT = 0x2
 
@@ -52,6 +54,9 @@ def _declare(lib):
     lib.attn_decode_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp,
                                       _sz, _vp, _vp]
     lib.attn_decode_paged.restype = _i
+    lib.attn_decode_paged_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
+                                              _vp, _vp]
+    lib.attn_decode_paged_noalloc.restype = _i
     lib.attn_paged_gather.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]
     lib.attn_paged_gather.restype = _i
     lib.attn_status_string.argtypes = [_i]

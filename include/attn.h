@@ -168,6 +168,39 @@ ATTN_API int attn_paged_gather(const void* cache, const int32_t* block_table, co
                       int Hkv, int d, int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len,
                       int32_t* status, attn_stream_t stream);
 
+/*
+ * attn_decode_paged_noalloc - attn_decode_paged for callers that cannot
+ * allocate device memory. No passage of the pages corresponds to it; it
+ * exists for the library's users.
+ *
+ * Some callers cannot call cudaMalloc or hand the library a workspace: code
+ * living inside a host framework that owns every device byte through its own
+ * allocator, or a latency-critical loop that must not pay for an allocation
+ * (which may synchronise the device) on the decode path. This variant takes
+ * the same arguments as attn_decode_paged minus workspace/workspace_bytes and
+ * keeps the split partials in a static device array of
+ * ATTN_DECODE_NOALLOC_SCRATCH_BYTES bytes that the library holds on every GPU
+ * it is loaded on until the process exits. It calls no allocating routine.
+ *
+ *   - Requests whose split workspace (attn_decode_workspace_bytes) exceeds
+ *     ATTN_DECODE_NOALLOC_SCRATCH_BYTES are rejected with ATTN_ERR_WORKSPACE
+ *     before anything is launched.
+ *   - The first call on each device looks up that device's address of the
+ *     array (a set-up step, done once per device with the device current);
+ *     make that first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind. Nothing in it has to start at zero: each call writes every
+ *     partial it later reads. Calls whose kernels overlap on the GPU (two
+ *     streams, or two host threads) race on the array: serialise them.
+ * Outputs, errors and device checks are exactly those of attn_decode_paged.
+ */
+#define ATTN_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20) /* 32 MiB */
+ATTN_API int attn_decode_paged_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                       const int32_t* block_table, const int32_t* seq_lens, void* o, float* lse,
+                                       int B, int Hq, int Hkv, int d, int num_blocks, int block_size,
+                                       int max_blocks_per_seq, int max_seq_len, float scale, int32_t* status,
+                                       attn_stream_t stream);
+
 /* attn_status_string - static English description of a status code. */
 ATTN_API const char* attn_status_string(int status);
 
