@@ -132,8 +132,10 @@ def kernel_source_hash(name: str) -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str, source: str):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged since."""
+def recorded_traffic(kernel: str, source: str, kv_bytes: int | None = None):
+    """DRAM bytes per launch from a committed ncu capture (profiles/traffic.json),
+    or None once the kernel source has changed since the counters were taken.
+    A capture of a smaller case is scaled to this launch by its KV bytes."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -142,7 +144,11 @@ def recorded_traffic(kernel: str, source: str):
         return None
     if not rec or rec.get("source_sha256_16") != kernel_source_hash(source):
         return None
-    return rec.get("bytes_per_launch")
+    if "bytes_per_launch" in rec:
+        return rec["bytes_per_launch"]
+    if "bytes_per_kv_byte" in rec and kv_bytes is not None:
+        return int(rec["bytes_per_kv_byte"] * kv_bytes)
+    return None
 
 
 def oracle_threads() -> int:
@@ -359,7 +365,7 @@ def run_ours(args, pcfg, dcfg):
                 "unit": "GB/s", "workload": dcfg["name"], "kv_bytes_per_step": kv_bytes, "ms_per_step": d_ms / K,
                 "roofline": {"bound": "hbm", "achieved": d_gbs_launch, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                              "frac": d_gbs_launch / peaks["hbm_gbs"],
-                             "traffic": recorded_traffic("decode_split_kernel", "decode_sm100.cu"),
+                             "traffic": recorded_traffic("decode_split_kernel", "decode_sm100.cu", kv_bytes),
                              "peak_source": f"hbm_gbs {tag}",
                              "kernel": "decode_split_kernel<128> + decode_merge_kernel<128>"},
             },
