@@ -13,18 +13,24 @@
 // of the window are never visited; only the tiles that straddle a mask edge
 // evaluate the mask per element.
 //
-// Roles (192 threads, one CTA per SM):
-//   warps 0-3  softmax: thread i owns query row i = TMEM lane i. Reads a
-//              128-column score row from TMEM, applies scale (folded with
-//              log2 e) and mask, updates the running max and sum, writes the
-//              probabilities back to TMEM as bf16 and, when needed, rescales
-//              the output accumulator in TMEM; finally O / l -> bf16 and LSE.
-//   warp 4     TMA producer: Q once, then K and V tiles into a ring of
-//              shared-memory stages (128-byte swizzle, 64-column boxes).
-//   warp 5     MMA issuer: S_j = Q K_j^T (both operands in shared memory) into
-//              one of two TMEM score buffers, and O += P_j V_j with P read
-//              straight from TMEM. Allocates and frees the 512 TMEM columns.
-// The score MMA of tile j+1 runs while the softmax works on tile j.
+// Roles (320 threads, one CTA per SM, two 128-row query tiles A and B of the
+// same head, so every K/V tile is loaded once for 256 query rows):
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread i owns
+//              query row i of its tile = TMEM lane i. Reads the 128-column
+//              score row from TMEM, applies scale (folded with log2 e) and,
+//              on edge tiles only, the mask; updates the running max and sum;
+//              rescales its output row in TMEM when the max moved; writes the
+//              probabilities back as bf16 over the consumed score columns;
+//              finally O / l -> bf16 and LSE.
+//   warp 8     TMA producer: both Q tiles once, then K and V tiles into a ring
+//              of shared-memory stages (128-byte swizzle, 64-column boxes).
+//   warp 9     MMA issuer: S_X = Q_X K_j^T (both operands in shared memory) and
+//              O_X += P_X V_j with P_X read straight from TMEM, alternating
+//              between the tiles so the tensor core works on one tile while
+//              the other tile's softmax runs. Allocates and frees TMEM.
+// A tile's score barrier is committed after its previous P.V, so when the
+// softmax sees new scores its output accumulator is stable and may be
+// rescaled in place.
 //
 // Lazy rescaling: the running max used for the exponentials only moves when
 // the true running max exceeds it by more than 8 (base 2). Every p stays
@@ -53,7 +59,20 @@ namespace {
 
 constexpr int kBM = 128;  // query rows per tile (= TMEM lanes)
 constexpr int kBN = 128;  // keys per tile
-constexpr int kPfThreads = 192;
+constexpr int kTilesPerCta = 2;
+constexpr int kRowsPerCta = kTilesPerCta * kBM;
+constexpr int kPfThreads = 384;  // 8 softmax warps + a warpgroup holding the TMA and MMA warps
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+// Register split (per thread): launched with 168 (65536 / 384, rounded down to
+// a multiple of 8 and capped by the 16K-register sub-partition holding three
+// warps); the TMA/MMA warpgroup gives registers back, the softmax warpgroups
+// take them: 256 x 208 + 128 x 88 = 384 x 168 = 64512.
+constexpr uint32_t kRegsLaunch = 168;
+constexpr uint32_t kRegsSoftmax = 208;
+constexpr uint32_t kRegsControl = 88;
+static_assert(256 * kRegsSoftmax + 128 * kRegsControl == kPfThreads * kRegsLaunch, "register split");
+static_assert(2 * kRegsSoftmax * 32 + kRegsControl * 32 <= 16384, "per sub-partition register file");
 constexpr float kRescaleThreshold = 8.0f;
 
 template <int D>
@@ -62,34 +81,33 @@ struct PfCfg {
   static constexpr int kHalves = D / 64;     // 128-byte swizzle columns per tile
   static constexpr int kTile = kHalves * kHalf;
   static constexpr int kStages = (D == 128) ? 2 : 4;
-  static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kTile;
+  static constexpr int kQOff = 0;            // Q tile A, then Q tile B
+  static constexpr int kKOff = kQOff + kTilesPerCta * kTile;
   static constexpr int kVOff = kKOff + kStages * kTile;
   static constexpr int kBarOff = kVOff + kStages * kTile;
   static constexpr int kBytes = kBarOff + 256;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
-  // TMEM column map (512 columns allocated)
-  static constexpr uint32_t kColS0 = 0;
-  static constexpr uint32_t kColS1 = 128;
-  static constexpr uint32_t kColO = 256;
-  static constexpr uint32_t kColP = 384;  // 128 bf16 probabilities = 64 columns
+  // TMEM columns (512 allocated): scores of A and B (128 fp32 columns each;
+  // the bf16 probabilities overwrite their first 64 columns), then outputs.
+  __host__ __device__ static constexpr uint32_t col_s(int x) { return x ? 128u : 0u; }
+  __host__ __device__ static constexpr uint32_t col_o(int x) { return 256u + static_cast<uint32_t>(x * D); }
 };
 
 // Barrier slots inside the barrier block (8 bytes each).
 enum : int {
   kBarQFull = 0,
-  kBarKFull = 1,   // + stage (up to 4)
-  kBarVFull = 5,   // + stage
-  kBarKEmpty = 9,  // + stage
-  kBarVEmpty = 13, // + stage
-  kBarSFull = 17,  // + buffer (2)
-  kBarPFull = 19,
-  kBarODone = 20,
-  kBarDrain = 21,
-  kNumBars = 22,
+  kBarKFull = 1,    // + stage (up to 4)
+  kBarVFull = 5,    // + stage
+  kBarKEmpty = 9,   // + stage
+  kBarVEmpty = 13,  // + stage
+  kBarSFull = 17,   // + tile (2)
+  kBarPFull = 19,   // + tile
+  kBarOFinal = 21,  // + tile
+  kBarDrain = 23,
+  kNumBars = 24,
 };
-constexpr int kTmemSlotOff = 192;
-constexpr int kAbortOff = 196;
+constexpr int kTmemSlotOff = 200;
+constexpr int kAbortOff = 204;
 
 // Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format: start
 // address, leading and stride byte offsets in 16-byte units, version 1,
@@ -111,37 +129,36 @@ struct PrefillParams {
   __nv_bfloat16* o;
   float* lse;
   int32_t* status;
-  int B, Hq, Hkv, N, group, mask_kind, window, num_q_tiles;
+  int B, Hq, Hkv, N, group, mask_kind, window, num_cta_tiles;
   float scale_log2;
   long long budget;
 };
 
-// Key tiles a query tile visits: [lo, hi], inclusive.
+// Key tiles the 256 query rows [q0, q0 + 256) visit: [lo, hi], inclusive.
 __device__ __forceinline__ void kv_tile_range(const PrefillParams& p, int q0, int& lo, int& hi) {
   hi = (p.N - 1) / kBN;
   lo = 0;
-  if (p.mask_kind != ATTN_MASK_FULL) hi = min(hi, (q0 + kBM - 1) / kBN);
+  if (p.mask_kind != ATTN_MASK_FULL) hi = min(hi, (q0 + kRowsPerCta - 1) / kBN);
   if (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) lo = max(0, q0 - p.window + 1) / kBN;
 }
 
-// True when every (row, key) pair of the tile is visible, so no per-element mask is needed.
-__device__ __forceinline__ bool tile_is_full(const PrefillParams& p, int q0, int k0) {
+// True when every (row, key) pair of a 128 x 128 tile is visible.
+__device__ __forceinline__ bool tile_is_full(const PrefillParams& p, int qr0, int k0) {
   bool full = (k0 + kBN <= p.N);
-  if (p.mask_kind != ATTN_MASK_FULL) full = full && (k0 + kBN - 1 <= q0);
-  if (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) full = full && (q0 + kBM - 1 - k0 < p.window);
+  if (p.mask_kind != ATTN_MASK_FULL) full = full && (k0 + kBN - 1 <= qr0);
+  if (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) full = full && (qr0 + kBM - 1 - k0 < p.window);
   return full;
-}
-
-__device__ __forceinline__ bool key_visible(const PrefillParams& p, int qi, int kj) {
-  if (kj >= p.N) return false;
-  if (p.mask_kind == ATTN_MASK_FULL) return true;
-  if (kj > qi) return false;
-  return p.mask_kind != ATTN_MASK_SLIDING_WINDOW || (qi - kj < p.window);
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int32_t* status) {
   *abort_flag = 1;
   if (status != nullptr) atomicOr(status, ATTN_STATUS_BIT_TIMEOUT);
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 template <int D>
@@ -159,8 +176,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int h = blockIdx.x;
   const int b = blockIdx.y;
   // heaviest query tiles first when the mask makes work grow with the tile index
-  const int qt = (p.mask_kind == ATTN_MASK_FULL) ? blockIdx.z : (p.num_q_tiles - 1 - blockIdx.z);
-  const int q0 = qt * kBM;
+  const int ct = (p.mask_kind == ATTN_MASK_FULL) ? blockIdx.z : (p.num_cta_tiles - 1 - blockIdx.z);
+  const int q0 = ct * kRowsPerCta;
   const int kvh = h / p.group;
   int kt_lo, kt_hi;
   kv_tile_range(p, q0, kt_lo, kt_hi);
@@ -179,15 +196,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(bar(kBarKEmpty + s), 1);
       mbar_init(bar(kBarVEmpty + s), 1);
     }
-    mbar_init(bar(kBarSFull + 0), 1);
-    mbar_init(bar(kBarSFull + 1), 1);
-    mbar_init(bar(kBarPFull), kBM);
-    mbar_init(bar(kBarODone), 1);
+    for (int x = 0; x < kTilesPerCta; ++x) {
+      mbar_init(bar(kBarSFull + x), 1);
+      mbar_init(bar(kBarPFull + x), kBM);
+      mbar_init(bar(kBarOFinal + x), 1);
+    }
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -197,18 +215,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const long long budget = p.budget;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+  if (warp >= kTmaWarp) {
+    regs_dec<kRegsControl>();
+    if (warp == kTmaWarp && lane == 0) {
+      // ---------------------------------------------------------- TMA producer
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       const int zq = b * p.Hq + h;
       const int zkv = b * p.Hkv + kvh;
-      mbar_arrive_expect_tx(bar(kBarQFull), C::kTile);
-      for (int hh = 0; hh < C::kHalves; ++hh)
-        tma_load_3d(sbase + C::kQOff + hh * C::kHalf, &tm_q, bar(kBarQFull), hh * 64, q0, zq);
-      // K_i is issued before V_{i-1}: the score MMA needs K one tile earlier than PV needs V.
+      mbar_arrive_expect_tx(bar(kBarQFull), kTilesPerCta * C::kTile);
+      for (int x = 0; x < kTilesPerCta; ++x)
+        for (int hh = 0; hh < C::kHalves; ++hh)
+          tma_load_3d(sbase + C::kQOff + x * C::kTile + hh * C::kHalf, &tm_q, bar(kBarQFull), hh * 64,
+                      q0 + x * kBM, zq);
+      // K_i is issued before V_{i-1}: the score MMA needs K one tile earlier than P.V needs V.
       int k_issued = 0, v_issued = 0;
       bool ok = true;
       for (int i = 0; i <= T && ok; ++i) {
@@ -218,11 +239,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             ok = false;
             break;
           }
-          const int k0 = (kt_lo + i) * kBN;
           mbar_arrive_expect_tx(bar(kBarKFull + s), C::kTile);
           for (int hh = 0; hh < C::kHalves; ++hh)
-            tma_load_3d(sbase + C::kKOff + s * C::kTile + hh * C::kHalf, &tm_k, bar(kBarKFull + s), hh * 64, k0,
-                        zkv);
+            tma_load_3d(sbase + C::kKOff + s * C::kTile + hh * C::kHalf, &tm_k, bar(kBarKFull + s), hh * 64,
+                        (kt_lo + i) * kBN, zkv);
           k_issued = i + 1;
         }
         if (i >= 1) {
@@ -232,11 +252,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             ok = false;
             break;
           }
-          const int k0 = (kt_lo + jv) * kBN;
           mbar_arrive_expect_tx(bar(kBarVFull + s), C::kTile);
           for (int hh = 0; hh < C::kHalves; ++hh)
-            tma_load_3d(sbase + C::kVOff + s * C::kTile + hh * C::kHalf, &tm_v, bar(kBarVFull + s), hh * 64, k0,
-                        zkv);
+            tma_load_3d(sbase + C::kVOff + s * C::kTile + hh * C::kHalf, &tm_v, bar(kBarVFull + s), hh * 64,
+                        (kt_lo + jv) * kBN, zkv);
           v_issued = jv + 1;
         }
       }
@@ -248,52 +267,72 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         mbar_wait_bounded(bar(kBarKFull + j % C::kStages), (j / C::kStages) & 1, kDrainBudgetCycles, &never);
       for (int j = (v_issued > C::kStages ? v_issued - C::kStages : 0); j < v_issued; ++j)
         mbar_wait_bounded(bar(kBarVFull + j % C::kStages), (j / C::kStages) & 1, kDrainBudgetCycles, &never);
-    }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == kMmaWarp && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_qk = idesc_bf16(kBM, kBN, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(kBM, D, 1);
-      const uint32_t sQ = sbase + C::kQOff;
-      bool ok = mbar_wait_bounded(bar(kBarQFull), 0, budget, abort_flag);
-      auto issue_s = [&](int j) -> bool {
-        const int s = j % C::kStages;
-        if (!mbar_wait_bounded(bar(kBarKFull + s), (j / C::kStages) & 1, budget, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t sK = sbase + C::kKOff + s * C::kTile;
-        const uint32_t d_col = tmem + ((j & 1) ? C::kColS1 : C::kColS0);
+      // S_x = Q_x K_j^T into tile x's score columns
+      auto issue_s = [&](int x, int j) {
+        const uint32_t sQ = sbase + C::kQOff + x * C::kTile;
+        const uint32_t sK = sbase + C::kKOff + (j % C::kStages) * C::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * C::kHalf + (kk & 3) * 32;
-          tc_mma_ss(d_col, desc_sw128(sQ + koff, 16, 1024), desc_sw128(sK + koff, 16, 1024), idesc_qk,
-                    kk > 0 ? 1u : 0u);
+          tc_mma_ss(tmem + C::col_s(x), desc_sw128(sQ + koff, 16, 1024), desc_sw128(sK + koff, 16, 1024),
+                    idesc_qk, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(kBarSFull + (j & 1)));
-        tc_commit(bar(kBarKEmpty + s));
-        return true;
+        tc_commit(bar(kBarSFull + x));
       };
-      if (ok) ok = issue_s(0);
+      // O_x (+)= P_x V_j, P_x in the first 64 score columns (16 keys = 8 columns per step)
+      auto issue_pv = [&](int x, int j) {
+        const uint32_t sV = sbase + C::kVOff + (j % C::kStages) * C::kTile;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          tc_mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8, desc_sw128(sV + kk * 2048, C::kHalf, 1024),
+                    idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait_bounded(bar(kBarQFull), 0, budget, abort_flag) &&
+                mbar_wait_bounded(bar(kBarKFull), 0, budget, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        tc_commit(bar(kBarKEmpty));
+      }
       for (int j = 0; j < T && ok; ++j) {
-        if (j + 1 < T && !issue_s(j + 1)) {
-          ok = false;
-          break;
-        }
         const int s = j % C::kStages;
-        if (!mbar_wait_bounded(bar(kBarPFull), j & 1, budget, abort_flag) ||
+        const int jn = j + 1;
+        // tile A: P.V of tile j, then the scores of tile j + 1 (in issue order, so the
+        // new scores overwrite P only after P.V has read it)
+        if (!mbar_wait_bounded(bar(kBarPFull + 0), j & 1, budget, abort_flag) ||
             !mbar_wait_bounded(bar(kBarVFull + s), (j / C::kStages) & 1, budget, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t sV = sbase + C::kVOff + s * C::kTile;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          // 16 keys per step: P columns [8 kk, 8 kk + 8), V rows [16 kk, 16 kk + 16)
-          tc_mma_ts(tmem + C::kColO, tmem + C::kColP + kk * 8, desc_sw128(sV + kk * 2048, C::kHalf, 1024), idesc_pv,
-                    (j > 0 || kk > 0) ? 1u : 0u);
+        issue_pv(0, j);
+        if (j == T - 1) tc_commit(bar(kBarOFinal + 0));
+        if (jn < T) {
+          if (!mbar_wait_bounded(bar(kBarKFull + jn % C::kStages), (jn / C::kStages) & 1, budget, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_s(0, jn);
         }
-        tc_commit(bar(kBarODone));
+        // tile B
+        if (!mbar_wait_bounded(bar(kBarPFull + 1), j & 1, budget, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv(1, j);
+        if (j == T - 1) tc_commit(bar(kBarOFinal + 1));
         tc_commit(bar(kBarVEmpty + s));
+        if (jn < T) {
+          issue_s(1, jn);
+          tc_commit(bar(kBarKEmpty + jn % C::kStages));
+        }
       }
       if (!ok) raise_abort(abort_flag, p.status);
       // Drain: every MMA this thread issued has completed before TMEM is freed.
@@ -302,35 +341,51 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_wait_bounded(bar(kBarDrain), 0, kDrainBudgetCycles, &never);
     }
   } else {
-    // ------------------------------------------------------------ softmax warps 0-3
-    const int r = threadIdx.x;  // tile row = TMEM lane
-    const int qi = q0 + r;      // query position
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    float m_used = -INFINITY;   // max the exponentials are taken against (base 2)
-    float l_sum = 0.f;          // running sum of 2^(x - m_used), fp32
+    regs_inc<kRegsSoftmax>();
+    // ------------------------------------------------------------ softmax warps 0-7
+    const int x = warp >> 2;                  // query tile A (0) or B (1)
+    const int r = threadIdx.x & (kBM - 1);    // row of the tile = TMEM lane
+    const int qr0 = q0 + x * kBM;             // first query position of the tile
+    const int qi = qr0 + r;                   // this thread's query position
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t colS = lane_base + C::col_s(x);
+    const uint32_t colO = lane_base + C::col_o(x);
+    const float sl2 = p.scale_log2;
+    float m_used = -INFINITY;  // max the exponentials are taken against (base 2)
+    float l_sum = 0.f;         // running sum of 2^(x - m_used), fp32
     bool ok = true;
     for (int j = 0; j < T; ++j) {
       const int k0 = (kt_lo + j) * kBN;
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBarSFull + (j & 1)), (j >> 1) & 1, budget, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBarSFull + x), j & 1, budget, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[kBN];
-      const uint32_t scol = lane_base + ((j & 1) ? C::kColS1 : C::kColS0);
+      uint32_t raw[kBN];
 #pragma unroll
       for (int c = 0; c < kBN / 32; ++c)
-        tmem_ld_32x32b_x32(scol + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        tmem_ld_32x32b_x32(colS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&raw[c * 32]));
       tc_wait_ld();
-
-      const bool full = tile_is_full(p, q0, k0);
-      float mt = -INFINITY;
+      float sv[kBN];
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        float x = __uint_as_float(sr[c]) * p.scale_log2;
-        if (!full && !key_visible(p, qi, k0 + c)) x = -INFINITY;
-        sr[c] = __float_as_uint(x);
-        mt = fmaxf(mt, x);
+      for (int c = 0; c < kBN; ++c) sv[c] = __uint_as_float(raw[c]);
+
+      if (!tile_is_full(p, qr0, k0)) {
+        // edge tile: visible keys of this row are columns [cmin, cmax]
+        int cmax = p.N - 1 - k0;
+        if (p.mask_kind != ATTN_MASK_FULL) cmax = min(cmax, qi - k0);
+        const int cmin = (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) ? qi - k0 - p.window + 1 : 0;
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) sv[c] = (c >= cmin && c <= cmax) ? sv[c] : -INFINITY;
       }
-      const float m_new = fmaxf(m_used, mt);
+      // row max of the raw scores (scale > 0 commutes with max): four independent chains
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kBN; c += 8) {
+        mx0 = max3f(mx0, sv[c], sv[c + 1]);
+        mx1 = max3f(mx1, sv[c + 2], sv[c + 3]);
+        mx2 = max3f(mx2, sv[c + 4], sv[c + 5]);
+        mx3 = max3f(mx3, sv[c + 6], sv[c + 7]);
+      }
+      const float m_new = fmaxf(m_used, max3f(mx0, mx1, fmaxf(mx2, mx3)) * sl2);
       bool rescale_o = false;
       float factor = 1.f;
       if (m_new > m_used + kRescaleThreshold) {  // also true for the first visible key (m_used = -inf)
@@ -340,43 +395,47 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         rescale_o = prev_finite;  // earlier tiles already put visible keys into O
         m_used = m_new;
       }
-      if (j > 0) {  // PV_{j-1} done: O is stable and the P buffer is free
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBarODone), (j - 1) & 1, budget, abort_flag));
-        if (!ok) break;
-      }
-      tc_fence_after();
+      // The score barrier was committed after this tile's previous P.V: O is stable.
       if (__any_sync(0xffffffffu, rescale_o)) {
         const float f = rescale_o ? factor : 1.f;
 #pragma unroll
         for (int c = 0; c < D / 16; ++c) {
           uint32_t ov[16];
-          tmem_ld_32x32b_x16(lane_base + C::kColO + c * 16, ov);
+          tmem_ld_32x32b_x16(colO + c * 16, ov);
           tc_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-          tmem_st_32x32b_x16(lane_base + C::kColO + c * 16, ov);
+          tmem_st_32x32b_x16(colO + c * 16, ov);
         }
       }
-      const float mref = (m_used == -INFINITY) ? 0.f : m_used;  // a row with nothing visible yet gets p = 0
-      float rs = 0.f;
+      // p = 2^(s * scale * log2 e - m): one FFMA and one ex2 per score; a row with
+      // nothing visible yet (m_used = -inf) uses 0, so its masked scores give p = 0.
+      const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
+      float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
 #pragma unroll
       for (int cc = 0; cc < kBN / 32; ++cc) {
         uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = fast_exp2(__uint_as_float(sr[cc * 32 + 2 * e]) - mref);
-          const float p1 = fast_exp2(__uint_as_float(sr[cc * 32 + 2 * e + 1]) - mref);
-          rs += p0 + p1;
+        for (int e = 0; e < 16; e += 2) {
+          const float p0 = fast_exp2(fmaf(sv[cc * 32 + 2 * e], sl2, neg_m));
+          const float p1 = fast_exp2(fmaf(sv[cc * 32 + 2 * e + 1], sl2, neg_m));
+          const float p2 = fast_exp2(fmaf(sv[cc * 32 + 2 * e + 2], sl2, neg_m));
+          const float p3 = fast_exp2(fmaf(sv[cc * 32 + 2 * e + 3], sl2, neg_m));
+          rs0 += p0;
+          rs1 += p1;
+          rs2 += p2;
+          rs3 += p3;
           pk[e] = pack_bf16x2(p0, p1);
+          pk[e + 1] = pack_bf16x2(p2, p3);
         }
-        tmem_st_32x32b_x16(lane_base + C::kColP + cc * 16, pk);
+        tmem_st_32x32b_x16(colS + cc * 16, pk);  // over score columns already consumed
       }
       tc_wait_st();
-      l_sum += rs;
+      l_sum += (rs0 + rs1) + (rs2 + rs3);
       tc_fence_before();
-      mbar_arrive(bar(kBarPFull));
+      mbar_arrive(bar(kBarPFull + x));
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBarODone), (T - 1) & 1, budget, abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBarOFinal + x), 0, budget, abort_flag));
     if (!ok) raise_abort(abort_flag, p.status);
     tc_fence_after();
 
@@ -388,7 +447,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     for (int c = 0; c < D / 32; ++c) {
       uint32_t ov[32];
       if (ok) {
-        tmem_ld_32x32b_x32(lane_base + C::kColO + c * 32, ov);
+        tmem_ld_32x32b_x32(colO + c * 32, ov);
         tc_wait_ld();
       }
       uint4 pk[4];
@@ -411,7 +470,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -464,13 +523,13 @@ int launch_prefill_t(const void* q, const void* k, const void* v, void* o, float
   p.group = Hq / Hkv;
   p.mask_kind = mask_kind;
   p.window = window;
-  p.num_q_tiles = (N + kBM - 1) / kBM;
+  p.num_cta_tiles = (N + kRowsPerCta - 1) / kRowsPerCta;
   p.scale_log2 = scale * kLog2e;
   p.budget = wait_budget_cycles();
   constexpr int smem = PfCfg<D>::kAlloc;
   if (cudaFuncSetAttribute(prefill_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  const dim3 grid(Hq, B, p.num_q_tiles);
+  const dim3 grid(Hq, B, p.num_cta_tiles);
   prefill_fwd_kernel<D><<<grid, kPfThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
