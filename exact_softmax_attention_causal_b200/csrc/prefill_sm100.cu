@@ -67,7 +67,7 @@ constexpr int kMmaWarp = 9;
 // Register split (per thread): launched with 168 (65536 / 384, rounded down to
 // a multiple of 8 and capped by the 16K-register sub-partition holding three
 // warps); the TMA/MMA warpgroup gives registers back, the softmax warpgroups
-// take them: 256 x 208 + 128 x 88 = 384 x 168 = 64512.
+// take them: 256 x 232 + 128 x 40 = 384 x 168 = 64512.
 constexpr uint32_t kRegsLaunch = 168;
 constexpr uint32_t kRegsSoftmax = 208;
 constexpr uint32_t kRegsControl = 88;
@@ -101,13 +101,14 @@ enum : int {
   kBarKEmpty = 9,   // + stage
   kBarVEmpty = 13,  // + stage
   kBarSFull = 17,   // + tile (2)
-  kBarPFull = 19,   // + tile
-  kBarOFinal = 21,  // + tile
-  kBarDrain = 23,
-  kNumBars = 24,
+  kBarPLo = 19,     // + tile: probabilities of keys 0-63 written
+  kBarPHi = 21,     // + tile: probabilities of keys 64-127 written
+  kBarOFinal = 23,  // + tile
+  kBarDrain = 25,
+  kNumBars = 26,
 };
-constexpr int kTmemSlotOff = 200;
-constexpr int kAbortOff = 204;
+constexpr int kTmemSlotOff = 224;
+constexpr int kAbortOff = 228;
 
 // Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format: start
 // address, leading and stride byte offsets in 16-byte units, version 1,
@@ -155,6 +156,50 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int32_t* s
   if (status != nullptr) atomicOr(status, ATTN_STATUS_BIT_TIMEOUT);
 }
 
+// 2^x for a pair of x on the FMA pipes instead of the special-function unit:
+// x = n + f with n = round(x) (added to the exponent field) and f in
+// [-1/2, 1/2]; 2^f by a degree-4 polynomial whose maximum relative error on
+// that interval is minimised (Remez exchange, fitted by fit_exp2_poly.py next
+// to this file: 2.7e-6 in float32). x is clamped to >= -126 so the result
+// stays a positive number below 2^-125 where the true value is smaller.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);
+  float2 p = ffma2(make_float2(0.009570102207362652f, 0.009570102207362652f), f,
+                   make_float2(0.05591785907745361f, 0.05591785907745361f));
+  p = ffma2(p, f, make_float2(0.240247443318367f, 0.240247443318367f));
+  p = ffma2(p, f, make_float2(0.6931217908859253f, 0.6931217908859253f));
+  p = ffma2(p, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
+  // the low mantissa bits of t hold n; shifting by 23 moves n into the exponent
+  const uint32_t r0 = __float_as_uint(p.x) + (__float_as_uint(t.x) << 23);
+  const uint32_t r1 = __float_as_uint(p.y) + (__float_as_uint(t.y) << 23);
+  return make_float2(__uint_as_float(r0), __uint_as_float(r1));
+}
+
+// Column pairs (of every 8) whose exponentials run on the FMA pipes: bit e set
+// = pair e uses exp2_poly2, the others use the special-function unit.
+constexpr uint32_t kPolyPairs = 0x00;
+// Scale-and-shift and the running sums with paired fp32 instructions.
+constexpr bool kPairedFma = true;
+
+// Multiply this thread's TMEM output row by f (warp-collective).
+template <int D>
+__device__ __forceinline__ void rescale_row_t(uint32_t colO, float f) {
+#pragma unroll
+  for (int c = 0; c < D / 16; ++c) {
+    uint32_t ov[16];
+    tmem_ld_32x32b_x16(colO + c * 16, ov);
+    tc_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+    tmem_st_32x32b_x16(colO + c * 16, ov);
+  }
+}
+
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -198,7 +243,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     for (int x = 0; x < kTilesPerCta; ++x) {
       mbar_init(bar(kBarSFull + x), 1);
-      mbar_init(bar(kBarPFull + x), kBM);
+      mbar_init(bar(kBarPLo + x), kBM);
+      mbar_init(bar(kBarPHi + x), kBM);
       mbar_init(bar(kBarOFinal + x), 1);
     }
     mbar_init(bar(kBarDrain), 1);
@@ -283,13 +329,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         tc_commit(bar(kBarSFull + x));
       };
-      // O_x (+)= P_x V_j, P_x in the first 64 score columns (16 keys = 8 columns per step)
-      auto issue_pv = [&](int x, int j) {
+      // O_x (+)= P_x V_j for keys [64 half, 64 half + 64); P_x sits in the first 64
+      // score columns (16 keys = 8 columns per MMA step)
+      auto issue_pv = [&](int x, int j, int half) {
         const uint32_t sV = sbase + C::kVOff + (j % C::kStages) * C::kTile;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
+        for (int kk = half * 4; kk < half * 4 + 4; ++kk)
           tc_mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8, desc_sw128(sV + kk * 2048, C::kHalf, 1024),
                     idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      // wait for one half of tile x's probabilities, then multiply that half by V
+      auto pv_half = [&](int x, int j, int half) -> bool {
+        if (!mbar_wait_bounded(bar((half ? kBarPHi : kBarPLo) + x), j & 1, budget, abort_flag)) return false;
+        tc_fence_after();
+        issue_pv(x, j, half);
+        return true;
       };
       bool ok = mbar_wait_bounded(bar(kBarQFull), 0, budget, abort_flag) &&
                 mbar_wait_bounded(bar(kBarKFull), 0, budget, abort_flag);
@@ -302,15 +356,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int j = 0; j < T && ok; ++j) {
         const int s = j % C::kStages;
         const int jn = j + 1;
-        // tile A: P.V of tile j, then the scores of tile j + 1 (in issue order, so the
-        // new scores overwrite P only after P.V has read it)
-        if (!mbar_wait_bounded(bar(kBarPFull + 0), j & 1, budget, abort_flag) ||
-            !mbar_wait_bounded(bar(kBarVFull + s), (j / C::kStages) & 1, budget, abort_flag)) {
+        // tile A: P.V of tile j (as each half of P lands), then the scores of tile
+        // j + 1 (in issue order, so the new scores overwrite P only after P.V read it)
+        if (!mbar_wait_bounded(bar(kBarVFull + s), (j / C::kStages) & 1, budget, abort_flag) ||
+            !pv_half(0, j, 0) || !pv_half(0, j, 1)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        issue_pv(0, j);
         if (j == T - 1) tc_commit(bar(kBarOFinal + 0));
         if (jn < T) {
           if (!mbar_wait_bounded(bar(kBarKFull + jn % C::kStages), (jn / C::kStages) & 1, budget, abort_flag)) {
@@ -321,12 +373,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           issue_s(0, jn);
         }
         // tile B
-        if (!mbar_wait_bounded(bar(kBarPFull + 1), j & 1, budget, abort_flag)) {
+        if (!pv_half(1, j, 0) || !pv_half(1, j, 1)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        issue_pv(1, j);
         if (j == T - 1) tc_commit(bar(kBarOFinal + 1));
         tc_commit(bar(kBarVEmpty + s));
         if (jn < T) {
@@ -351,6 +401,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t colS = lane_base + C::col_s(x);
     const uint32_t colO = lane_base + C::col_o(x);
     const float sl2 = p.scale_log2;
+    auto rescale_rows = [](uint32_t col, float f) { rescale_row_t<D>(col, f); };
     float m_used = -INFINITY;  // max the exponentials are taken against (base 2)
     float l_sum = 0.f;         // running sum of 2^(x - m_used), fp32
     bool ok = true;
@@ -396,44 +447,50 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         m_used = m_new;
       }
       // The score barrier was committed after this tile's previous P.V: O is stable.
-      if (__any_sync(0xffffffffu, rescale_o)) {
-        const float f = rescale_o ? factor : 1.f;
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          uint32_t ov[16];
-          tmem_ld_32x32b_x16(colO + c * 16, ov);
-          tc_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-          tmem_st_32x32b_x16(colO + c * 16, ov);
-        }
-      }
-      // p = 2^(s * scale * log2 e - m): one FFMA and one ex2 per score; a row with
-      // nothing visible yet (m_used = -inf) uses 0, so its masked scores give p = 0.
+      if (__any_sync(0xffffffffu, rescale_o)) rescale_rows(colO, rescale_o ? factor : 1.f);
+
+      // p = 2^(s * scale * log2 e - m); a row with nothing visible yet uses m = 0.
+      // P goes out in two halves, each announced on its own barrier, so the MMA
+      // warp starts P.V on keys 0-63 while keys 64-127 are still being exponentiated.
       const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-      float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
 #pragma unroll
       for (int cc = 0; cc < kBN / 32; ++cc) {
         uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const float p0 = fast_exp2(fmaf(sv[cc * 32 + 2 * e], sl2, neg_m));
-          const float p1 = fast_exp2(fmaf(sv[cc * 32 + 2 * e + 1], sl2, neg_m));
-          const float p2 = fast_exp2(fmaf(sv[cc * 32 + 2 * e + 2], sl2, neg_m));
-          const float p3 = fast_exp2(fmaf(sv[cc * 32 + 2 * e + 3], sl2, neg_m));
-          rs0 += p0;
-          rs1 += p1;
-          rs2 += p2;
-          rs3 += p3;
-          pk[e] = pack_bf16x2(p0, p1);
-          pk[e + 1] = pack_bf16x2(p2, p3);
+        for (int e = 0; e < 16; ++e) {
+          const int c = cc * 32 + 2 * e;
+          float2 xv;
+          if (kPairedFma) {
+            xv = ffma2(make_float2(sv[c], sv[c + 1]), make_float2(sl2, sl2), make_float2(neg_m, neg_m));
+          } else {
+            xv.x = fmaf(sv[c], sl2, neg_m);
+            xv.y = fmaf(sv[c + 1], sl2, neg_m);
+          }
+          float2 pv;
+          if ((kPolyPairs >> (e & 7)) & 1) {
+            pv = exp2_poly2(xv);
+          } else {
+            pv.x = fast_exp2(xv.x);
+            pv.y = fast_exp2(xv.y);
+          }
+          float2& acc = (e & 3) == 0 ? acc0 : (e & 3) == 1 ? acc1 : (e & 3) == 2 ? acc2 : acc3;
+          if (kPairedFma) {
+            acc = fadd2(acc, pv);
+          } else {
+            acc.x += pv.x;
+            acc.y += pv.y;
+          }
+          pk[e] = pack_bf16x2(pv.x, pv.y);
         }
         tmem_st_32x32b_x16(colS + cc * 16, pk);  // over score columns already consumed
+        if (cc == 1 || cc == 3) {
+          tc_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar((cc == 1 ? kBarPLo : kBarPHi) + x));
+        }
       }
-      tc_wait_st();
-      l_sum += (rs0 + rs1) + (rs2 + rs3);
-      tc_fence_before();
-      mbar_arrive(bar(kBarPFull + x));
+      l_sum += ((acc0.x + acc0.y) + (acc1.x + acc1.y)) + ((acc2.x + acc2.y) + (acc3.x + acc3.y));
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBarOFinal + x), 0, budget, abort_flag));
     if (!ok) raise_abort(abort_flag, p.status);
