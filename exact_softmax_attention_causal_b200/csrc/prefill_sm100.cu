@@ -7,27 +7,35 @@
 // and LSE = log sum_j exp(scale * q_i . k_j) over the visible keys.
 //
 // How: FlashAttention's online softmax (section 8 of the same page; the
-// "Inference attention" post, section "FlashAttention"): one CTA owns a
-// 128-row query tile of one (batch, head) and streams 128-key tiles of K and
-// V, never writing scores to HBM. Tiles entirely above the diagonal or left
-// of the window are never visited; only the tiles that straddle a mask edge
-// evaluate the mask per element.
+// "Inference attention" post, section "FlashAttention"), never writing scores
+// to HBM. A work item is 256 query rows (two 128-row tiles A and B) of one
+// (batch, head); it streams 128-key tiles of K and V, each loaded once for
+// both tiles. Key tiles entirely above the diagonal or left of the window are
+// never visited; only tiles that straddle a mask edge evaluate the mask per
+// element.
 //
-// Roles (320 threads, one CTA per SM, two 128-row query tiles A and B of the
-// same head, so every K/V tile is loaded once for 256 query rows):
+// Persistent schedule: one CTA per SM walks a share of the items, heaviest
+// first, handed out in snake order so the per-CTA totals stay even. Across
+// items the K/V ring keeps streaming, the next item's Q loads as soon as the
+// current item's last score MMA has read Q, and its first score MMAs overlap
+// the current item's epilogue.
+//
+// Roles (384 threads):
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread i owns
 //              query row i of its tile = TMEM lane i. Reads the 128-column
 //              score row from TMEM, applies scale (folded with log2 e) and,
 //              on edge tiles only, the mask; updates the running max and sum;
 //              rescales its output row in TMEM when the max moved; writes the
-//              probabilities back as bf16 over the consumed score columns;
-//              finally O / l -> bf16 and LSE.
-//   warp 8     TMA producer: both Q tiles once, then K and V tiles into a ring
-//              of shared-memory stages (128-byte swizzle, 64-column boxes).
+//              probabilities back as bf16 over the consumed score columns, in
+//              two halves each announced on its own barrier; finally
+//              O / l -> bf16 and LSE.
+//   warp 8     TMA producer: both Q tiles per item, then K and V tiles into a
+//              ring of shared-memory stages (128-byte swizzle, 64-column boxes).
 //   warp 9     MMA issuer: S_X = Q_X K_j^T (both operands in shared memory) and
 //              O_X += P_X V_j with P_X read straight from TMEM, alternating
 //              between the tiles so the tensor core works on one tile while
 //              the other tile's softmax runs. Allocates and frees TMEM.
+//   warps 10-11 idle (they complete the register-donating warpgroup).
 // A tile's score barrier is committed after its previous P.V, so when the
 // softmax sees new scores its output accumulator is stable and may be
 // rescaled in place.
@@ -39,8 +47,8 @@
 // skipping most rescales, as the "Inference attention" post describes it).
 //
 // All pipeline waits are bounded; on expiry the CTA records
-// ATTN_STATUS_BIT_TIMEOUT, writes NaN rows, drains its copies and MMAs
-// (bounded again), frees TMEM and exits.
+// ATTN_STATUS_BIT_TIMEOUT, writes NaN rows for every item it has left, drains
+// its copies and MMAs (bounded again), frees TMEM and exits.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -67,7 +75,7 @@ constexpr int kMmaWarp = 9;
 // Register split (per thread): launched with 168 (65536 / 384, rounded down to
 // a multiple of 8 and capped by the 16K-register sub-partition holding three
 // warps); the TMA/MMA warpgroup gives registers back, the softmax warpgroups
-// take them: 256 x 232 + 128 x 40 = 384 x 168 = 64512.
+// take them: 256 x 208 + 128 x 88 = 384 x 168 = 64512.
 constexpr uint32_t kRegsLaunch = 168;
 constexpr uint32_t kRegsSoftmax = 208;
 constexpr uint32_t kRegsControl = 88;
@@ -105,7 +113,8 @@ enum : int {
   kBarPHi = 21,     // + tile: probabilities of keys 64-127 written
   kBarOFinal = 23,  // + tile
   kBarDrain = 25,
-  kNumBars = 26,
+  kBarQEmpty = 26,  // both Q tiles consumed by the item's last score MMA
+  kNumBars = 27,
 };
 constexpr int kTmemSlotOff = 224;
 constexpr int kAbortOff = 228;
@@ -131,9 +140,30 @@ struct PrefillParams {
   float* lse;
   int32_t* status;
   int B, Hq, Hkv, N, group, mask_kind, window, num_cta_tiles;
+  int num_items;  // num_cta_tiles * Hq * B
   float scale_log2;
   long long budget;
 };
+
+// One work item: 256 query rows of one (batch, head). Items are numbered
+// heaviest first (for causal and window masks the work of a row tile grows
+// with its index), heads of a K/V group adjacent so concurrently running CTAs
+// share K/V tiles in L2.
+struct WorkItem {
+  int q0, h, b;
+};
+__device__ __forceinline__ WorkItem item_at(const PrefillParams& p, int w) {
+  const int per = p.Hq * p.B;
+  const int rank = w / per;
+  const int rem = w - rank * per;
+  const int ct = (p.mask_kind == ATTN_MASK_FULL) ? rank : (p.num_cta_tiles - 1 - rank);
+  return WorkItem{ct * kRowsPerCta, rem % p.Hq, rem / p.Hq};
+}
+// Snake assignment of the heaviest-first list over the persistent CTAs:
+// round r hands item r * G + c (r even) or r * G + G - 1 - c (r odd) to CTA c.
+__device__ __forceinline__ int item_index(int round, int c, int G) {
+  return round * G + ((round & 1) ? (G - 1 - c) : c);
+}
 
 // Key tiles the 256 query rows [q0, q0 + 256) visit: [lo, hi], inclusive.
 __device__ __forceinline__ void kv_tile_range(const PrefillParams& p, int q0, int& lo, int& hi) {
@@ -206,6 +236,9 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
+// Persistent: one CTA per SM walks its share of the work items. Barrier phases
+// run on across items: K/V stages and score/probability barriers count key
+// tiles (g), Q and final-output barriers count items (it).
 template <int D>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -218,15 +251,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int h = blockIdx.x;
-  const int b = blockIdx.y;
-  // heaviest query tiles first when the mask makes work grow with the tile index
-  const int ct = (p.mask_kind == ATTN_MASK_FULL) ? blockIdx.z : (p.num_cta_tiles - 1 - blockIdx.z);
-  const int q0 = ct * kRowsPerCta;
-  const int kvh = h / p.group;
-  int kt_lo, kt_hi;
-  kv_tile_range(p, q0, kt_lo, kt_hi);
-  const int T = kt_hi - kt_lo + 1;
+  const int cta = blockIdx.x;
+  const int G = gridDim.x;
 
   const uint32_t bars = sbase + C::kBarOff;
   auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
@@ -235,6 +261,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQFull), 1);
+    mbar_init(bar(kBarQEmpty), 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
       mbar_init(bar(kBarVFull + s), 1);
@@ -268,47 +295,62 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      const int zq = b * p.Hq + h;
-      const int zkv = b * p.Hkv + kvh;
-      mbar_arrive_expect_tx(bar(kBarQFull), kTilesPerCta * C::kTile);
-      for (int x = 0; x < kTilesPerCta; ++x)
-        for (int hh = 0; hh < C::kHalves; ++hh)
-          tma_load_3d(sbase + C::kQOff + x * C::kTile + hh * C::kHalf, &tm_q, bar(kBarQFull), hh * 64,
-                      q0 + x * kBM, zq);
-      // K_i is issued before V_{i-1}: the score MMA needs K one tile earlier than P.V needs V.
-      int k_issued = 0, v_issued = 0;
+      int g = 0;             // key tiles issued before this item (K and V alike)
+      int k_issued = 0, v_issued = 0, it = 0;
       bool ok = true;
-      for (int i = 0; i <= T && ok; ++i) {
-        if (i < T) {
-          const int s = i % C::kStages, round = i / C::kStages;
-          if (round > 0 && !mbar_wait_bounded(bar(kBarKEmpty + s), (round - 1) & 1, budget, abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar(kBarKFull + s), C::kTile);
-          for (int hh = 0; hh < C::kHalves; ++hh)
-            tma_load_3d(sbase + C::kKOff + s * C::kTile + hh * C::kHalf, &tm_k, bar(kBarKFull + s), hh * 64,
-                        (kt_lo + i) * kBN, zkv);
-          k_issued = i + 1;
+      for (int round = 0; ok; ++round) {
+        const int w = item_index(round, cta, G);
+        if (w >= p.num_items) break;
+        const WorkItem wi = item_at(p, w);
+        int kt_lo, kt_hi;
+        kv_tile_range(p, wi.q0, kt_lo, kt_hi);
+        const int T = kt_hi - kt_lo + 1;
+        const int zq = wi.b * p.Hq + wi.h;
+        const int zkv = wi.b * p.Hkv + wi.h / p.group;
+        // Q of this item once the previous item's last score MMA has read its Q
+        if (it > 0 && !mbar_wait_bounded(bar(kBarQEmpty), (it - 1) & 1, budget, abort_flag)) {
+          ok = false;
+          break;
         }
-        if (i >= 1) {
-          const int jv = i - 1;
-          const int s = jv % C::kStages, round = jv / C::kStages;
-          if (round > 0 && !mbar_wait_bounded(bar(kBarVEmpty + s), (round - 1) & 1, budget, abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar(kBarVFull + s), C::kTile);
+        mbar_arrive_expect_tx(bar(kBarQFull), kTilesPerCta * C::kTile);
+        for (int x = 0; x < kTilesPerCta; ++x)
           for (int hh = 0; hh < C::kHalves; ++hh)
-            tma_load_3d(sbase + C::kVOff + s * C::kTile + hh * C::kHalf, &tm_v, bar(kBarVFull + s), hh * 64,
-                        (kt_lo + jv) * kBN, zkv);
-          v_issued = jv + 1;
+            tma_load_3d(sbase + C::kQOff + x * C::kTile + hh * C::kHalf, &tm_q, bar(kBarQFull), hh * 64,
+                        wi.q0 + x * kBM, zq);
+        // K_i is issued before V_{i-1}: the score MMA needs K one tile earlier than P.V needs V.
+        for (int i = 0; i <= T; ++i) {
+          if (i < T) {
+            const int gi = g + i, s = gi % C::kStages, rnd = gi / C::kStages;
+            if (rnd > 0 && !mbar_wait_bounded(bar(kBarKEmpty + s), (rnd - 1) & 1, budget, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(kBarKFull + s), C::kTile);
+            for (int hh = 0; hh < C::kHalves; ++hh)
+              tma_load_3d(sbase + C::kKOff + s * C::kTile + hh * C::kHalf, &tm_k, bar(kBarKFull + s), hh * 64,
+                          (kt_lo + i) * kBN, zkv);
+            k_issued = gi + 1;
+          }
+          if (i >= 1) {
+            const int gv = g + i - 1, s = gv % C::kStages, rnd = gv / C::kStages;
+            if (rnd > 0 && !mbar_wait_bounded(bar(kBarVEmpty + s), (rnd - 1) & 1, budget, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(kBarVFull + s), C::kTile);
+            for (int hh = 0; hh < C::kHalves; ++hh)
+              tma_load_3d(sbase + C::kVOff + s * C::kTile + hh * C::kHalf, &tm_v, bar(kBarVFull + s), hh * 64,
+                          (kt_lo + i - 1) * kBN, zkv);
+            v_issued = gv + 1;
+          }
         }
+        g += T;
+        ++it;
       }
       if (!ok) raise_abort(abort_flag, p.status);
-      // Drain: the newest copy of every stage has landed before the CTA may exit.
+      // Drain: the newest copy of every stage and of Q has landed before the CTA may exit.
       volatile int never = 0;
-      mbar_wait_bounded(bar(kBarQFull), 0, kDrainBudgetCycles, &never);
+      if (it > 0) mbar_wait_bounded(bar(kBarQFull), (it - 1) & 1, kDrainBudgetCycles, &never);
       for (int j = (k_issued > C::kStages ? k_issued - C::kStages : 0); j < k_issued; ++j)
         mbar_wait_bounded(bar(kBarKFull + j % C::kStages), (j / C::kStages) & 1, kDrainBudgetCycles, &never);
       for (int j = (v_issued > C::kStages ? v_issued - C::kStages : 0); j < v_issued; ++j)
@@ -317,72 +359,89 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_qk = idesc_bf16(kBM, kBN, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(kBM, D, 1);
-      // S_x = Q_x K_j^T into tile x's score columns
-      auto issue_s = [&](int x, int j) {
-        const uint32_t sQ = sbase + C::kQOff + x * C::kTile;
-        const uint32_t sK = sbase + C::kKOff + (j % C::kStages) * C::kTile;
+      // Descriptors are built once; an operand at byte offset o from its base has
+      // descriptor base + o / 16 (the start address is the low field, and every
+      // tile lies below 256 KB, so the addition never carries out of it).
+      const uint64_t dq0 = desc_sw128(sbase + C::kQOff, 16, 1024);
+      const uint64_t dk0 = desc_sw128(sbase + C::kKOff, 16, 1024);
+      const uint64_t dv0 = desc_sw128(sbase + C::kVOff, C::kHalf, 1024);
+      constexpr uint64_t kTileUnits = C::kTile >> 4;
+      // S_x = Q_x K^T of global key tile g into tile x's score columns
+      auto issue_s = [&](int x, int g) {
+        const uint64_t dq = dq0 + static_cast<uint64_t>(x) * kTileUnits;
+        const uint64_t dk = dk0 + static_cast<uint64_t>(g % C::kStages) * kTileUnits;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * C::kHalf + (kk & 3) * 32;
-          tc_mma_ss(tmem + C::col_s(x), desc_sw128(sQ + koff, 16, 1024), desc_sw128(sK + koff, 16, 1024),
-                    idesc_qk, kk > 0 ? 1u : 0u);
+          const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * C::kHalf + (kk & 3) * 32) >> 4);
+          tc_mma_ss(tmem + C::col_s(x), dq + koff, dk + koff, idesc_qk, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar(kBarSFull + x));
       };
-      // O_x (+)= P_x V_j for keys [64 half, 64 half + 64); P_x sits in the first 64
-      // score columns (16 keys = 8 columns per MMA step)
-      auto issue_pv = [&](int x, int j, int half) {
-        const uint32_t sV = sbase + C::kVOff + (j % C::kStages) * C::kTile;
+      // O_x (+)= P_x V for keys [64 half, 64 half + 64) of global key tile g; P_x sits in
+      // the first 64 score columns (16 keys = 8 columns per MMA step); `first` starts O_x
+      auto pv_half = [&](int x, int g, int half, bool first) -> bool {
+        if (!mbar_wait_bounded(bar((half ? kBarPHi : kBarPLo) + x), g & 1, budget, abort_flag)) return false;
+        tc_fence_after();
+        const uint64_t dv = dv0 + static_cast<uint64_t>(g % C::kStages) * kTileUnits;
 #pragma unroll
         for (int kk = half * 4; kk < half * 4 + 4; ++kk)
-          tc_mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8, desc_sw128(sV + kk * 2048, C::kHalf, 1024),
-                    idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-      };
-      // wait for one half of tile x's probabilities, then multiply that half by V
-      auto pv_half = [&](int x, int j, int half) -> bool {
-        if (!mbar_wait_bounded(bar((half ? kBarPHi : kBarPLo) + x), j & 1, budget, abort_flag)) return false;
-        tc_fence_after();
-        issue_pv(x, j, half);
+          tc_mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4),
+                    idesc_pv, (!first || kk > 0) ? 1u : 0u);
         return true;
       };
-      bool ok = mbar_wait_bounded(bar(kBarQFull), 0, budget, abort_flag) &&
-                mbar_wait_bounded(bar(kBarKFull), 0, budget, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        tc_commit(bar(kBarKEmpty));
-      }
-      for (int j = 0; j < T && ok; ++j) {
-        const int s = j % C::kStages;
-        const int jn = j + 1;
-        // tile A: P.V of tile j (as each half of P lands), then the scores of tile
-        // j + 1 (in issue order, so the new scores overwrite P only after P.V read it)
-        if (!mbar_wait_bounded(bar(kBarVFull + s), (j / C::kStages) & 1, budget, abort_flag) ||
-            !pv_half(0, j, 0) || !pv_half(0, j, 1)) {
+      int g = 0, it = 0;
+      bool ok = true;
+      for (int round = 0; ok; ++round) {
+        const int w = item_index(round, cta, G);
+        if (w >= p.num_items) break;
+        const WorkItem wi = item_at(p, w);
+        int kt_lo, kt_hi;
+        kv_tile_range(p, wi.q0, kt_lo, kt_hi);
+        const int T = kt_hi - kt_lo + 1;
+        if (!mbar_wait_bounded(bar(kBarQFull), it & 1, budget, abort_flag) ||
+            !mbar_wait_bounded(bar(kBarKFull + g % C::kStages), (g / C::kStages) & 1, budget, abort_flag)) {
           ok = false;
           break;
         }
-        if (j == T - 1) tc_commit(bar(kBarOFinal + 0));
-        if (jn < T) {
-          if (!mbar_wait_bounded(bar(kBarKFull + jn % C::kStages), (jn / C::kStages) & 1, budget, abort_flag)) {
+        tc_fence_after();
+        issue_s(0, g);
+        issue_s(1, g);
+        tc_commit(bar(kBarKEmpty + g % C::kStages));
+        if (T == 1) tc_commit(bar(kBarQEmpty));
+        for (int j = 0; j < T; ++j) {
+          const int gj = g + j, gn = gj + 1;
+          const int s = gj % C::kStages;
+          // tile A: P.V of key tile j (as each half of P lands), then the scores of tile
+          // j + 1 (in issue order, so the new scores overwrite P only after P.V read it)
+          if (!mbar_wait_bounded(bar(kBarVFull + s), (gj / C::kStages) & 1, budget, abort_flag) ||
+              !pv_half(0, gj, 0, j == 0) || !pv_half(0, gj, 1, j == 0)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          issue_s(0, jn);
+          if (j == T - 1) tc_commit(bar(kBarOFinal + 0));
+          if (j + 1 < T) {
+            if (!mbar_wait_bounded(bar(kBarKFull + gn % C::kStages), (gn / C::kStages) & 1, budget, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(0, gn);
+          }
+          // tile B
+          if (!pv_half(1, gj, 0, j == 0) || !pv_half(1, gj, 1, j == 0)) {
+            ok = false;
+            break;
+          }
+          if (j == T - 1) tc_commit(bar(kBarOFinal + 1));
+          tc_commit(bar(kBarVEmpty + s));
+          if (j + 1 < T) {
+            issue_s(1, gn);
+            tc_commit(bar(kBarKEmpty + gn % C::kStages));
+            if (j + 2 == T) tc_commit(bar(kBarQEmpty));  // that was the item's last read of Q
+          }
         }
-        // tile B
-        if (!pv_half(1, j, 0) || !pv_half(1, j, 1)) {
-          ok = false;
-          break;
-        }
-        if (j == T - 1) tc_commit(bar(kBarOFinal + 1));
-        tc_commit(bar(kBarVEmpty + s));
-        if (jn < T) {
-          issue_s(1, jn);
-          tc_commit(bar(kBarKEmpty + jn % C::kStages));
-        }
+        g += T;
+        ++it;
       }
       if (!ok) raise_abort(abort_flag, p.status);
       // Drain: every MMA this thread issued has completed before TMEM is freed.
@@ -393,136 +452,152 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   } else {
     regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax warps 0-7
-    const int x = warp >> 2;                  // query tile A (0) or B (1)
-    const int r = threadIdx.x & (kBM - 1);    // row of the tile = TMEM lane
-    const int qr0 = q0 + x * kBM;             // first query position of the tile
-    const int qi = qr0 + r;                   // this thread's query position
+    const int x = warp >> 2;                // query tile A (0) or B (1)
+    const int r = threadIdx.x & (kBM - 1);  // row of the tile = TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t colS = lane_base + C::col_s(x);
     const uint32_t colO = lane_base + C::col_o(x);
     const float sl2 = p.scale_log2;
     auto rescale_rows = [](uint32_t col, float f) { rescale_row_t<D>(col, f); };
-    float m_used = -INFINITY;  // max the exponentials are taken against (base 2)
-    float l_sum = 0.f;         // running sum of 2^(x - m_used), fp32
+    int g = 0, it = 0;
     bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      const int k0 = (kt_lo + j) * kBN;
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBarSFull + x), j & 1, budget, abort_flag));
-      if (!ok) break;
+    for (int round = 0;; ++round) {
+      const int w = item_index(round, cta, G);
+      if (w >= p.num_items) break;
+      const WorkItem wi = item_at(p, w);
+      int kt_lo, kt_hi;
+      kv_tile_range(p, wi.q0, kt_lo, kt_hi);
+      const int T = kt_hi - kt_lo + 1;
+      const int qr0 = wi.q0 + x * kBM;  // first query position of the tile
+      const int qi = qr0 + r;           // this thread's query position
+      float m_used = -INFINITY;         // max the exponentials are taken against (base 2)
+      float l_sum = 0.f;                // running sum of 2^(x - m_used), fp32
+      for (int j = 0; j < T && ok; ++j) {
+        const int gj = g + j;
+        const int k0 = (kt_lo + j) * kBN;
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBarSFull + x), gj & 1, budget, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t raw[kBN];
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c)
+          tmem_ld_32x32b_x32(colS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&raw[c * 32]));
+        tc_wait_ld();
+        float sv[kBN];
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) sv[c] = __uint_as_float(raw[c]);
+
+        if (!tile_is_full(p, qr0, k0)) {
+          // edge tile: visible keys of this row are columns [cmin, cmax]
+          int cmax = p.N - 1 - k0;
+          if (p.mask_kind != ATTN_MASK_FULL) cmax = min(cmax, qi - k0);
+          const int cmin = (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) ? qi - k0 - p.window + 1 : 0;
+#pragma unroll
+          for (int c = 0; c < kBN; ++c) sv[c] = (c >= cmin && c <= cmax) ? sv[c] : -INFINITY;
+        }
+        // row max of the raw scores (scale > 0 commutes with max): four independent chains
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kBN; c += 8) {
+          mx0 = max3f(mx0, sv[c], sv[c + 1]);
+          mx1 = max3f(mx1, sv[c + 2], sv[c + 3]);
+          mx2 = max3f(mx2, sv[c + 4], sv[c + 5]);
+          mx3 = max3f(mx3, sv[c + 6], sv[c + 7]);
+        }
+        const float m_new = fmaxf(m_used, max3f(mx0, mx1, fmaxf(mx2, mx3)) * sl2);
+        bool rescale_o = false;
+        float factor = 1.f;
+        if (m_new > m_used + kRescaleThreshold) {  // also true for the first visible key (m_used = -inf)
+          const bool prev_finite = (m_used != -INFINITY);
+          factor = prev_finite ? fast_exp2(m_used - m_new) : 0.f;
+          l_sum *= factor;
+          rescale_o = prev_finite;  // earlier tiles already put visible keys into O
+          m_used = m_new;
+        }
+        // The score barrier was committed after this tile's previous P.V: O is stable.
+        if (__any_sync(0xffffffffu, rescale_o)) rescale_rows(colO, rescale_o ? factor : 1.f);
+
+        // p = 2^(s * scale * log2 e - m); a row with nothing visible yet uses m = 0.
+        // P goes out in two halves, each announced on its own barrier, so the MMA
+        // warp starts P.V on keys 0-63 while keys 64-127 are still being exponentiated.
+        const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
+#pragma unroll
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c = cc * 32 + 2 * e;
+            float2 xv;
+            if (kPairedFma) {
+              xv = ffma2(make_float2(sv[c], sv[c + 1]), make_float2(sl2, sl2), make_float2(neg_m, neg_m));
+            } else {
+              xv.x = fmaf(sv[c], sl2, neg_m);
+              xv.y = fmaf(sv[c + 1], sl2, neg_m);
+            }
+            float2 pv;
+            if ((kPolyPairs >> (e & 7)) & 1) {
+              pv = exp2_poly2(xv);
+            } else {
+              pv.x = fast_exp2(xv.x);
+              pv.y = fast_exp2(xv.y);
+            }
+            float2& acc = (e & 3) == 0 ? acc0 : (e & 3) == 1 ? acc1 : (e & 3) == 2 ? acc2 : acc3;
+            if (kPairedFma) {
+              acc = fadd2(acc, pv);
+            } else {
+              acc.x += pv.x;
+              acc.y += pv.y;
+            }
+            pk[e] = pack_bf16x2(pv.x, pv.y);
+          }
+          tmem_st_32x32b_x16(colS + cc * 16, pk);  // over score columns already consumed
+          if (cc == 1 || cc == 3) {
+            tc_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar((cc == 1 ? kBarPLo : kBarPHi) + x));
+          }
+        }
+        l_sum += ((acc0.x + acc0.y) + (acc1.x + acc1.y)) + ((acc2.x + acc2.y) + (acc3.x + acc3.y));
+      }
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBarOFinal + x), it & 1, budget, abort_flag));
+      if (!ok) raise_abort(abort_flag, p.status);
       tc_fence_after();
-      uint32_t raw[kBN];
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c)
-        tmem_ld_32x32b_x32(colS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&raw[c * 32]));
-      tc_wait_ld();
-      float sv[kBN];
-#pragma unroll
-      for (int c = 0; c < kBN; ++c) sv[c] = __uint_as_float(raw[c]);
 
-      if (!tile_is_full(p, qr0, k0)) {
-        // edge tile: visible keys of this row are columns [cmin, cmax]
-        int cmax = p.N - 1 - k0;
-        if (p.mask_kind != ATTN_MASK_FULL) cmax = min(cmax, qi - k0);
-        const int cmin = (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) ? qi - k0 - p.window + 1 : 0;
+      // ---- epilogue: O / l -> bf16, LSE (natural log). After a timeout every
+      // remaining row of this CTA is written as NaN without touching TMEM.
+      const bool row_valid = qi < p.N;
+      const size_t row = static_cast<size_t>(wi.b * p.Hq + wi.h) * p.N + (row_valid ? qi : 0);
+      __nv_bfloat16* orow = p.o + row * D;
+      const float inv_l = ok ? 1.f / l_sum : NAN;
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) sv[c] = (c >= cmin && c <= cmax) ? sv[c] : -INFINITY;
-      }
-      // row max of the raw scores (scale > 0 commutes with max): four independent chains
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kBN; c += 8) {
-        mx0 = max3f(mx0, sv[c], sv[c + 1]);
-        mx1 = max3f(mx1, sv[c + 2], sv[c + 3]);
-        mx2 = max3f(mx2, sv[c + 4], sv[c + 5]);
-        mx3 = max3f(mx3, sv[c + 6], sv[c + 7]);
-      }
-      const float m_new = fmaxf(m_used, max3f(mx0, mx1, fmaxf(mx2, mx3)) * sl2);
-      bool rescale_o = false;
-      float factor = 1.f;
-      if (m_new > m_used + kRescaleThreshold) {  // also true for the first visible key (m_used = -inf)
-        const bool prev_finite = (m_used != -INFINITY);
-        factor = prev_finite ? fast_exp2(m_used - m_new) : 0.f;
-        l_sum *= factor;
-        rescale_o = prev_finite;  // earlier tiles already put visible keys into O
-        m_used = m_new;
-      }
-      // The score barrier was committed after this tile's previous P.V: O is stable.
-      if (__any_sync(0xffffffffu, rescale_o)) rescale_rows(colO, rescale_o ? factor : 1.f);
-
-      // p = 2^(s * scale * log2 e - m); a row with nothing visible yet uses m = 0.
-      // P goes out in two halves, each announced on its own barrier, so the MMA
-      // warp starts P.V on keys 0-63 while keys 64-127 are still being exponentiated.
-      const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-      float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
-#pragma unroll
-      for (int cc = 0; cc < kBN / 32; ++cc) {
-        uint32_t pk[16];
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        if (ok) {
+          tmem_ld_32x32b_x32(colO + c * 32, ov);
+          tc_wait_ld();
+        }
+        uint4 pk[4];
+        uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int c = cc * 32 + 2 * e;
-          float2 xv;
-          if (kPairedFma) {
-            xv = ffma2(make_float2(sv[c], sv[c + 1]), make_float2(sl2, sl2), make_float2(neg_m, neg_m));
-          } else {
-            xv.x = fmaf(sv[c], sl2, neg_m);
-            xv.y = fmaf(sv[c + 1], sl2, neg_m);
-          }
-          float2 pv;
-          if ((kPolyPairs >> (e & 7)) & 1) {
-            pv = exp2_poly2(xv);
-          } else {
-            pv.x = fast_exp2(xv.x);
-            pv.y = fast_exp2(xv.y);
-          }
-          float2& acc = (e & 3) == 0 ? acc0 : (e & 3) == 1 ? acc1 : (e & 3) == 2 ? acc2 : acc3;
-          if (kPairedFma) {
-            acc = fadd2(acc, pv);
-          } else {
-            acc.x += pv.x;
-            acc.y += pv.y;
-          }
-          pk[e] = pack_bf16x2(pv.x, pv.y);
+          const float a0 = ok ? __uint_as_float(ov[2 * e]) * inv_l : NAN;
+          const float a1 = ok ? __uint_as_float(ov[2 * e + 1]) * inv_l : NAN;
+          pw[e] = pack_bf16x2(a0, a1);
         }
-        tmem_st_32x32b_x16(colS + cc * 16, pk);  // over score columns already consumed
-        if (cc == 1 || cc == 3) {
-          tc_wait_st();
-          tc_fence_before();
-          mbar_arrive(bar((cc == 1 ? kBarPLo : kBarPHi) + x));
+        if (row_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = pk[e];
         }
       }
-      l_sum += ((acc0.x + acc0.y) + (acc1.x + acc1.y)) + ((acc2.x + acc2.y) + (acc3.x + acc3.y));
+      if (row_valid && p.lse != nullptr) p.lse[row] = ok ? (m_used + __log2f(l_sum)) * kLn2 : NAN;
+      // The next item's first P.V overwrites O: its P is announced only after
+      // these loads completed (tcgen05.wait::ld above, fence before the arrive).
+      tc_fence_before();
+      g += T;
+      ++it;
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBarOFinal + x), 0, budget, abort_flag));
-    if (!ok) raise_abort(abort_flag, p.status);
-    tc_fence_after();
-
-    // ---- epilogue: O / l -> bf16, LSE (natural log)
-    const bool row_valid = qi < p.N;
-    __nv_bfloat16* orow = p.o + (static_cast<size_t>(b * p.Hq + h) * p.N + (row_valid ? qi : 0)) * D;
-    const float inv_l = ok ? 1.f / l_sum : NAN;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t ov[32];
-      if (ok) {
-        tmem_ld_32x32b_x32(colO + c * 32, ov);
-        tc_wait_ld();
-      }
-      uint4 pk[4];
-      uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float a0 = ok ? __uint_as_float(ov[2 * e]) * inv_l : NAN;
-        const float a1 = ok ? __uint_as_float(ov[2 * e + 1]) * inv_l : NAN;
-        pw[e] = pack_bf16x2(a0, a1);
-      }
-      if (row_valid) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e] = pk[e];
-      }
-    }
-    if (row_valid && p.lse != nullptr)
-      p.lse[static_cast<size_t>(b * p.Hq + h) * p.N + qi] = ok ? (m_used + __log2f(l_sum)) * kLn2 : NAN;
   }
 
   tc_fence_before();
@@ -581,12 +656,17 @@ int launch_prefill_t(const void* q, const void* k, const void* v, void* o, float
   p.mask_kind = mask_kind;
   p.window = window;
   p.num_cta_tiles = (N + kRowsPerCta - 1) / kRowsPerCta;
+  p.num_items = p.num_cta_tiles * Hq * B;
   p.scale_log2 = scale * kLog2e;
   p.budget = wait_budget_cycles();
   constexpr int smem = PfCfg<D>::kAlloc;
   if (cudaFuncSetAttribute(prefill_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  const dim3 grid(Hq, B, p.num_cta_tiles);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    return ATTN_ERR_CUDA;
+  const dim3 grid(p.num_items < sms ? p.num_items : sms);  // persistent: one CTA per SM
   prefill_fwd_kernel<D><<<grid, kPfThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
