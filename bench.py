@@ -34,7 +34,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from exact_softmax_attention_causal_b200 import accounting, workloads  # noqa: E402
+from exact_softmax_attention_causal_b200 import accounting, sharding, workloads  # noqa: E402
 
 METRIC = "prefill causal-GQA TFLOP/s & paged-decode KV GB/s, % of B200 peak"
 FALLBACK_HBM_GBS = 6650.0
@@ -245,7 +245,7 @@ def run_ours(args, pcfg, dcfg):
         import torch.distributed as dist
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
-    seed = args.seed + 1000 * rank  # every rank owns an independent batch
+    seed = sharding.rank_seed(args.seed, rank)  # every rank owns an independent batch
 
     B, Hq, Hkv, N, d = pcfg["B"], pcfg["Hq"], pcfg["Hkv"], pcfg["N"], pcfg["d"]
     xp = workloads.prefill_inputs(B, Hq, Hkv, N, d, seed)
@@ -323,10 +323,7 @@ def run_ours(args, pcfg, dcfg):
     barrier()
     e2e_ms = e2e_ev[0].elapsed_time(e2e_ev[1])
 
-    times = torch.tensor([p_ms, d_ms, region_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    p_ms, d_ms, region_ms, e2e_ms = times.tolist()
+    p_ms, d_ms, region_ms, e2e_ms = sharding.max_over_ranks([p_ms, d_ms, region_ms, e2e_ms], device=dev)
 
     result = None
     if rank == 0:
@@ -339,7 +336,7 @@ def run_ours(args, pcfg, dcfg):
         d_gbs_launch = kv_bytes / d_avg_s / 1e9
         result = {
             "metric": METRIC,
-            "value": p_flops * K * world / (p_ms / 1e3) / 1e12,
+            "value": sharding.job_throughput(p_flops, world, K, p_ms) / 1e12,
             "unit": "TFLOP/s",
             "n_gpus": world,
             "steps": K,
@@ -356,12 +353,12 @@ def run_ours(args, pcfg, dcfg):
                          "traffic": recorded_traffic("prefill_fwd_kernel", "prefill_sm100.cu"),
                          "peak_source": f"bf16_tflops (burst) {tag}",
                          "kernel": "prefill_fwd_kernel<128>", "flops_per_launch": p_flops},
-            "e2e": {"value": p_flops * K * world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": sharding.job_throughput(p_flops, world, K, e2e_ms) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": 3 * K,
             "clocks": clk.summary(),
             "decode": {
-                "metric": "paged-decode KV GB/s", "value": kv_bytes * K * world / (d_ms / 1e3) / 1e9,
+                "metric": "paged-decode KV GB/s", "value": sharding.job_throughput(kv_bytes, world, K, d_ms) / 1e9,
                 "unit": "GB/s", "workload": dcfg["name"], "kv_bytes_per_step": kv_bytes, "ms_per_step": d_ms / K,
                 "roofline": {"bound": "hbm", "achieved": d_gbs_launch, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                              "frac": d_gbs_launch / peaks["hbm_gbs"],
