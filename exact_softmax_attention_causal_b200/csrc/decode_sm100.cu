@@ -319,32 +319,40 @@ struct MergeParams {
   int B, Hq, splits, chunk, max_seq_len;
 };
 
-// One warp per (sequence, query head): lse = log sum_s exp(lse_s),
-// O = sum_s exp(lse_s - lse) O_s, over the chunks that hold tokens.
+// One CTA of 4 warps per (sequence, query head): lse = log sum_s exp(lse_s),
+// O = sum_s exp(lse_s - lse) O_s over the chunks that hold tokens. The warps
+// take every 4th chunk and combine their partial sums in shared memory, so a
+// single long sequence with hundreds of chunks still merges in parallel.
+constexpr int kMergeWarps = 4;
+
 template <int D>
-__global__ void __launch_bounds__(128) decode_merge_kernel(const MergeParams p) {
-  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (wid >= p.B * p.Hq) return;
-  const int b = wid / p.Hq;
-  const size_t row = static_cast<size_t>(wid);
-  const int seq_len = p.seq_lens[b];
+__global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const MergeParams p) {
   constexpr int PER = D / 32;  // columns per lane
+  __shared__ float s_max[kMergeWarps];
+  __shared__ int s_nan[kMergeWarps];
+  __shared__ float s_sum[kMergeWarps];
+  __shared__ float s_acc[kMergeWarps][D];
+  const size_t row = blockIdx.x;  // b * Hq + h
+  const int b = static_cast<int>(row / p.Hq);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seq_len = p.seq_lens[b];
   __nv_bfloat16* orow = p.o + row * D + lane * PER;
   if (seq_len < 1 || seq_len > p.max_seq_len) {
-    if (lane == 0) {
+    if (threadIdx.x == 0) {
       flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
       if (p.lse) p.lse[row] = NAN;
     }
+    if (warp == 0)
 #pragma unroll
-    for (int e = 0; e < PER; ++e) orow[e] = __float2bfloat16_rn(NAN);
+      for (int e = 0; e < PER; ++e) orow[e] = __float2bfloat16_rn(NAN);
     return;
   }
   const int ns = (seq_len + p.chunk - 1) / p.chunk;
   const float* lrow = p.lse_part + row * p.splits;
+  // global max over the chunks
   float M = -INFINITY;
   bool nan_seen = false;
-  for (int s = lane; s < ns; s += 32) {
+  for (int s = threadIdx.x; s < ns; s += kMergeWarps * 32) {
     const float x = lrow[s];
     nan_seen |= (x != x);
     M = fmaxf(M, x);
@@ -352,34 +360,57 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const MergeParams p) 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   nan_seen = __any_sync(0xffffffffu, nan_seen);
-  float total = 0.f;
-  for (int s = lane; s < ns; s += 32) total += fast_exp2((lrow[s] - M) * kLog2e);
+  if (lane == 0) {
+    s_max[warp] = M;
+    s_nan[warp] = nan_seen ? 1 : 0;
+  }
+  __syncthreads();
+  M = s_max[0];
+  int any_nan = s_nan[0];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
-  const float lse = M + __logf(total);
+  for (int w = 1; w < kMergeWarps; ++w) {
+    M = fmaxf(M, s_max[w]);
+    any_nan |= s_nan[w];
+  }
+  // this warp's chunks: weights relative to the global max
+  float sum = 0.f;
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   const float* obase = p.o_part + row * p.splits * D + lane * PER;
-  for (int s = 0; s < ns; ++s) {
-    const float w = fast_exp2((lrow[s] - lse) * kLog2e);
+  for (int s = warp; s < ns; s += kMergeWarps) {
+    const float w = fast_exp2((lrow[s] - M) * kLog2e);
+    sum += w;
     const float* src = obase + static_cast<size_t>(s) * D;
 #pragma unroll
-    for (int e = 0; e < PER; e += 4) {
-      const float4 v = *reinterpret_cast<const float4*>(src + e);
+    for (int e = 0; e < PER; e += 2) {
+      const float2 v = *reinterpret_cast<const float2*>(src + e);
       acc[e] += w * v.x;
       acc[e + 1] += w * v.y;
-      acc[e + 2] += w * v.z;
-      acc[e + 3] += w * v.w;
     }
   }
+  if (lane == 0) s_sum[warp] = sum;
 #pragma unroll
-  for (int e = 0; e < PER; e += 2) {
-    const float a0 = nan_seen ? NAN : acc[e];
-    const float a1 = nan_seen ? NAN : acc[e + 1];
-    *reinterpret_cast<__nv_bfloat162*>(orow + e) = __floats2bfloat162_rn(a0, a1);
+  for (int e = 0; e < PER; ++e) s_acc[warp][lane * PER + e] = acc[e];
+  __syncthreads();
+  if (warp == 0) {
+    float total = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) total += s_sum[w];
+    const float inv = 1.f / total;
+    float out[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < kMergeWarps; ++w) v += s_acc[w][lane * PER + e];
+      out[e] = any_nan ? NAN : v * inv;
+    }
+#pragma unroll
+    for (int e = 0; e < PER; e += 2)
+      *reinterpret_cast<__nv_bfloat162*>(orow + e) = __floats2bfloat162_rn(out[e], out[e + 1]);
+    if (lane == 0 && p.lse) p.lse[row] = any_nan ? NAN : M + __logf(total);
   }
-  if (lane == 0 && p.lse) p.lse[row] = nan_seen ? NAN : lse;
 }
 
 // Gather: out[b][h][t][:] = cache[block_table[b][t / bs]][t % bs][h][:] for
@@ -468,8 +499,7 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   m.splits = plan.splits;
   m.chunk = plan.chunk;
   m.max_seq_len = max_seq_len;
-  const int warps = B * Hq;
-  decode_merge_kernel<D><<<(warps + 3) / 4, 128, 0, stream>>>(m);
+  decode_merge_kernel<D><<<B * Hq, kMergeWarps * 32, 0, stream>>>(m);
   return cudaGetLastError();
 }
 
