@@ -75,10 +75,10 @@ constexpr int kMmaWarp = 9;
 // Register split (per thread): launched with 168 (65536 / 384, rounded down to
 // a multiple of 8 and capped by the 16K-register sub-partition holding three
 // warps); the TMA/MMA warpgroup gives registers back, the softmax warpgroups
-// take them: 256 x 208 + 128 x 88 = 384 x 168 = 64512.
+// take them: 256 x 224 + 128 x 56 = 384 x 168 = 64512.
 constexpr uint32_t kRegsLaunch = 168;
-constexpr uint32_t kRegsSoftmax = 208;
-constexpr uint32_t kRegsControl = 88;
+constexpr uint32_t kRegsSoftmax = 224;
+constexpr uint32_t kRegsControl = 56;
 static_assert(256 * kRegsSoftmax + 128 * kRegsControl == kPfThreads * kRegsLaunch, "register split");
 static_assert(2 * kRegsSoftmax * 32 + kRegsControl * 32 <= 16384, "per sub-partition register file");
 constexpr float kRescaleThreshold = 8.0f;
@@ -88,11 +88,16 @@ struct PfCfg {
   static constexpr int kHalf = 128 * 128;    // bytes of one 64-column box of 128 rows
   static constexpr int kHalves = D / 64;     // 128-byte swizzle columns per tile
   static constexpr int kTile = kHalves * kHalf;
-  static constexpr int kStages = (D == 128) ? 2 : 4;
+  static constexpr int kKStages = (D == 128) ? 2 : 4;  // K ring depth
+  static constexpr int kVStages = (D == 128) ? 2 : 4;  // V ring depth
   static constexpr int kQOff = 0;            // Q tile A, then Q tile B
   static constexpr int kKOff = kQOff + kTilesPerCta * kTile;
-  static constexpr int kVOff = kKOff + kStages * kTile;
-  static constexpr int kBarOff = kVOff + kStages * kTile;
+  static constexpr int kVOff = kKOff + kKStages * kTile;
+  // Epilogue staging: per softmax warp 32 rows x 64 columns of bf16 (4 KB, one
+  // 128-byte-swizzled TMA store box), written once per 64-column half of O.
+  static constexpr int kStageOff = kVOff + kVStages * kTile;
+  static constexpr int kStageBytes = 8 * 32 * 128;
+  static constexpr int kBarOff = kStageOff + kStageBytes;
   static constexpr int kBytes = kBarOff + 256;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
   // TMEM columns (512 allocated): scores of A and B (128 fp32 columns each;
@@ -210,6 +215,42 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   return make_float2(__uint_as_float(r0), __uint_as_float(r1));
 }
 
+// One MMA step of S = Q K^T: descriptors are the operand bases plus a fixed
+// offset (16-byte units) added inside the asm, so the compiler cannot hoist a
+// descriptor per step into registers.
+template <uint32_t OFF, uint32_t IDESC>
+__device__ __forceinline__ void mma_ss_step(uint32_t d_tmem, uint64_t a_base, uint64_t b_base, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n .reg .b64 da, db;\n setp.ne.b32 p, %3, 0;\n add.s64 da, %1, %4;\n add.s64 db, %2, %4;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_base), "l"(b_base), "r"(accumulate), "n"(OFF), "n"(IDESC)
+      : "memory");
+}
+// One MMA step of O += P V with P in TMEM at column offset ACOL and V at OFF.
+template <uint32_t ACOL, uint32_t OFF, uint32_t IDESC>
+__device__ __forceinline__ void mma_ts_step(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_base, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n .reg .b32 ta;\n .reg .b64 db;\n setp.ne.b32 p, %3, 0;\n add.u32 ta, %1, %4;\n"
+      " add.s64 db, %2, %5;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %6, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_base), "r"(accumulate), "n"(ACOL), "n"(OFF), "n"(IDESC)
+      : "memory");
+}
+// All D/16 steps of one score MMA (K dimension = head dim; 64-column boxes of
+// 16 KB hold 4 steps of 32 bytes each).
+template <int D, int KK = 0>
+__device__ __forceinline__ void mma_scores(uint32_t d_tmem, uint64_t dq, uint64_t dk) {
+  constexpr uint32_t off = static_cast<uint32_t>(((KK >> 2) * (128 * 128) + (KK & 3) * 32) >> 4);
+  mma_ss_step<off, idesc_bf16(kBM, kBN, 0)>(d_tmem, dq, dk, KK > 0 ? 1u : 0u);
+  if constexpr (KK + 1 < D / 16) mma_scores<D, KK + 1>(d_tmem, dq, dk);
+}
+// Steps [KK, END) of one P.V MMA (16 keys per step: 8 TMEM columns of P, 2 KB of V).
+template <int D, int KK, int END>
+__device__ __forceinline__ void mma_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t dv, bool first) {
+  constexpr uint32_t voff = static_cast<uint32_t>((KK * 2048) >> 4);
+  mma_ts_step<KK * 8, voff, idesc_bf16(kBM, D, 1)>(d_tmem, p_tmem, dv, (!first || KK > 0) ? 1u : 0u);
+  if constexpr (KK + 1 < END) mma_pv<D, KK + 1, END>(d_tmem, p_tmem, dv, first);
+}
+
 // Column pairs (of every 8) whose exponentials run on the FMA pipes: bit e set
 // = pair e uses exp2_poly2, the others use the special-function unit.
 constexpr uint32_t kPolyPairs = 0x00;
@@ -242,7 +283,8 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 template <int D>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                       const PrefillParams p) {
   using C = PfCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -262,7 +304,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQFull), 1);
     mbar_init(bar(kBarQEmpty), 1);
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < 4; ++s) {  // every slot initialised; only kKStages / kVStages used
       mbar_init(bar(kBarKFull + s), 1);
       mbar_init(bar(kBarVFull + s), 1);
       mbar_init(bar(kBarKEmpty + s), 1);
@@ -320,7 +362,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // K_i is issued before V_{i-1}: the score MMA needs K one tile earlier than P.V needs V.
         for (int i = 0; i <= T; ++i) {
           if (i < T) {
-            const int gi = g + i, s = gi % C::kStages, rnd = gi / C::kStages;
+            const int gi = g + i, s = gi % C::kKStages, rnd = gi / C::kKStages;
             if (rnd > 0 && !mbar_wait_bounded(bar(kBarKEmpty + s), (rnd - 1) & 1, budget, abort_flag)) {
               ok = false;
               break;
@@ -332,7 +374,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             k_issued = gi + 1;
           }
           if (i >= 1) {
-            const int gv = g + i - 1, s = gv % C::kStages, rnd = gv / C::kStages;
+            const int gv = g + i - 1, s = gv % C::kVStages, rnd = gv / C::kVStages;
             if (rnd > 0 && !mbar_wait_bounded(bar(kBarVEmpty + s), (rnd - 1) & 1, budget, abort_flag)) {
               ok = false;
               break;
@@ -351,14 +393,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // Drain: the newest copy of every stage and of Q has landed before the CTA may exit.
       volatile int never = 0;
       if (it > 0) mbar_wait_bounded(bar(kBarQFull), (it - 1) & 1, kDrainBudgetCycles, &never);
-      for (int j = (k_issued > C::kStages ? k_issued - C::kStages : 0); j < k_issued; ++j)
-        mbar_wait_bounded(bar(kBarKFull + j % C::kStages), (j / C::kStages) & 1, kDrainBudgetCycles, &never);
-      for (int j = (v_issued > C::kStages ? v_issued - C::kStages : 0); j < v_issued; ++j)
-        mbar_wait_bounded(bar(kBarVFull + j % C::kStages), (j / C::kStages) & 1, kDrainBudgetCycles, &never);
+      for (int j = (k_issued > C::kKStages ? k_issued - C::kKStages : 0); j < k_issued; ++j)
+        mbar_wait_bounded(bar(kBarKFull + j % C::kKStages), (j / C::kKStages) & 1, kDrainBudgetCycles, &never);
+      for (int j = (v_issued > C::kVStages ? v_issued - C::kVStages : 0); j < v_issued; ++j)
+        mbar_wait_bounded(bar(kBarVFull + j % C::kVStages), (j / C::kVStages) & 1, kDrainBudgetCycles, &never);
     } else if (warp == kMmaWarp && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc_qk = idesc_bf16(kBM, kBN, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16(kBM, D, 1);
       // Descriptors are built once; an operand at byte offset o from its base has
       // descriptor base + o / 16 (the start address is the low field, and every
       // tile lies below 256 KB, so the addition never carries out of it).
@@ -368,13 +408,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       constexpr uint64_t kTileUnits = C::kTile >> 4;
       // S_x = Q_x K^T of global key tile g into tile x's score columns
       auto issue_s = [&](int x, int g) {
-        const uint64_t dq = dq0 + static_cast<uint64_t>(x) * kTileUnits;
-        const uint64_t dk = dk0 + static_cast<uint64_t>(g % C::kStages) * kTileUnits;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * C::kHalf + (kk & 3) * 32) >> 4);
-          tc_mma_ss(tmem + C::col_s(x), dq + koff, dk + koff, idesc_qk, kk > 0 ? 1u : 0u);
-        }
+        mma_scores<D>(tmem + C::col_s(x), dq0 + static_cast<uint64_t>(x) * kTileUnits,
+                      dk0 + static_cast<uint64_t>(g % C::kKStages) * kTileUnits);
         tc_commit(bar(kBarSFull + x));
       };
       // O_x (+)= P_x V for keys [64 half, 64 half + 64) of global key tile g; P_x sits in
@@ -382,11 +417,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       auto pv_half = [&](int x, int g, int half, bool first) -> bool {
         if (!mbar_wait_bounded(bar((half ? kBarPHi : kBarPLo) + x), g & 1, budget, abort_flag)) return false;
         tc_fence_after();
-        const uint64_t dv = dv0 + static_cast<uint64_t>(g % C::kStages) * kTileUnits;
-#pragma unroll
-        for (int kk = half * 4; kk < half * 4 + 4; ++kk)
-          tc_mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4),
-                    idesc_pv, (!first || kk > 0) ? 1u : 0u);
+        const uint64_t dv = dv0 + static_cast<uint64_t>(g % C::kVStages) * kTileUnits;
+        if (half == 0)
+          mma_pv<D, 0, 4>(tmem + C::col_o(x), tmem + C::col_s(x), dv, first);
+        else
+          mma_pv<D, 4, 8>(tmem + C::col_o(x), tmem + C::col_s(x), dv, first);
         return true;
       };
       int g = 0, it = 0;
@@ -399,28 +434,28 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         kv_tile_range(p, wi.q0, kt_lo, kt_hi);
         const int T = kt_hi - kt_lo + 1;
         if (!mbar_wait_bounded(bar(kBarQFull), it & 1, budget, abort_flag) ||
-            !mbar_wait_bounded(bar(kBarKFull + g % C::kStages), (g / C::kStages) & 1, budget, abort_flag)) {
+            !mbar_wait_bounded(bar(kBarKFull + g % C::kKStages), (g / C::kKStages) & 1, budget, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         issue_s(0, g);
         issue_s(1, g);
-        tc_commit(bar(kBarKEmpty + g % C::kStages));
+        tc_commit(bar(kBarKEmpty + g % C::kKStages));
         if (T == 1) tc_commit(bar(kBarQEmpty));
         for (int j = 0; j < T; ++j) {
           const int gj = g + j, gn = gj + 1;
-          const int s = gj % C::kStages;
+          const int s = gj % C::kVStages;  // V stage of key tile j
           // tile A: P.V of key tile j (as each half of P lands), then the scores of tile
           // j + 1 (in issue order, so the new scores overwrite P only after P.V read it)
-          if (!mbar_wait_bounded(bar(kBarVFull + s), (gj / C::kStages) & 1, budget, abort_flag) ||
+          if (!mbar_wait_bounded(bar(kBarVFull + s), (gj / C::kVStages) & 1, budget, abort_flag) ||
               !pv_half(0, gj, 0, j == 0) || !pv_half(0, gj, 1, j == 0)) {
             ok = false;
             break;
           }
           if (j == T - 1) tc_commit(bar(kBarOFinal + 0));
           if (j + 1 < T) {
-            if (!mbar_wait_bounded(bar(kBarKFull + gn % C::kStages), (gn / C::kStages) & 1, budget, abort_flag)) {
+            if (!mbar_wait_bounded(bar(kBarKFull + gn % C::kKStages), (gn / C::kKStages) & 1, budget, abort_flag)) {
               ok = false;
               break;
             }
@@ -436,7 +471,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tc_commit(bar(kBarVEmpty + s));
           if (j + 1 < T) {
             issue_s(1, gn);
-            tc_commit(bar(kBarKEmpty + gn % C::kStages));
+            tc_commit(bar(kBarKEmpty + gn % C::kKStages));
             if (j + 2 == T) tc_commit(bar(kBarQEmpty));  // that was the item's last read of Q
           }
         }
@@ -564,31 +599,47 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (!ok) raise_abort(abort_flag, p.status);
       tc_fence_after();
 
-      // ---- epilogue: O / l -> bf16, LSE (natural log). After a timeout every
-      // remaining row of this CTA is written as NaN without touching TMEM.
+      // ---- epilogue: O / l -> bf16 through a swizzled shared staging box and a TMA
+      // store per warp and 64-column half (rows past N are clipped by the store);
+      // LSE (natural log) per thread. After a timeout every remaining row of this
+      // CTA is written as NaN without touching TMEM.
       const bool row_valid = qi < p.N;
       const size_t row = static_cast<size_t>(wi.b * p.Hq + wi.h) * p.N + (row_valid ? qi : 0);
-      __nv_bfloat16* orow = p.o + row * D;
       const float inv_l = ok ? 1.f / l_sum : NAN;
+      const uint32_t stage = sbase + C::kStageOff + warp * 4096;
+      const int wrow = r & 31;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t ov[32];
-        if (ok) {
-          tmem_ld_32x32b_x32(colO + c * 32, ov);
-          tc_wait_ld();
+      for (int hh = 0; hh < D / 64; ++hh) {
+        if (lane == 0) bulk_wait_read_all();  // the previous store has read the staging box
+        __syncwarp();
+#pragma unroll
+        for (int q32 = 0; q32 < 2; ++q32) {  // 32 columns at a time: 4 swizzled 16-byte chunks
+          uint32_t ov[32];
+          if (ok) {
+            tmem_ld_32x32b_x32(colO + hh * 64 + q32 * 32, ov);
+            tc_wait_ld();
+          }
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float a0 = ok ? __uint_as_float(ov[c4 * 8 + 2 * e]) * inv_l : NAN;
+              const float a1 = ok ? __uint_as_float(ov[c4 * 8 + 2 * e + 1]) * inv_l : NAN;
+              w4[e] = pack_bf16x2(a0, a1);
+            }
+            const int c = q32 * 4 + c4;
+            const uint32_t dst = stage + wrow * 128 + ((c ^ (wrow & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(dst), "r"(w4[0]), "r"(w4[1]),
+                         "r"(w4[2]), "r"(w4[3])
+                         : "memory");
+          }
         }
-        uint4 pk[4];
-        uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float a0 = ok ? __uint_as_float(ov[2 * e]) * inv_l : NAN;
-          const float a1 = ok ? __uint_as_float(ov[2 * e + 1]) * inv_l : NAN;
-          pw[e] = pack_bf16x2(a0, a1);
-        }
-        if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = pk[e];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && qr0 + (warp & 3) * 32 < p.N) {  // a box wholly past N has nothing to write
+          tma_store_3d(&tm_o, stage, hh * 64, qr0 + (warp & 3) * 32, wi.b * p.Hq + wi.h);
+          bulk_commit();
         }
       }
       if (row_valid && p.lse != nullptr) p.lse[row] = ok ? (m_used + __log2f(l_sum)) * kLn2 : NAN;
@@ -598,6 +649,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       g += T;
       ++it;
     }
+    if (lane == 0) bulk_wait_all();  // output stores complete before the CTA exits
   }
 
   tc_fence_before();
@@ -623,13 +675,13 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // [heads][n][d] bf16 viewed as a rank-3 tensor (d innermost); box = 64 columns
 // x 128 rows x 1 head, 128-byte swizzle. Rows past n read as zero.
-bool encode_bhnd(CUtensorMap* map, const void* base, int d, int n, int heads) {
+bool encode_bhnd(CUtensorMap* map, const void* base, int d, int n, int heads, int box_rows = 128) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
                               static_cast<cuuint64_t>(heads)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(n) * d * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estride[3] = {1, 1, 1};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
                          estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -640,9 +692,9 @@ bool encode_bhnd(CUtensorMap* map, const void* base, int d, int n, int heads) {
 template <int D>
 int launch_prefill_t(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
                      int mask_kind, int window, float scale, int32_t* status, cudaStream_t stream) {
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!encode_bhnd(&tq, q, D, N, B * Hq) || !encode_bhnd(&tk, k, D, N, B * Hkv) ||
-      !encode_bhnd(&tv, v, D, N, B * Hkv))
+      !encode_bhnd(&tv, v, D, N, B * Hkv) || !encode_bhnd(&to, o, D, N, B * Hq, 32))
     return ATTN_ERR_CUDA;
   PrefillParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -667,7 +719,7 @@ int launch_prefill_t(const void* q, const void* k, const void* v, void* o, float
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
     return ATTN_ERR_CUDA;
   const dim3 grid(p.num_items < sms ? p.num_items : sms);  // persistent: one CTA per SM
-  prefill_fwd_kernel<D><<<grid, kPfThreads, smem, stream>>>(tq, tk, tv, p);
+  prefill_fwd_kernel<D><<<grid, kPfThreads, smem, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
