@@ -48,10 +48,13 @@ def test_head_maps(hq, hkv):
     _full_check(2, hq, hkv, 256, 128, "causal", seed=2)
 
 
-@pytest.mark.parametrize("N", [1, 7, 129, 640])
+@pytest.mark.parametrize("N", [1, 7, 129, 257, 640])
 def test_sizes(N):
     _full_check(1, 2, 1, N, 128, "causal", seed=3)
     _full_check(1, 2, 1, N, 64, "full", seed=3)
+    # small windows: the second query tile of an item may have no row before N
+    _full_check(1, 2, 1, N, 128, "window", window=1, seed=3)
+    _full_check(1, 2, 1, N, 64, "window", window=3, seed=3)
 
 
 def test_causal_row0_is_v0_exactly():
