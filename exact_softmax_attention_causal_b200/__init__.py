@@ -21,7 +21,7 @@ from ._lib import AttnError, STATUS_BIT_DEVICE_CHECK, STATUS_BIT_TIMEOUT  # noqa
 
 MASKS = {"full": 0, "causal": 1, "window": 2, "sliding_window": 2}
 
-__all__ = ["prefill", "decode_paged", "paged_gather", "decode_plan", "decode_workspace_bytes", "AttnError",
+__all__ = ["prefill", "prefill_paged", "decode_paged", "paged_gather", "decode_plan", "decode_workspace_bytes", "AttnError",
            "version"]
 
 
@@ -78,6 +78,43 @@ def prefill(q, k, v, mask: str = "causal", window: int = 0, scale: float | None 
     rc = _lib.lib().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d, MASKS[mask],
                                  int(window), float(scale), _ptr(status), _stream_handle(stream))
     _lib.check(rc, "attn_prefill")
+    return out, lse
+
+
+def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int, mask: str = "causal",
+                  window: int = 0, scale: float | None = None, out=None, lse=None, status=None, stream=None,
+                  return_lse: bool = True):
+    """Prefix (chunked) prefill: the newest Nq positions of every sequence attend
+    to its seq_lens[b] cached tokens through the block table; returns (O, LSE).
+
+    q [B, Hq, Nq, d] bf16; caches [num_blocks, block_size, Hkv, d] bf16;
+    block_table [B, max_blocks] int32; seq_lens [B] int32 (each >= Nq).
+    Query row i of sequence b sits at position seq_lens[b] - Nq + i.
+    """
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hq, Nq, d = q.shape
+    num_blocks, block_size, Hkv, d2 = k_cache.shape
+    if d2 != d or v_cache.shape != k_cache.shape:
+        raise ValueError("caches must be [num_blocks, block_size, Hkv, d] matching q")
+    if block_table.shape[0] != B or seq_lens.shape[0] != B:
+        raise ValueError("block_table and seq_lens need one row per sequence")
+    if mask not in MASKS:
+        raise ValueError(f"mask must be one of {sorted(MASKS)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    rc = _lib.lib().attn_prefill_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+                                       _ptr(out), _ptr(lse), B, Hq, Hkv, Nq, d, num_blocks, block_size,
+                                       block_table.shape[1], int(max_seq_len), MASKS[mask], int(window),
+                                       float(scale), _ptr(status), _stream_handle(stream))
+    _lib.check(rc, "attn_prefill_paged")
     return out, lse
 
 

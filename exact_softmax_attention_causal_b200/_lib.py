@@ -15,6 +15,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn_b20
 # Exported symbols, as declared in include/attn.h.
 SYMBOLS = (
     "attn_prefill",
+    "attn_prefill_paged",
     "attn_decode_plan",
     "attn_decode_workspace_bytes",
     "attn_decode_paged",
@@ -47,6 +48,9 @@ _sz = ctypes.c_size_t
 def _declare(lib):
     lib.attn_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _vp]
     lib.attn_prefill.restype = _i
+    lib.attn_prefill_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                                       _i, _f, _vp, _vp]
+    lib.attn_prefill_paged.restype = _i
     lib.attn_decode_plan.argtypes = [_i, _i, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i)]
     lib.attn_decode_plan.restype = _i
     lib.attn_decode_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]

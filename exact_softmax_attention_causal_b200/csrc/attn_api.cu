@@ -77,6 +77,33 @@ int attn_prefill(const void* q, const void* k, const void* v, void* o, float* ls
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
+int attn_prefill_paged(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                       const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int d,
+                       int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, int mask_kind,
+                       int window, float scale, int32_t* status, attn_stream_t stream) {
+  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !o) return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || d <= 0 || num_blocks <= 0 || block_size <= 0 ||
+      max_blocks_per_seq <= 0 || max_seq_len < Nq)
+    return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(max_blocks_per_seq) * block_size < max_seq_len) return ATTN_ERR_INVALID_ARG;
+  if (mask_kind != ATTN_MASK_FULL && mask_kind != ATTN_MASK_CAUSAL && mask_kind != ATTN_MASK_SLIDING_WINDOW)
+    return ATTN_ERR_INVALID_ARG;
+  if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window < 1) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Hq * Nq > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
+  if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window >= max_seq_len) mask_kind = ATTN_MASK_CAUSAL;
+  return launch_prefill_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, Nq, d, num_blocks,
+                              block_size, max_blocks_per_seq, max_seq_len, mask_kind, window, scale, status,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
 int attn_decode_plan(int B, int Hq, int Hkv, int max_seq_len, int num_sms, int* chunk_tokens, int* num_splits) {
   DecodePlan plan;
   const int rc = plan_decode(B, Hq, Hkv, max_seq_len, num_sms, &plan);

@@ -43,4 +43,10 @@ cudaError_t launch_paged_gather(const void* cache, const int32_t* block_table, c
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
                    int d, int mask_kind, int window, float scale, int32_t* status, cudaStream_t stream);
 
+// Prefill of the newest Nq positions of each sequence against its paged context.
+int launch_prefill_paged(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                         const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int d,
+                         int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, int mask_kind,
+                         int window, float scale, int32_t* status, cudaStream_t stream);
+
 }  // namespace attn

@@ -144,10 +144,16 @@ struct PrefillParams {
   __nv_bfloat16* o;
   float* lse;
   int32_t* status;
-  int B, Hq, Hkv, N, group, mask_kind, window, num_cta_tiles;
+  int B, Hq, Hkv, N, group, mask_kind, window, num_cta_tiles;  // N = query rows per sequence
   int num_items;  // num_cta_tiles * Hq * B
   float scale_log2;
   long long budget;
+  // Paged context (prefix prefill): the keys of sequence b are its seq_lens[b]
+  // cached tokens, read through block_table; the N query rows are its newest N
+  // positions. Unused (null) for the contiguous prefill, where keys = rows = N.
+  const int32_t* block_table;  // [B, max_blocks]
+  const int32_t* seq_lens;     // [B]
+  int max_blocks, block_size, num_blocks, max_seq_len;
 };
 
 // One work item: 256 query rows of one (batch, head). Items are numbered
@@ -170,19 +176,36 @@ __device__ __forceinline__ int item_index(int round, int c, int G) {
   return round * G + ((round & 1) ? (G - 1 - c) : c);
 }
 
-// Key tiles the 256 query rows [q0, q0 + 256) visit: [lo, hi], inclusive.
-__device__ __forceinline__ void kv_tile_range(const PrefillParams& p, int q0, int& lo, int& hi) {
-  hi = (p.N - 1) / kBN;
-  lo = 0;
-  if (p.mask_kind != ATTN_MASK_FULL) hi = min(hi, (q0 + kRowsPerCta - 1) / kBN);
-  if (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) lo = max(0, q0 - p.window + 1) / kBN;
+// Geometry of one item: nk keys, query row i at position pos0 + i (bottom-right
+// alignment: the rows are the newest positions of the sequence), and the key
+// tiles [lo, lo + T) its 256 rows see. For a paged context with an out-of-range
+// seq_len the item is computed over nk = N and its rows come out as NaN.
+struct ItemGeom {
+  int nk, pos0, lo, T;
+  bool bad;
+};
+template <bool PAGED>
+__device__ __forceinline__ ItemGeom item_geom(const PrefillParams& p, const WorkItem& wi) {
+  int nk = p.N;
+  bool bad = false;
+  if (PAGED) {
+    const int sl = __ldg(p.seq_lens + wi.b);
+    bad = sl < p.N || sl > p.max_seq_len;
+    nk = bad ? p.N : sl;
+  }
+  const int pos0 = nk - p.N;
+  int hi = (nk - 1) / kBN, lo = 0;
+  if (p.mask_kind != ATTN_MASK_FULL) hi = min(hi, (pos0 + wi.q0 + kRowsPerCta - 1) / kBN);
+  if (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) lo = max(0, pos0 + wi.q0 - p.window + 1) / kBN;
+  return ItemGeom{nk, pos0, lo, hi - lo + 1, bad};
 }
 
-// True when every (row, key) pair of a 128 x 128 tile is visible.
-__device__ __forceinline__ bool tile_is_full(const PrefillParams& p, int qr0, int k0) {
-  bool full = (k0 + kBN <= p.N);
-  if (p.mask_kind != ATTN_MASK_FULL) full = full && (k0 + kBN - 1 <= qr0);
-  if (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) full = full && (qr0 + kBM - 1 - k0 < p.window);
+// True when every (row, key) pair of a 128 x 128 tile is visible: rows at
+// positions [qpos0, qpos0 + 128), keys [k0, k0 + 128) of nk.
+__device__ __forceinline__ bool tile_is_full(const PrefillParams& p, int qpos0, int k0, int nk) {
+  bool full = (k0 + kBN <= nk);
+  if (p.mask_kind != ATTN_MASK_FULL) full = full && (k0 + kBN - 1 <= qpos0);
+  if (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) full = full && (qpos0 + kBM - 1 - k0 < p.window);
   return full;
 }
 
@@ -280,10 +303,11 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 // Persistent: one CTA per SM walks its share of the work items. Barrier phases
 // run on across items: K/V stages and score/probability barriers count key
 // tiles (g), Q and final-output barriers count items (it).
-template <int D>
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                       const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_vr,
                        const PrefillParams p) {
   using C = PfCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -344,11 +368,47 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int w = item_index(round, cta, G);
         if (w >= p.num_items) break;
         const WorkItem wi = item_at(p, w);
-        int kt_lo, kt_hi;
-        kv_tile_range(p, wi.q0, kt_lo, kt_hi);
-        const int T = kt_hi - kt_lo + 1;
+        const ItemGeom gm = item_geom<PAGED>(p, wi);
+        const int kt_lo = gm.lo, T = gm.T;
         const int zq = wi.b * p.Hq + wi.h;
-        const int zkv = wi.b * p.Hkv + wi.h / p.group;
+        const int kvh = wi.h / p.group;
+        const int zkv = wi.b * p.Hkv + kvh;
+        // One K or V tile: a 128-row box of the contiguous tensor, or, for a paged
+        // context, 128 / block_size boxes of one block each, found through the
+        // block table. A block past the sequence or with an entry outside the pool
+        // is requested at block index num_blocks: TMA fills it with zeros (the
+        // softmax masks those keys and flags the bad entry). The sequence's last,
+        // partly filled block goes row by row (tm_row: one-row boxes) so that its
+        // slots past seq_len arrive as zeros, never as stale pool contents: their
+        // probabilities are 0, and 0 * NaN would still poison P.V.
+        auto load_kv = [&](const CUtensorMap* tm, const CUtensorMap* tm_row, uint32_t dst, uint32_t bar_full,
+                           int kt) {
+          if (!PAGED) {
+            for (int hh = 0; hh < C::kHalves; ++hh)
+              tma_load_3d(dst + hh * C::kHalf, tm, bar_full, hh * 64, kt * kBN, zkv);
+          } else {
+            const int bs = p.block_size;
+            for (int e = 0; e < kBN / bs; ++e) {
+              const int key = kt * kBN + e * bs;
+              int phys = p.num_blocks;
+              if (!gm.bad && key < gm.nk) {
+                const int entry = __ldg(p.block_table + static_cast<size_t>(wi.b) * p.max_blocks + key / bs);
+                if (entry >= 0 && entry < p.num_blocks) phys = entry;
+              }
+              const uint32_t bdst = dst + e * bs * 128;
+              if (key + bs <= gm.nk || phys == p.num_blocks) {
+                for (int hh = 0; hh < C::kHalves; ++hh)
+                  tma_load_4d(bdst + hh * C::kHalf, tm, bar_full, hh * 64, kvh, 0, phys);
+              } else {
+                const int valid = gm.nk - key;  // 1 .. bs - 1 rows hold tokens
+                for (int slot = 0; slot < bs; ++slot)
+                  for (int hh = 0; hh < C::kHalves; ++hh)
+                    tma_load_4d(bdst + hh * C::kHalf + slot * 128, tm_row, bar_full, hh * 64, kvh, slot,
+                                slot < valid ? phys : p.num_blocks);
+              }
+            }
+          }
+        };
         // Q of this item once the previous item's last score MMA has read its Q
         if (it > 0 && !mbar_wait_bounded(bar(kBarQEmpty), (it - 1) & 1, budget, abort_flag)) {
           ok = false;
@@ -368,9 +428,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               break;
             }
             mbar_arrive_expect_tx(bar(kBarKFull + s), C::kTile);
-            for (int hh = 0; hh < C::kHalves; ++hh)
-              tma_load_3d(sbase + C::kKOff + s * C::kTile + hh * C::kHalf, &tm_k, bar(kBarKFull + s), hh * 64,
-                          (kt_lo + i) * kBN, zkv);
+            load_kv(&tm_k, &tm_kr, sbase + C::kKOff + s * C::kTile, bar(kBarKFull + s), kt_lo + i);
             k_issued = gi + 1;
           }
           if (i >= 1) {
@@ -380,9 +438,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               break;
             }
             mbar_arrive_expect_tx(bar(kBarVFull + s), C::kTile);
-            for (int hh = 0; hh < C::kHalves; ++hh)
-              tma_load_3d(sbase + C::kVOff + s * C::kTile + hh * C::kHalf, &tm_v, bar(kBarVFull + s), hh * 64,
-                          (kt_lo + i - 1) * kBN, zkv);
+            load_kv(&tm_v, &tm_vr, sbase + C::kVOff + s * C::kTile, bar(kBarVFull + s), kt_lo + i - 1);
             v_issued = gv + 1;
           }
         }
@@ -430,9 +486,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int w = item_index(round, cta, G);
         if (w >= p.num_items) break;
         const WorkItem wi = item_at(p, w);
-        int kt_lo, kt_hi;
-        kv_tile_range(p, wi.q0, kt_lo, kt_hi);
-        const int T = kt_hi - kt_lo + 1;
+        const int T = item_geom<PAGED>(p, wi).T;
         if (!mbar_wait_bounded(bar(kBarQFull), it & 1, budget, abort_flag) ||
             !mbar_wait_bounded(bar(kBarKFull + g % C::kKStages), (g / C::kKStages) & 1, budget, abort_flag)) {
           ok = false;
@@ -500,11 +554,28 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int w = item_index(round, cta, G);
       if (w >= p.num_items) break;
       const WorkItem wi = item_at(p, w);
-      int kt_lo, kt_hi;
-      kv_tile_range(p, wi.q0, kt_lo, kt_hi);
-      const int T = kt_hi - kt_lo + 1;
-      const int qr0 = wi.q0 + x * kBM;  // first query position of the tile
-      const int qi = qr0 + r;           // this thread's query position
+      const ItemGeom gm = item_geom<PAGED>(p, wi);
+      const int kt_lo = gm.lo, T = gm.T;
+      const int qr0 = wi.q0 + x * kBM;  // first query row of the tile
+      const int qi = qr0 + r;           // this thread's query row
+      const int qpos = gm.pos0 + qi;    // its position among the keys
+      // A paged item whose seq_len is out of range, or that reads a block-table
+      // entry outside the pool, yields NaN rows and the device-check status bit.
+      bool item_bad = false;
+      if (PAGED) {
+        item_bad = gm.bad;
+        if (!item_bad) {
+          const int first = kt_lo * kBN / p.block_size;
+          const int last = (min((kt_lo + T) * kBN, gm.nk) - 1) / p.block_size;
+          bool bad_entry = false;
+          for (int e = first + lane; e <= last; e += 32) {
+            const int entry = __ldg(p.block_table + static_cast<size_t>(wi.b) * p.max_blocks + e);
+            bad_entry |= entry < 0 || entry >= p.num_blocks;
+          }
+          item_bad = __any_sync(0xffffffffu, bad_entry);
+        }
+        if (item_bad && lane == 0 && p.status != nullptr) atomicOr(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
+      }
       float m_used = -INFINITY;         // max the exponentials are taken against (base 2)
       float l_sum = 0.f;                // running sum of 2^(x - m_used), fp32
       for (int j = 0; j < T && ok; ++j) {
@@ -522,11 +593,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
         for (int c = 0; c < kBN; ++c) sv[c] = __uint_as_float(raw[c]);
 
-        if (!tile_is_full(p, qr0, k0)) {
+        if (!tile_is_full(p, gm.pos0 + qr0, k0, gm.nk)) {
           // edge tile: visible keys of this row are columns [cmin, cmax]
-          int cmax = p.N - 1 - k0;
-          if (p.mask_kind != ATTN_MASK_FULL) cmax = min(cmax, qi - k0);
-          const int cmin = (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) ? qi - k0 - p.window + 1 : 0;
+          int cmax = gm.nk - 1 - k0;
+          if (p.mask_kind != ATTN_MASK_FULL) cmax = min(cmax, qpos - k0);
+          const int cmin = (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) ? qpos - k0 - p.window + 1 : 0;
 #pragma unroll
           for (int c = 0; c < kBN; ++c) sv[c] = (c >= cmin && c <= cmax) ? sv[c] : -INFINITY;
         }
@@ -605,7 +676,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // CTA is written as NaN without touching TMEM.
       const bool row_valid = qi < p.N;
       const size_t row = static_cast<size_t>(wi.b * p.Hq + wi.h) * p.N + (row_valid ? qi : 0);
-      const float inv_l = ok ? 1.f / l_sum : NAN;
+      const bool out_ok = ok && !item_bad;
+      const float inv_l = out_ok ? 1.f / l_sum : NAN;
       const uint32_t stage = sbase + C::kStageOff + warp * 4096;
       const int wrow = r & 31;
 #pragma unroll
@@ -642,7 +714,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           bulk_commit();
         }
       }
-      if (row_valid && p.lse != nullptr) p.lse[row] = ok ? (m_used + __log2f(l_sum)) * kLn2 : NAN;
+      if (row_valid && p.lse != nullptr) p.lse[row] = out_ok ? (m_used + __log2f(l_sum)) * kLn2 : NAN;
       // The next item's first P.V overwrites O: its P is announced only after
       // these loads completed (tcgen05.wait::ld above, fence before the arrive).
       tc_fence_before();
@@ -689,13 +761,52 @@ bool encode_bhnd(CUtensorMap* map, const void* base, int d, int n, int heads, in
   return r == CUDA_SUCCESS;
 }
 
-template <int D>
+// The paged pool [num_blocks][block_size][Hkv][d] bf16 as a rank-4 tensor
+// (d, Hkv, slot, block); box = 64 columns x 1 head x box_slots slots x 1
+// block, 128-byte swizzle: box_slots = block_size loads one block of one head,
+// box_slots = 1 one token row.
+bool encode_pool(CUtensorMap* map, const void* base, int d, int hkv, int block_size, int num_blocks,
+                 int box_slots) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(hkv),
+                              static_cast<cuuint64_t>(block_size), static_cast<cuuint64_t>(num_blocks)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(hkv) * d * 2,
+                                 static_cast<cuuint64_t>(block_size) * hkv * d * 2};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_slots), 1};
+  const cuuint32_t estride[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct PagedContext {
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  int num_blocks, block_size, max_blocks, max_seq_len;
+};
+
+// N = query rows per sequence. Contiguous: k, v are [B, Hkv, N, d]. Paged
+// (ctx != null): k, v are the pools and every sequence's keys come from its
+// block-table row.
+template <int D, bool PAGED>
 int launch_prefill_t(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
-                     int mask_kind, int window, float scale, int32_t* status, cudaStream_t stream) {
-  CUtensorMap tq, tk, tv, to;
-  if (!encode_bhnd(&tq, q, D, N, B * Hq) || !encode_bhnd(&tk, k, D, N, B * Hkv) ||
-      !encode_bhnd(&tv, v, D, N, B * Hkv) || !encode_bhnd(&to, o, D, N, B * Hq, 32))
-    return ATTN_ERR_CUDA;
+                     int mask_kind, int window, float scale, int32_t* status, cudaStream_t stream,
+                     const PagedContext* ctx) {
+  CUtensorMap tq, tk, tv, to, tkr, tvr;
+  if (!encode_bhnd(&tq, q, D, N, B * Hq) || !encode_bhnd(&to, o, D, N, B * Hq, 32)) return ATTN_ERR_CUDA;
+  if (PAGED) {
+    if (!encode_pool(&tk, k, D, Hkv, ctx->block_size, ctx->num_blocks, ctx->block_size) ||
+        !encode_pool(&tv, v, D, Hkv, ctx->block_size, ctx->num_blocks, ctx->block_size) ||
+        !encode_pool(&tkr, k, D, Hkv, ctx->block_size, ctx->num_blocks, 1) ||
+        !encode_pool(&tvr, v, D, Hkv, ctx->block_size, ctx->num_blocks, 1))
+      return ATTN_ERR_CUDA;
+  } else {
+    if (!encode_bhnd(&tk, k, D, N, B * Hkv) || !encode_bhnd(&tv, v, D, N, B * Hkv)) return ATTN_ERR_CUDA;
+    tkr = tk;  // unused without a paged context
+    tvr = tv;
+  }
   PrefillParams p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -711,15 +822,22 @@ int launch_prefill_t(const void* q, const void* k, const void* v, void* o, float
   p.num_items = p.num_cta_tiles * Hq * B;
   p.scale_log2 = scale * kLog2e;
   p.budget = wait_budget_cycles();
+  p.block_table = PAGED ? ctx->block_table : nullptr;
+  p.seq_lens = PAGED ? ctx->seq_lens : nullptr;
+  p.max_blocks = PAGED ? ctx->max_blocks : 0;
+  p.block_size = PAGED ? ctx->block_size : 0;
+  p.num_blocks = PAGED ? ctx->num_blocks : 0;
+  p.max_seq_len = PAGED ? ctx->max_seq_len : N;
   constexpr int smem = PfCfg<D>::kAlloc;
-  if (cudaFuncSetAttribute(prefill_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(prefill_fwd_kernel<D, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
     return ATTN_ERR_CUDA;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
     return ATTN_ERR_CUDA;
   const dim3 grid(p.num_items < sms ? p.num_items : sms);  // persistent: one CTA per SM
-  prefill_fwd_kernel<D><<<grid, kPfThreads, smem, stream>>>(tq, tk, tv, to, p);
+  prefill_fwd_kernel<D, PAGED><<<grid, kPfThreads, smem, stream>>>(tq, tk, tv, to, tkr, tvr, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -727,8 +845,23 @@ int launch_prefill_t(const void* q, const void* k, const void* v, void* o, float
 
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
                    int d, int mask_kind, int window, float scale, int32_t* status, cudaStream_t stream) {
-  if (d == 128) return launch_prefill_t<128>(q, k, v, o, lse, B, Hq, Hkv, N, mask_kind, window, scale, status, stream);
-  return launch_prefill_t<64>(q, k, v, o, lse, B, Hq, Hkv, N, mask_kind, window, scale, status, stream);
+  if (d == 128)
+    return launch_prefill_t<128, false>(q, k, v, o, lse, B, Hq, Hkv, N, mask_kind, window, scale, status, stream,
+                                        nullptr);
+  return launch_prefill_t<64, false>(q, k, v, o, lse, B, Hq, Hkv, N, mask_kind, window, scale, status, stream,
+                                     nullptr);
+}
+
+int launch_prefill_paged(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                         const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int d,
+                         int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, int mask_kind,
+                         int window, float scale, int32_t* status, cudaStream_t stream) {
+  const PagedContext ctx{block_table, seq_lens, num_blocks, block_size, max_blocks_per_seq, max_seq_len};
+  if (d == 128)
+    return launch_prefill_t<128, true>(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Nq, mask_kind, window, scale, status,
+                                       stream, &ctx);
+  return launch_prefill_t<64, true>(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Nq, mask_kind, window, scale, status,
+                                    stream, &ctx);
 }
 
 }  // namespace attn

@@ -118,6 +118,37 @@ def paged_decode_inputs(B: int, Hq: int, Hkv: int, d: int, *, seq_lens=None, len
     return PagedDecodeInputs(q, k_cache, v_cache, table, seq_lens, block_size, int(max_seq_len), seed)
 
 
+@dataclasses.dataclass
+class PagedPrefillInputs:
+    q: torch.Tensor            # [B, Hq, Nq, d] bf16: the newest Nq positions of each sequence
+    k_cache: torch.Tensor      # [num_blocks, block_size, Hkv, d] bf16
+    v_cache: torch.Tensor
+    block_table: torch.Tensor  # [B, max_blocks] int32
+    seq_lens: torch.Tensor     # [B] int32, each >= Nq
+    block_size: int
+    max_seq_len: int
+    seed: int
+
+
+def paged_prefill_inputs(B: int, Hq: int, Hkv: int, Nq: int, d: int, *, seq_lens=None, len_range=None,
+                         block_size: int = 16, max_seq_len: int | None = None, seed: int = 0,
+                         extra_blocks: int = 0) -> PagedPrefillInputs:
+    """Same recipe as paged_decode_inputs, with Nq query rows per sequence."""
+    gen = torch.Generator("cpu").manual_seed(seed)
+    if seq_lens is None:
+        lo, hi = len_range
+        seq_lens = torch.randint(max(lo, Nq), hi + 1, (B,), generator=gen, dtype=torch.int64)
+    seq_lens = torch.as_tensor(seq_lens, dtype=torch.int32).reshape(B)
+    if max_seq_len is None:
+        max_seq_len = int(len_range[1]) if len_range is not None else int(seq_lens.max())
+    max_blocks = blocks_needed(max_seq_len, block_size)
+    table, pool = paged_layout(seq_lens.tolist(), block_size, max_blocks, gen, extra_blocks)
+    q = _normal_bf16((B, Hq, Nq, d), gen)
+    k_cache = _normal_bf16((pool, block_size, Hkv, d), gen)
+    v_cache = _normal_bf16((pool, block_size, Hkv, d), gen)
+    return PagedPrefillInputs(q, k_cache, v_cache, table, seq_lens, block_size, int(max_seq_len), seed)
+
+
 # Named workloads. Sizes follow the pages' shapes: Llama-style GQA-8
 # ("USAAIO Lesson 90", GQA part), 131,072-token contexts ("Modern Attention
 # Mechanisms", section 1) and 16-token blocks ("Module 09", "The Block Table").
@@ -129,6 +160,12 @@ PREFILL_WORKLOADS = {
     "gqa_dial_prefill_mha": dict(B=2, Hq=32, Hkv=32, N=8192, d=128, mask="causal", window=0),
     "gqa_dial_prefill_gqa8": dict(B=2, Hq=32, Hkv=8, N=8192, d=128, mask="causal", window=0),
     "gqa_dial_prefill_mqa": dict(B=2, Hq=32, Hkv=1, N=8192, d=128, mask="causal", window=0),
+}
+
+# Chunked prefill: 512 new tokens per sequence on top of a paged context.
+PAGED_PREFILL_WORKLOADS = {
+    "chunked_prefill_b4_q512": dict(B=4, Hq=32, Hkv=8, Nq=512, d=128, len_range=(4096, 16384), block_size=16,
+                                    mask="causal", window=0),
 }
 
 DECODE_WORKLOADS = {

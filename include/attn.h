@@ -99,6 +99,42 @@ ATTN_API int attn_prefill(const void* q, const void* k, const void* v, void* o, 
                  int N, int d, int mask_kind, int window, float scale, int32_t* status, attn_stream_t stream);
 
 /*
+ * attn_prefill_paged - prefix (chunked) prefill: the newest Nq positions of
+ * each sequence attend to its whole cached context, read through a block
+ * table.
+ *
+ * Positions are bottom-right aligned ("Modern Attention Mechanisms", section 4:
+ * after a prefix of length P, query row i has position P + i): sequence b has
+ * seq_lens[b] cached tokens (its Nq new tokens already appended, as in
+ * "Module 09: Efficient Attention", "Chunked Prefill"), so query row i sits at
+ * position seq_lens[b] - Nq + i. Key j is visible to it under CAUSAL iff
+ * j <= seq_lens[b] - Nq + i, under SLIDING_WINDOW iff additionally
+ * seq_lens[b] - Nq + i - j < window, under FULL iff j < seq_lens[b]. The cache
+ * layout and addressing are those of attn_decode_paged.
+ *
+ *   q            [B, Hq, Nq, d] bf16                        read
+ *   k_cache,
+ *   v_cache      [num_blocks, block_size, Hkv, d] bf16      read (only referenced slots)
+ *   block_table  [B, max_blocks_per_seq] int32              read: the entries covering
+ *                the keys each query row sees must lie in [0, num_blocks)
+ *   seq_lens     [B] int32, each in [Nq, max_seq_len]       read
+ *   o            [B, Hq, Nq, d] bf16                        written
+ *   lse          [B, Hq, Nq] fp32, natural log              written when non-NULL
+ *   block_size   16, 32, 64 or 128 (else ATTN_ERR_UNSUPPORTED)
+ *   max_seq_len  >= Nq and <= max_blocks_per_seq * block_size
+ *   status       device int32 or NULL.
+ *
+ * A seq_len outside [Nq, max_seq_len] or a needed block-table entry outside
+ * the pool is never dereferenced: that sequence's rows of o and lse are NaN
+ * and ATTN_STATUS_BIT_DEVICE_CHECK is OR-ed into *status. With seq_lens[b] ==
+ * Nq for every b and a contiguous block table this equals attn_prefill.
+ */
+ATTN_API int attn_prefill_paged(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                                const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int d,
+                                int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len,
+                                int mask_kind, int window, float scale, int32_t* status, attn_stream_t stream);
+
+/*
  * attn_decode_plan - the split-KV plan attn_decode_paged uses (host only, no
  * GPU needed). Long sequences are cut into chunks of *chunk_tokens tokens
  * (a multiple of 16); each (sequence, K/V head, chunk) is one unit of work

@@ -20,6 +20,7 @@ from .attention import (  # noqa: F401
     sdpa_rows,
     prefill_ref,
     prefill_rows_ref,
+    prefill_paged_ref,
     gather_paged_ref,
     decode_paged_ref,
     decode_rows_ref,

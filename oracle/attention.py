@@ -258,6 +258,37 @@ def decode_paged_ref(q, k_cache, v_cache, block_table, seq_lens, scale: float):
     return out, lse
 
 
+def prefill_paged_ref(q, k_cache, v_cache, block_table, seq_lens, mask_kind: int, window: int, scale: float,
+                      seqs=None):
+    """Prefix prefill over a paged context: the definition composed of two
+    pinned pieces.
+
+    Module 09: Efficient Attention, "Chunked Prefill": a prompt is processed in
+    chunks, each chunk's queries attending to everything cached before it and to
+    itself. Sequence b's keys are its seq_lens[b] cached tokens, gathered token
+    by token through its block table (gather_paged_ref); its Nq query rows are
+    the newest Nq positions (Modern Attention Mechanisms, section 4: after a
+    prefix of length P, query row i has position P + i), which allowed_mask
+    applies when n_q < n_k. q [B, Hq, Nq, d]. Returns (O [B, Hq, Nq, d],
+    LSE [B, Hq, Nq]) for the sequences in `seqs` (all when None; others zero).
+    """
+    q = _as_f64(q)
+    lens = _as_int(seq_lens)
+    b_, hq, n_q, d = q.shape
+    seqs = range(b_) if seqs is None else seqs
+    out = np.zeros((b_, hq, n_q, d), dtype=np.float64)
+    lse = np.zeros((b_, hq, n_q), dtype=np.float64)
+    table = _as_int(block_table)
+    for bi in seqs:
+        n_k = int(lens[bi])
+        kb = gather_paged_ref(k_cache, table[bi:bi + 1], lens[bi:bi + 1], n_k)
+        vb = gather_paged_ref(v_cache, table[bi:bi + 1], lens[bi:bi + 1], n_k)
+        o_b, l_b = prefill_ref(q[bi:bi + 1], kb, vb, mask_kind, window, scale)
+        out[bi] = o_b[0]
+        lse[bi] = l_b[0]
+    return out, lse
+
+
 def lse_merge_ref(o_parts, lse_parts):
     """Combine per-chunk partial results into the full softmax result.
 

@@ -93,6 +93,31 @@ def test_decode_rejects_bad_arguments(kw, code):
     assert _decode(**kw) == code
 
 
+def _prefill_paged(**kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, sl=FAKE, o=FAKE, lse=NULL, B=2, Hq=8, Hkv=2, Nq=64, d=128, nb=10,
+             bs=16, mb=8, msl=128, mask=1, window=0, scale=0.1)
+    a.update(kw)
+    return _lib.lib().attn_prefill_paged(a["q"], a["kc"], a["vc"], a["bt"], a["sl"], a["o"], a["lse"], a["B"],
+                                         a["Hq"], a["Hkv"], a["Nq"], a["d"], a["nb"], a["bs"], a["mb"], a["msl"],
+                                         a["mask"], a["window"], a["scale"], NULL, NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(sl=NULL), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(Nq=0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(msl=32), _lib.ATTN_ERR_INVALID_ARG),   # max_seq_len < Nq
+    (dict(mb=7), _lib.ATTN_ERR_INVALID_ARG),     # 7 blocks of 16 cannot hold 128 tokens
+    (dict(Hq=6, Hkv=4), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(mask=2, window=0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(q=ctypes.c_void_p(0x10004)), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(d=96), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(bs=8, mb=16), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(bs=48, mb=3, msl=128), _lib.ATTN_ERR_UNSUPPORTED),
+])
+def test_prefill_paged_rejects_bad_arguments(kw, code):
+    assert _prefill_paged(**kw) == code
+
+
 def test_gather_rejects_bad_arguments():
     lib = _lib.lib()
     assert lib.attn_paged_gather(NULL, FAKE, FAKE, FAKE, 1, 1, 64, 4, 16, 2, 32, NULL, NULL) == _lib.ATTN_ERR_INVALID_ARG

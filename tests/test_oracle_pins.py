@@ -471,3 +471,40 @@ def test_planted_wrong_window_is_caught(monkeypatch):
     o, _ = oa.prefill_ref(q, k, v, oracle.MASK_SLIDING_WINDOW, 3, 0.5)
     o_ref, _ = _brute_force(q, k, v, oracle.MASK_SLIDING_WINDOW, 3, 0.5)
     assert np.max(np.abs(o - o_ref)) > 1e-3
+
+
+# --------------------------------------------------------------------------
+# prefix (chunked) prefill over a paged context
+# --------------------------------------------------------------------------
+def test_paged_prefill_square_case_is_prefill():
+    """seq_len == Nq: the chunk is the whole sequence, so the paged prefix
+    prefill is the plain prefill of the gathered cache."""
+    rng = np.random.default_rng(31)
+    Hq, Hkv, N, d, bs = 4, 2, 9, 6, 4
+    q = rng.standard_normal((1, Hq, N, d))
+    k = rng.standard_normal((1, Hkv, N, d))
+    v = rng.standard_normal((1, Hkv, N, d))
+    kc, vc, table, sl = _paged_from_contiguous([k[0].transpose(1, 0, 2)], [v[0].transpose(1, 0, 2)], bs, 5)
+    for kind, w in [(oracle.MASK_CAUSAL, 0), (oracle.MASK_FULL, 0), (oracle.MASK_SLIDING_WINDOW, 3)]:
+        o_p, l_p = oracle.prefill_paged_ref(q, kc, vc, table, sl, kind, w, 0.4)
+        o_c, l_c = oracle.prefill_ref(q, k, v, kind, w, 0.4)
+        assert np.array_equal(o_p, o_c) and np.array_equal(l_p, l_c)
+
+
+@pytest.mark.parametrize("kind,w", [(oracle.MASK_CAUSAL, 0), (oracle.MASK_SLIDING_WINDOW, 4)])
+def test_chunked_prefill_equals_full_forward(kind, w):
+    """Module 09, "Chunked Prefill": slicing a prompt into chunks changes the
+    schedule, never the result. Chunk c's rows, attending to every position up
+    to the chunk's end, equal the same rows of the one-shot prefill."""
+    rng = np.random.default_rng(37)
+    Hq, Hkv, N, d, bs = 2, 1, 13, 5, 4
+    q = rng.standard_normal((1, Hq, N, d))
+    k = rng.standard_normal((1, Hkv, N, d))
+    v = rng.standard_normal((1, Hkv, N, d))
+    o_full, l_full = oracle.prefill_ref(q, k, v, kind, w, 0.5)
+    for a, b in [(0, 5), (5, 6), (6, 13)]:
+        kc, vc, table, sl = _paged_from_contiguous([k[0, :, :b].transpose(1, 0, 2)],
+                                                   [v[0, :, :b].transpose(1, 0, 2)], bs, b)
+        o_c, l_c = oracle.prefill_paged_ref(q[:, :, a:b], kc, vc, table, sl, kind, w, 0.5)
+        np.testing.assert_allclose(o_c[0], o_full[0, :, a:b], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(l_c[0], l_full[0, :, a:b], rtol=0, atol=1e-13)
