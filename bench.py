@@ -378,6 +378,104 @@ def run_ours(args, pcfg, dcfg):
     return 0
 
 
+def run_single_op(args):
+    """Time one entry point on one named workload; one JSON line with its roofline.
+
+    prefill (TFLOP/s, tensor roofline), prefill_paged (TFLOP/s over the visible
+    pairs of each chunk against its context), decode (KV GB/s, HBM roofline).
+    L2 is flushed before every timed launch; CUDA events on the launching stream.
+    """
+    import exact_softmax_attention_causal_b200 as attn
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    seed = sharding.rank_seed(args.seed, rank)
+    peaks = measured_peaks()
+    tag = "of measured" if peaks["source"] == "measured" else "of fallback"
+    name = args.workload
+    if args.op == "prefill":
+        cfg = workloads.PREFILL_WORKLOADS[name]
+        x = workloads.prefill_inputs(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["N"], cfg["d"], seed)
+        q, k, v = x.q.to(dev), x.k.to(dev), x.v.to(dev)
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        work = accounting.prefill_flops(cfg["B"], cfg["Hq"], cfg["N"], cfg["d"], cfg["mask"], cfg["window"])
+
+        def launch():
+            attn.prefill(q, k, v, mask=cfg["mask"], window=cfg["window"], out=o, lse=lse)
+        unit, bound, peak, scale_div = "TFLOP/s", "tensor", peaks["bf16_tflops"], 1e12
+        metric = "prefill TFLOP/s (visible pairs)"
+    elif args.op == "prefill_paged":
+        cfg = dict(workloads.PAGED_PREFILL_WORKLOADS[name])
+        mask, window = cfg.pop("mask"), cfg.pop("window")
+        B, Hq, Hkv, Nq, d = (cfg.pop(kk) for kk in ("B", "Hq", "Hkv", "Nq", "d"))
+        x = workloads.paged_prefill_inputs(B, Hq, Hkv, Nq, d, seed=seed, **cfg)
+        q, kc, vc = x.q.to(dev), x.k_cache.to(dev), x.v_cache.to(dev)
+        bt, sl = x.block_table.to(dev), x.seq_lens.to(dev)
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        work = accounting.prefill_paged_flops(x.seq_lens.tolist(), Nq, Hq, d, mask, window)
+        msl = x.max_seq_len
+
+        def launch():
+            attn.prefill_paged(q, kc, vc, bt, sl, msl, mask=mask, window=window, out=o, lse=lse)
+        unit, bound, peak, scale_div = "TFLOP/s", "tensor", peaks["bf16_tflops"], 1e12
+        metric = "chunked prefill TFLOP/s (visible pairs)"
+        cfg = dict(workloads.PAGED_PREFILL_WORKLOADS[name])
+    else:
+        cfg = dict(workloads.DECODE_WORKLOADS[name])
+        x = workloads.paged_decode_inputs(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"], len_range=cfg.get("len_range"),
+                                          seq_lens=cfg.get("seq_lens"), block_size=cfg["block_size"], seed=seed)
+        q, kc, vc = x.q.to(dev), x.k_cache.to(dev), x.v_cache.to(dev)
+        bt, sl = x.block_table.to(dev), x.seq_lens.to(dev)
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+        ws = torch.empty(attn.decode_workspace_bytes(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"], x.max_seq_len,
+                                                     x.block_size), dtype=torch.uint8, device=dev)
+        work = accounting.decode_kv_bytes(x.seq_lens.tolist(), cfg["Hkv"], cfg["d"])
+        msl = x.max_seq_len
+
+        def launch():
+            attn.decode_paged(q, kc, vc, bt, sl, msl, out=o, lse=lse, workspace=ws)
+        unit, bound, peak, scale_div = "GB/s", "hbm", peaks["hbm_gbs"], 1e9
+        metric = "paged-decode KV GB/s"
+    del x
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            launch()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        for e0, e1 in events:
+            flush.fill_(1)
+            e0.record()
+            launch()
+            e1.record()
+        torch.cuda.synchronize()
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in events)
+    (ms_max,) = sharding.max_over_ranks([ms], device=dev)
+    achieved = work / (ms / args.steps / 1e3) / scale_div
+    if rank == 0:
+        line = {
+            "metric": metric, "value": sharding.job_throughput(work, world, args.steps, ms_max) / scale_div,
+            "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic", "op": args.op,
+            "config": dict(workload=name, **{kk: vv for kk, vv in cfg.items()},
+                           l2="flushed (256 MiB write) before every timed launch"),
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                         "traffic": None, "peak_source": tag},
+            "work_per_launch": work, "gpu_launches": args.steps * (2 if args.op == "decode" else 1),
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def dcfg_max_len(dcfg):
     if dcfg.get("len_range") is not None:
         return int(dcfg["len_range"][1])
@@ -390,7 +488,11 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama3_8b_causal_gqa", choices=sorted(workloads.PREFILL_WORKLOADS))
+    ap.add_argument("--op", choices=["step", "prefill", "prefill_paged", "decode"], default="step",
+                    help="step: the full hot-path step (default); otherwise time one entry point on --workload")
+    ap.add_argument("--workload", default=None,
+                    choices=sorted(list(workloads.PREFILL_WORKLOADS) + list(workloads.PAGED_PREFILL_WORKLOADS) +
+                                   list(workloads.DECODE_WORKLOADS)))
     ap.add_argument("--decode-workload", default="paged_decode_b64", choices=sorted(workloads.DECODE_WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -399,6 +501,30 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.op != "step":
+        defaults = {"prefill": "llama3_8b_causal_gqa", "prefill_paged": "chunked_prefill_b4_q512",
+                    "decode": "paged_decode_b64"}
+        args.workload = args.workload or defaults[args.op]
+        table = {"prefill": workloads.PREFILL_WORKLOADS, "prefill_paged": workloads.PAGED_PREFILL_WORKLOADS,
+                 "decode": workloads.DECODE_WORKLOADS}[args.op]
+        if args.workload not in table:
+            ap.error(f"--workload {args.workload} is not a {args.op} workload")
+        if args.impl == "reference":
+            ap.error("--op is only for the CUDA path")
+        world, _, _ = dist_env()
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                    device_id=torch.device("cuda", dist_env()[2]))
+            try:
+                return run_single_op(args)
+            finally:
+                dist.destroy_process_group()
+        return run_single_op(args)
+    args.workload = args.workload or "llama3_8b_causal_gqa"
+    if args.workload not in workloads.PREFILL_WORKLOADS:
+        ap.error("the full step takes a prefill workload")
     pcfg = dict(workloads.PREFILL_WORKLOADS[args.workload], name=args.workload)
     dcfg = dict(workloads.DECODE_WORKLOADS[args.decode_workload], name=args.decode_workload)
     world, _, _ = dist_env()

@@ -42,3 +42,24 @@ def decode_io_bytes(seq_lens, B: int, Hq: int, Hkv: int, d: int, block_size: int
     """KV bytes plus q, o, lse, block-table and seq_len bytes."""
     tables = sum(-(-int(n) // block_size) for n in seq_lens) * 4 + 4 * B
     return decode_kv_bytes(seq_lens, Hkv, d) + B * Hq * d * 2 * 2 + B * Hq * 4 + tables
+
+
+def prefix_visible_pairs(n_k: int, n_q: int, mask: str, window: int = 0) -> int:
+    """Visible (query, key) pairs when the n_q query rows are the newest of n_k
+    positions (row i at position n_k - n_q + i)."""
+    p0 = n_k - n_q
+    if mask == "full":
+        return n_q * n_k
+    # row i sees min(p0 + i + 1, w) keys (causal: w = infinity)
+    w = n_k if mask == "causal" else min(int(window), n_k)
+    first, last = p0 + 1, p0 + n_q  # keys seen by the first and last rows before the window cap
+    if last <= w:
+        return (first + last) * n_q // 2
+    if first >= w:
+        return w * n_q
+    below = w - first  # rows whose count is still below the cap
+    return (first + w - 1) * below // 2 + w * (n_q - below)
+
+
+def prefill_paged_flops(seq_lens, n_q: int, Hq: int, d: int, mask: str, window: int = 0) -> int:
+    return 4 * Hq * d * sum(prefix_visible_pairs(int(n), n_q, mask, window) for n in seq_lens)

@@ -508,3 +508,11 @@ def test_chunked_prefill_equals_full_forward(kind, w):
         o_c, l_c = oracle.prefill_paged_ref(q[:, :, a:b], kc, vc, table, sl, kind, w, 0.5)
         np.testing.assert_allclose(o_c[0], o_full[0, :, a:b], rtol=0, atol=1e-13)
         np.testing.assert_allclose(l_c[0], l_full[0, :, a:b], rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("n_k,n_q,mask,w", [(10, 10, "causal", 0), (10, 3, "causal", 0), (300, 77, "full", 0),
+                                            (300, 77, "window", 100), (300, 77, "window", 250), (300, 77, "window", 5),
+                                            (77, 77, "window", 1000), (5, 1, "window", 2)])
+def test_prefix_visible_pairs_closed_form(n_k, n_q, mask, w):
+    kind = accounting.MASK_IDS[mask]
+    assert accounting.prefix_visible_pairs(n_k, n_q, mask, w) == int(oracle.allowed_mask(n_q, n_k, kind, w).sum())
