@@ -5,7 +5,8 @@ p*v per pair, so 4 * d per pair per query head. Visible pairs per head:
 full N^2, causal N(N+1)/2, window sum_i min(i+1, w).
 
 Decode bytes count the K and V bytes a step must read from HBM:
-sum_b seq_len_b * Hkv * d * 2 (K and V) * 2 (bf16).
+sum_b seq_len_b * Hkv * d * 2 (K and V) * 2 (bf16). A windowed decode reads
+only the visible tokens: the last W positions plus the first n_sink ones.
 """
 
 from __future__ import annotations
@@ -63,3 +64,18 @@ def prefix_visible_pairs(n_k: int, n_q: int, mask: str, window: int = 0) -> int:
 
 def prefill_paged_flops(seq_lens, n_q: int, Hq: int, d: int, mask: str, window: int = 0) -> int:
     return 4 * Hq * d * sum(prefix_visible_pairs(int(n), n_q, mask, window) for n in seq_lens)
+
+
+def decode_visible_tokens(n: int, window: int = 0, n_sink: int = 0) -> int:
+    """Tokens a decode query at position n - 1 sees: all n without a window;
+    with window W the positions max(0, n - W) .. n - 1 plus the sink positions
+    below that start (at most n_sink of them)."""
+    n = int(n)
+    if window <= 0:
+        return n
+    lo = max(0, n - int(window))
+    return min(int(n_sink), lo) + (n - lo)
+
+
+def decode_window_kv_bytes(seq_lens, Hkv: int, d: int, window: int = 0, n_sink: int = 0) -> int:
+    return sum(decode_visible_tokens(n, window, n_sink) for n in seq_lens) * Hkv * d * 2 * 2

@@ -14,6 +14,8 @@ Recipe (all on the CPU, ``torch.Generator('cpu').manual_seed(seed)``):
   entries past a sequence's last block are -1. Then Q [B, Hq, d], the K pool
   and the V pool [num_blocks, block_size, Hkv, d], each float32 normal rounded
   to bf16. Large tensors are drawn in chunks of 2**24 elements, in order.
+  With learned sinks, one float32 logit per query head is drawn last,
+  uniform in [-1, 6) (the pages' examples use s = 0, 2, 5).
 
 Paged layout: Module 09: Efficient Attention, "The Block Table" and "Code: A
 Paged KV Cache from Scratch" (pool (num_blocks, block_size, num_kv_heads,
@@ -73,6 +75,7 @@ class PagedDecodeInputs:
     block_size: int
     max_seq_len: int
     seed: int
+    sinks: torch.Tensor | None = None  # [Hq] float32 learned sink logits
 
     @property
     def num_blocks(self) -> int:
@@ -102,7 +105,7 @@ def paged_layout(seq_lens, block_size: int, max_blocks: int, gen: torch.Generato
 
 def paged_decode_inputs(B: int, Hq: int, Hkv: int, d: int, *, seq_lens=None, len_range=None,
                         block_size: int = 16, max_seq_len: int | None = None, seed: int = 0,
-                        extra_blocks: int = 0) -> PagedDecodeInputs:
+                        extra_blocks: int = 0, learned_sinks: bool = False) -> PagedDecodeInputs:
     gen = torch.Generator("cpu").manual_seed(seed)
     if seq_lens is None:
         lo, hi = len_range
@@ -115,7 +118,10 @@ def paged_decode_inputs(B: int, Hq: int, Hkv: int, d: int, *, seq_lens=None, len
     q = _normal_bf16((B, Hq, d), gen)
     k_cache = _normal_bf16((pool, block_size, Hkv, d), gen)
     v_cache = _normal_bf16((pool, block_size, Hkv, d), gen)
-    return PagedDecodeInputs(q, k_cache, v_cache, table, seq_lens, block_size, int(max_seq_len), seed)
+    sinks = None
+    if learned_sinks:
+        sinks = torch.rand(Hq, generator=gen, dtype=torch.float32) * 7.0 - 1.0
+    return PagedDecodeInputs(q, k_cache, v_cache, table, seq_lens, block_size, int(max_seq_len), seed, sinks)
 
 
 @dataclasses.dataclass
@@ -173,6 +179,20 @@ DECODE_WORKLOADS = {
     "gqa_dial_decode_mha": dict(B=1, Hq=32, Hkv=32, d=128, seq_lens=[131072], block_size=16),
     "gqa_dial_decode_gqa8": dict(B=1, Hq=32, Hkv=8, d=128, seq_lens=[131072], block_size=16),
     "gqa_dial_decode_mqa": dict(B=1, Hq=32, Hkv=1, d=128, seq_lens=[131072], block_size=16),
+}
+
+# Windowed decode with sinks. gpt-oss-120b shapes ("Modern Attention
+# Mechanisms", the gpt-oss walk-through: 64 query heads over 8 K/V heads,
+# head_dim 64, window 128 on the local layers, full causal on the others, one
+# learned sink logit per head) and a StreamingLLM-style cache (window 4096, as
+# in Mistral-7B-v0.1, plus the first 4 positions kept as sinks).
+WINDOW_DECODE_WORKLOADS = {
+    "gptoss_window128_sinks_b64": dict(B=64, Hq=64, Hkv=8, d=64, len_range=(1024, 32768), block_size=16,
+                                       window=128, n_sink=0, learned_sinks=True),
+    "gptoss_full_sinks_b64": dict(B=64, Hq=64, Hkv=8, d=64, len_range=(1024, 32768), block_size=16,
+                                  window=0, n_sink=0, learned_sinks=True),
+    "streaming_window4096_nsink4_b64": dict(B=64, Hq=32, Hkv=8, d=128, len_range=(8192, 32768), block_size=16,
+                                            window=4096, n_sink=4, learned_sinks=False),
 }
 
 

@@ -25,6 +25,11 @@ Sources (page title, section):
 * "Inference attention" post (brunomaga.github.io), section "FlashDecoding":
   partial outputs of key chunks with their softmax statistics, combined with
   the online softmax's rescaling.
+* "Module 5. Modern Attention Mechanisms", section 10 "Attention sink refers
+  to two different objects" and section 12 (its mask builder and SDPA): the
+  StreamingLLM rule that keeps the first n_sink real positions visible next
+  to a finite window, and the learned per-head sink logit s_h, an extra score
+  column that takes softmax mass but adds no value vector.
 
 The oracle computes a DIRECT softmax: it materialises full score rows (in
 row blocks only to bound memory), applies the mask, subtracts the row max,
@@ -35,7 +40,9 @@ widened exactly to float64 and everything after that is float64.
 
 LSE is the natural-log log-sum-exp over the visible keys of the scaled scores,
 log(sum_j exp(scale * q.k_j)): the "running log-sum-exp" the slides name,
-written as m + log(l) in the online softmax's notation.
+written as m + log(l) in the online softmax's notation. With a learned sink
+the row that is normalised has one more column, so LSE includes it:
+log(sum_j exp(scale * q.k_j) + exp(s_h)) (the log of the softmax denominator).
 """
 
 from __future__ import annotations
@@ -67,7 +74,7 @@ def _as_int(x) -> np.ndarray:
     return np.asarray(x, dtype=np.int64)
 
 
-def allowed_mask(n_q: int, n_k: int, mask_kind: int, window: int = 0, rows=None) -> np.ndarray:
+def allowed_mask(n_q: int, n_k: int, mask_kind: int, window: int = 0, rows=None, n_sink: int = 0) -> np.ndarray:
     """Boolean [n_q, n_k] visibility, True = query row i may attend key j.
 
     Modern Attention Mechanisms, section 4: causality compares positions,
@@ -76,9 +83,18 @@ def allowed_mask(n_q: int, n_k: int, mask_kind: int, window: int = 0, rows=None)
     position P + i (keys sit at positions 0..n_k-1). For the square case
     (n_q == n_k) this is j <= i and i - W < j <= i. ``rows`` restricts the
     result to those query rows (all rows when None).
+
+    Section 10 / section 12 (StreamingLLM sinks): with a finite window, the
+    first ``n_sink`` positions stay visible to every query at or after them,
+    p_k < n_sink and p_k <= p_q. n_sink is accepted only with the window mask
+    and must lie in [0, n_k].
     """
     if n_q <= 0 or n_k <= 0 or n_q > n_k:
         raise ValueError("need 0 < n_q <= n_k")
+    if n_sink < 0 or n_sink > n_k:
+        raise ValueError("n_sink must satisfy 0 <= n_sink <= n_k")
+    if n_sink and mask_kind != MASK_SLIDING_WINDOW:
+        raise ValueError("n_sink is meaningful only together with a finite window")
     rows = np.arange(n_q) if rows is None else np.asarray(rows, dtype=np.int64)
     p_q = (n_k - n_q) + rows[:, None]
     p_k = np.arange(n_k)[None, :]
@@ -90,16 +106,23 @@ def allowed_mask(n_q: int, n_k: int, mask_kind: int, window: int = 0, rows=None)
         if window <= 0:
             raise ValueError("window must be positive")
         diff = p_q - p_k
-        return (diff >= 0) & (diff < window)
+        allowed = (diff >= 0) & (diff < window)
+        return allowed | ((p_k < n_sink) & (p_k <= p_q))
     raise ValueError(f"unknown mask kind {mask_kind}")
 
 
-def sdpa_rows(q_rows, k, v, allowed, scale: float):
+def sdpa_rows(q_rows, k, v, allowed, scale: float, sink=None):
     """Direct softmax attention of some query rows against one K/V head.
 
     Modern Attention Mechanisms, section 4 (the SDPA definition and the
     additive -inf mask) and section 12 (subtract the row maximum, exponentiate,
     normalise; a row with no visible key is rejected, the "error" policy).
+
+    ``sink`` (a finite scalar or one value per row) is section 10's learned
+    sink logit: one more score column, in the units of the scaled scores,
+    that enters the row maximum and the denominator and is dropped before the
+    product with V. With a sink a row without visible keys is well defined
+    (all mass on the sink: O = 0, LSE = sink).
 
     q_rows [R, d], k [T, d], v [T, d_v], allowed [R, T] bool.
     Returns (O [R, d_v], LSE [R]) in float64.
@@ -108,14 +131,24 @@ def sdpa_rows(q_rows, k, v, allowed, scale: float):
     k = _as_f64(k)
     v = _as_f64(v)
     allowed = np.asarray(allowed, dtype=bool)
-    if not allowed.any(axis=1).all():
-        bad = np.nonzero(~allowed.any(axis=1))[0][:8].tolist()
+    has_key = allowed.any(axis=1)
+    if sink is None and not has_key.all():
+        bad = np.nonzero(~has_key)[0][:8].tolist()
         raise ValueError(f"fully masked rows: {bad}")
     scores = (q_rows @ k.T) * float(scale)
     scores = np.where(allowed, scores, -np.inf)
-    row_max = scores.max(axis=1)
+    token_max = scores.max(axis=1)  # -inf on a row without keys
+    if sink is None:
+        row_max = token_max
+    else:
+        sink = np.broadcast_to(_as_f64(sink), token_max.shape)
+        if not np.isfinite(sink).all():
+            raise ValueError("sink logits must be finite")
+        row_max = np.maximum(token_max, sink)
     e = np.exp(scores - row_max[:, None])  # exp(-inf) == 0 for masked keys
     denom = e.sum(axis=1)
+    if sink is not None:
+        denom = denom + np.exp(sink - row_max)
     out = (e / denom[:, None]) @ v
     lse = row_max + np.log(denom)
     return out, lse
@@ -216,14 +249,19 @@ def _gather_one(cache, table_row, n: int) -> np.ndarray:
     return rows
 
 
-def decode_rows_ref(q, k_cache, v_cache, block_table, seq_lens, b: int, heads, scale: float):
-    """One decode query per head of sequence b against its whole paged cache.
+def decode_rows_ref(q, k_cache, v_cache, block_table, seq_lens, b: int, heads, scale: float, window: int = 0,
+                    n_sink: int = 0, sinks=None):
+    """One decode query per head of sequence b against its paged cache.
 
-    USAAIO Lesson 90, part 2: the new query attends over all cached keys and
-    values (its own already appended), so no mask applies. K/V are gathered
-    through the block table (Module 09, paged cache section) and the direct
-    softmax of sdpa_rows does the rest. q [B, Hq, d]; caches
-    [num_blocks, block_size, Hkv, d]. Returns (O [len(heads), d], LSE [len(heads)]).
+    USAAIO Lesson 90, part 2: the new query attends over the cached keys and
+    values (its own already appended), so it sits at position n - 1. K/V are
+    gathered through the block table (Module 09, paged cache section) and the
+    direct softmax of sdpa_rows does the rest. Without a window every cached
+    token is visible; with ``window`` = W > 0 the query sees the positions
+    n - W .. n - 1 plus the first ``n_sink`` (allowed_mask with n_q = 1).
+    ``sinks`` [Hq] holds each query head's learned sink logit (or None).
+    q [B, Hq, d]; caches [num_blocks, block_size, Hkv, d].
+    Returns (O [len(heads), d], LSE [len(heads)]).
     """
     hq = q.shape[1]
     hkv = k_cache.shape[2]
@@ -231,28 +269,34 @@ def decode_rows_ref(q, k_cache, v_cache, block_table, seq_lens, b: int, heads, s
     n = int(_as_int(seq_lens)[b])
     if n <= 0:
         raise ValueError("a decode row needs at least one cached token")
+    kind = MASK_SLIDING_WINDOW if window > 0 else MASK_CAUSAL
+    allowed = allowed_mask(1, n, kind, window, n_sink=min(int(n_sink), n))
     kc = _as_f64(k_cache)
     vc = _as_f64(v_cache)
     row = _as_int(block_table)[b]
     k_seq = _gather_one(kc, row, n)
     v_seq = _gather_one(vc, row, n)
     qb = _as_f64(q[b])
+    sk = None if sinks is None else _as_f64(sinks)
     outs, lses = [], []
     for h in heads:
         kvh = kv_head_of(h, hq, hkv)
-        o, l = sdpa_rows(qb[h][None, :], k_seq[:, kvh], v_seq[:, kvh], np.ones((1, n), dtype=bool), scale)
+        o, l = sdpa_rows(qb[h][None, :], k_seq[:, kvh], v_seq[:, kvh], allowed, scale,
+                         sink=None if sk is None else sk[h])
         outs.append(o[0])
         lses.append(l[0])
     return np.stack(outs), np.asarray(lses)
 
 
-def decode_paged_ref(q, k_cache, v_cache, block_table, seq_lens, scale: float):
+def decode_paged_ref(q, k_cache, v_cache, block_table, seq_lens, scale: float, window: int = 0, n_sink: int = 0,
+                     sinks=None):
     """Paged decode for every sequence and head: (O [B, Hq, d], LSE [B, Hq])."""
     b_, hq = q.shape[0], q.shape[1]
     out = np.empty((b_, hq, q.shape[2]), dtype=np.float64)
     lse = np.empty((b_, hq), dtype=np.float64)
     for bi in range(b_):
-        o, l = decode_rows_ref(q, k_cache, v_cache, block_table, seq_lens, bi, range(hq), scale)
+        o, l = decode_rows_ref(q, k_cache, v_cache, block_table, seq_lens, bi, range(hq), scale, window, n_sink,
+                               sinks)
         out[bi] = o
         lse[bi] = l
     return out, lse
