@@ -382,7 +382,8 @@ def run_single_op(args):
     """Time one entry point on one named workload; one JSON line with its roofline.
 
     prefill (TFLOP/s, tensor roofline), prefill_paged (TFLOP/s over the visible
-    pairs of each chunk against its context), decode (KV GB/s, HBM roofline).
+    pairs of each chunk against its context), decode (KV GB/s, HBM roofline),
+    decode_window (GB/s of the K/V bytes of the visible tokens only).
     L2 is flushed before every timed launch; CUDA events on the launching stream.
     """
     import exact_softmax_attention_causal_b200 as attn
@@ -423,6 +424,27 @@ def run_single_op(args):
         unit, bound, peak, scale_div = "TFLOP/s", "tensor", peaks["bf16_tflops"], 1e12
         metric = "chunked prefill TFLOP/s (visible pairs)"
         cfg = dict(workloads.PAGED_PREFILL_WORKLOADS[name])
+    elif args.op == "decode_window":
+        cfg = dict(workloads.WINDOW_DECODE_WORKLOADS[name])
+        x = workloads.paged_decode_inputs(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"], len_range=cfg.get("len_range"),
+                                          seq_lens=cfg.get("seq_lens"), block_size=cfg["block_size"], seed=seed,
+                                          learned_sinks=cfg["learned_sinks"])
+        q, kc, vc = x.q.to(dev), x.k_cache.to(dev), x.v_cache.to(dev)
+        bt, sl = x.block_table.to(dev), x.seq_lens.to(dev)
+        sinks = None if x.sinks is None else x.sinks.to(dev)
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+        win, n_sink = cfg["window"], cfg["n_sink"]
+        ws = torch.empty(attn.decode_window_workspace_bytes(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"], x.max_seq_len,
+                                                            x.block_size, win, n_sink), dtype=torch.uint8, device=dev)
+        work = accounting.decode_window_kv_bytes(x.seq_lens.tolist(), cfg["Hkv"], cfg["d"], win, n_sink)
+        msl = x.max_seq_len
+
+        def launch():
+            attn.decode_paged_window(q, kc, vc, bt, sl, msl, window=win, n_sink=n_sink, sinks=sinks, out=o, lse=lse,
+                                     workspace=ws)
+        unit, bound, peak, scale_div = "GB/s", "hbm", peaks["hbm_gbs"], 1e9
+        metric = "windowed paged-decode KV GB/s (visible tokens)"
     else:
         cfg = dict(workloads.DECODE_WORKLOADS[name])
         x = workloads.paged_decode_inputs(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"], len_range=cfg.get("len_range"),
@@ -469,7 +491,7 @@ def run_single_op(args):
                            l2="flushed (256 MiB write) before every timed launch"),
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                          "traffic": None, "peak_source": tag},
-            "work_per_launch": work, "gpu_launches": args.steps * (2 if args.op == "decode" else 1),
+            "work_per_launch": work, "gpu_launches": args.steps * (2 if args.op.startswith("decode") else 1),
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
@@ -488,11 +510,11 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["step", "prefill", "prefill_paged", "decode"], default="step",
+    ap.add_argument("--op", choices=["step", "prefill", "prefill_paged", "decode", "decode_window"], default="step",
                     help="step: the full hot-path step (default); otherwise time one entry point on --workload")
     ap.add_argument("--workload", default=None,
                     choices=sorted(list(workloads.PREFILL_WORKLOADS) + list(workloads.PAGED_PREFILL_WORKLOADS) +
-                                   list(workloads.DECODE_WORKLOADS)))
+                                   list(workloads.DECODE_WORKLOADS) + list(workloads.WINDOW_DECODE_WORKLOADS)))
     ap.add_argument("--decode-workload", default="paged_decode_b64", choices=sorted(workloads.DECODE_WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -503,10 +525,10 @@ def main(argv=None):
         ap.error("--warmup must be at least 3")
     if args.op != "step":
         defaults = {"prefill": "llama3_8b_causal_gqa", "prefill_paged": "chunked_prefill_b4_q512",
-                    "decode": "paged_decode_b64"}
+                    "decode": "paged_decode_b64", "decode_window": "gptoss_window128_sinks_b64"}
         args.workload = args.workload or defaults[args.op]
         table = {"prefill": workloads.PREFILL_WORKLOADS, "prefill_paged": workloads.PAGED_PREFILL_WORKLOADS,
-                 "decode": workloads.DECODE_WORKLOADS}[args.op]
+                 "decode": workloads.DECODE_WORKLOADS, "decode_window": workloads.WINDOW_DECODE_WORKLOADS}[args.op]
         if args.workload not in table:
             ap.error(f"--workload {args.workload} is not a {args.op} workload")
         if args.impl == "reference":

@@ -1,7 +1,9 @@
 """Exact softmax attention for NVIDIA B200 (sm_100a).
 
-Causal / sliding-window / full grouped-query prefill and paged single-token
-decode, computed by hand-written CUDA kernels behind the C ABI of
+Causal / sliding-window / full grouped-query prefill (contiguous, or the
+newest positions against a paged context) and paged single-token decode (whole
+cache, or a sliding window with sink positions and learned sink logits),
+computed by hand-written CUDA kernels behind the C ABI of
 ``include/attn.h``. This module is the thin Python binding: it checks tensor
 dtypes, shapes and devices, allocates outputs with PyTorch (device memory
 plumbing only) and passes raw pointers and the current CUDA stream to the
@@ -21,8 +23,8 @@ from ._lib import AttnError, STATUS_BIT_DEVICE_CHECK, STATUS_BIT_TIMEOUT  # noqa
 
 MASKS = {"full": 0, "causal": 1, "window": 2, "sliding_window": 2}
 
-__all__ = ["prefill", "prefill_paged", "decode_paged", "paged_gather", "decode_plan", "decode_workspace_bytes", "AttnError",
-           "version"]
+__all__ = ["prefill", "prefill_paged", "decode_paged", "decode_paged_window", "paged_gather", "decode_plan",
+           "decode_workspace_bytes", "decode_window_workspace_bytes", "AttnError", "version"]
 
 
 def version() -> int:
@@ -166,6 +168,56 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int, s
                                       workspace.numel() * workspace.element_size(), _ptr(status),
                                       _stream_handle(stream))
     _lib.check(rc, "attn_decode_paged")
+    return out, lse
+
+
+def decode_window_workspace_bytes(B: int, Hq: int, Hkv: int, d: int, max_seq_len: int, block_size: int, window: int,
+                                  n_sink: int) -> int:
+    n = int(_lib.lib().attn_decode_window_workspace_bytes(B, Hq, Hkv, d, max_seq_len, block_size, window, n_sink))
+    if n == 0:
+        raise AttnError(_lib.ATTN_ERR_INVALID_ARG, "attn_decode_window_workspace_bytes")
+    return n
+
+
+def decode_paged_window(q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int, window: int = 0,
+                        n_sink: int = 0, sinks=None, scale: float | None = None, out=None, lse=None, workspace=None,
+                        status=None, stream=None, return_lse: bool = True):
+    """Paged decode with a sliding window of `window` positions (0: none), the
+    first `n_sink` positions kept visible, and optional learned per-head sink
+    logits `sinks` (fp32 [Hq], appended to the scaled scores with no value).
+    Returns (O [B, Hq, d] bf16, LSE [B, Hq] fp32, including the sink column).
+    """
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hq, d = q.shape
+    num_blocks, block_size, Hkv, d2 = k_cache.shape
+    if d2 != d or v_cache.shape != k_cache.shape:
+        raise ValueError("caches must be [num_blocks, block_size, Hkv, d] matching q")
+    if block_table.shape[0] != B or seq_lens.shape[0] != B:
+        raise ValueError("block_table and seq_lens need one row per sequence")
+    if sinks is not None:
+        _need(sinks, "sinks", torch.float32, 1)
+        if sinks.shape[0] != Hq:
+            raise ValueError("sinks needs one logit per query head")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if workspace is None:
+        nbytes = decode_window_workspace_bytes(B, Hq, Hkv, d, max_seq_len, block_size, int(window), int(n_sink))
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    rc = _lib.lib().attn_decode_paged_window(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                             _ptr(seq_lens), _ptr(sinks), _ptr(out), _ptr(lse), B, Hq, Hkv, d,
+                                             num_blocks, block_size, block_table.shape[1], int(max_seq_len),
+                                             int(window), int(n_sink), float(scale), _ptr(workspace),
+                                             workspace.numel() * workspace.element_size(), _ptr(status),
+                                             _stream_handle(stream))
+    _lib.check(rc, "attn_decode_paged_window")
     return out, lse
 
 

@@ -20,6 +20,8 @@ SYMBOLS = (
     "attn_decode_workspace_bytes",
     "attn_decode_paged",
     "attn_decode_paged_noalloc",
+    "attn_decode_window_workspace_bytes",
+    "attn_decode_paged_window",
     "attn_paged_gather",
     "attn_status_string",
     "attn_version",
@@ -61,6 +63,11 @@ def _declare(lib):
     lib.attn_decode_paged_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                               _vp, _vp]
     lib.attn_decode_paged_noalloc.restype = _i
+    lib.attn_decode_window_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
+    lib.attn_decode_window_workspace_bytes.restype = _sz
+    lib.attn_decode_paged_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                                             _i, _i, _f, _vp, _sz, _vp, _vp]
+    lib.attn_decode_paged_window.restype = _i
     lib.attn_paged_gather.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]
     lib.attn_paged_gather.restype = _i
     lib.attn_status_string.argtypes = [_i]

@@ -113,20 +113,26 @@ int attn_decode_plan(int B, int Hq, int Hkv, int max_seq_len, int num_sms, int* 
   return ATTN_OK;
 }
 
-size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int max_seq_len, int block_size) {
+}  // extern "C"
+
+namespace {
+
+// Workspace bytes of a (possibly windowed) decode, 0 for invalid sizes.
+size_t decode_bytes(int B, int Hq, int Hkv, int d, int max_seq_len, int block_size, int window, int n_sink) {
   if (d != 64 && d != 128) return 0;
   if (block_size <= 0 || block_size % 16 != 0) return 0;
+  if (window < 0 || n_sink < 0 || max_seq_len <= 0) return 0;
   int sms = 0;
   if (current_sm_count(&sms) != ATTN_OK) return 0;
   DecodePlan plan;
-  if (plan_decode(B, Hq, Hkv, max_seq_len, sms, &plan) != ATTN_OK) return 0;
+  if (plan_decode(B, Hq, Hkv, decode_plan_length(max_seq_len, window, n_sink), sms, &plan) != ATTN_OK) return 0;
   return decode_workspace_bytes(B, Hq, d, plan);
 }
 
-int attn_decode_paged(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
-                      const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int d,
-                      int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, float scale,
-                      void* workspace, size_t workspace_bytes, int32_t* status, attn_stream_t stream) {
+int decode_common(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                  const int32_t* seq_lens, const float* sinks, void* o, float* lse, int B, int Hq, int Hkv, int d,
+                  int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, int window, int n_sink,
+                  float scale, void* workspace, size_t workspace_bytes, int32_t* status, attn_stream_t stream) {
   if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !o) return ATTN_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || num_blocks <= 0 || block_size <= 0 || max_blocks_per_seq <= 0 ||
       max_seq_len <= 0)
@@ -134,23 +140,62 @@ int attn_decode_paged(const void* q, const void* k_cache, const void* v_cache, c
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (static_cast<long long>(max_blocks_per_seq) * block_size < max_seq_len) return ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  // sinks: the first n_sink positions, only beside a finite window, 0 <= n_sink <= n
+  if (window < 0 || n_sink < 0 || n_sink > max_seq_len || (n_sink > 0 && window == 0)) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
     return ATTN_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_INVALID_ARG;
+  if (sinks && (reinterpret_cast<uintptr_t>(sinks) & 3u)) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (block_size % 16 != 0) return ATTN_ERR_UNSUPPORTED;
   if (B > 65535 || static_cast<long long>(Hkv) * ((Hq / Hkv + 15) / 16) > 65535) return ATTN_ERR_UNSUPPORTED;
+  // a window that covers every position hides nothing: the sink positions are inside it
+  if (window >= max_seq_len) window = n_sink = 0;
   int sms = 0;
   if (current_sm_count(&sms) != ATTN_OK) return ATTN_ERR_CUDA;
   DecodePlan plan;
-  if (plan_decode(B, Hq, Hkv, max_seq_len, sms, &plan) != ATTN_OK) return ATTN_ERR_INVALID_ARG;
+  if (plan_decode(B, Hq, Hkv, decode_plan_length(max_seq_len, window, n_sink), sms, &plan) != ATTN_OK)
+    return ATTN_ERR_INVALID_ARG;
   if (!workspace || !aligned16(workspace) || workspace_bytes < decode_workspace_bytes(B, Hq, d, plan))
     return ATTN_ERR_WORKSPACE;
-  const cudaError_t e = launch_decode(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, d, num_blocks,
-                                      block_size, max_blocks_per_seq, max_seq_len, scale, workspace, plan, status,
-                                      reinterpret_cast<cudaStream_t>(stream));
+  const cudaError_t e = launch_decode(q, k_cache, v_cache, block_table, seq_lens, sinks, o, lse, B, Hq, Hkv, d,
+                                      num_blocks, block_size, max_blocks_per_seq, max_seq_len, window, n_sink, scale,
+                                      workspace, plan, status, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int max_seq_len, int block_size) {
+  return decode_bytes(B, Hq, Hkv, d, max_seq_len, block_size, 0, 0);
+}
+
+size_t attn_decode_window_workspace_bytes(int B, int Hq, int Hkv, int d, int max_seq_len, int block_size, int window,
+                                          int n_sink) {
+  if (window >= max_seq_len) window = n_sink = 0;
+  return decode_bytes(B, Hq, Hkv, d, max_seq_len, block_size, window, n_sink);
+}
+
+int attn_decode_paged(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                      const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int d,
+                      int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, float scale,
+                      void* workspace, size_t workspace_bytes, int32_t* status, attn_stream_t stream) {
+  return decode_common(q, k_cache, v_cache, block_table, seq_lens, nullptr, o, lse, B, Hq, Hkv, d, num_blocks,
+                       block_size, max_blocks_per_seq, max_seq_len, 0, 0, scale, workspace, workspace_bytes, status,
+                       stream);
+}
+
+int attn_decode_paged_window(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                             const int32_t* seq_lens, const float* sinks, void* o, float* lse, int B, int Hq, int Hkv,
+                             int d, int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len,
+                             int window, int n_sink, float scale, void* workspace, size_t workspace_bytes,
+                             int32_t* status, attn_stream_t stream) {
+  return decode_common(q, k_cache, v_cache, block_table, seq_lens, sinks, o, lse, B, Hq, Hkv, d, num_blocks,
+                       block_size, max_blocks_per_seq, max_seq_len, window, n_sink, scale, workspace,
+                       workspace_bytes, status, stream);
 }
 
 int attn_paged_gather(const void* cache, const int32_t* block_table, const int32_t* seq_lens, void* out, int B,

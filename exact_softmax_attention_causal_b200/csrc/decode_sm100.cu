@@ -21,6 +21,17 @@
 //
 // The kernel is HBM-bound: each K/V byte of a (sequence, K/V head) is read
 // once and shared by the whole query-head group.
+//
+// Sliding window and sinks ("Module 5. Modern Attention Mechanisms", sections
+// 9, 10 and 12): with a window of W positions the query at position n - 1
+// sees positions max(0, n - W) .. n - 1, plus the first n_sink positions
+// (StreamingLLM). The kernels walk a list of the 16-token sub-blocks that
+// hold a visible token (the sink sub-blocks, then the window's), so the
+// splits, the loads and the merge only ever touch visible sub-blocks; rows of
+// a listed sub-block that are not visible are zero-filled instead of loaded
+// and masked to -inf. A learned per-head sink logit s_h (gpt-oss) is one more
+// score column with no value; the merge folds it in:
+// lse = log(exp(lse_tokens) + exp(s_h)), O = O_tokens * exp(lse_tokens - lse).
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -51,7 +62,31 @@ struct DecodeParams {
   int B, Hq, Hkv, group, hchunks;
   int num_blocks, block_size, max_blocks_per_seq, max_seq_len;
   int chunk, splits;
+  int window, n_sink;  // window 0: every cached token is visible (n_sink is then 0)
   float scale_log2;  // scale * log2(e): scores live in the base-2 domain
+};
+
+// The visible tokens of a query at position seq_len - 1, as a list of
+// 16-token sub-blocks: sub-blocks 0 .. a-1 hold the sink positions [0, s) not
+// already inside the window, sub-blocks w0 .. ceil(seq_len / 16) - 1 the
+// window [lo, seq_len). Every listed sub-block holds at least one visible
+// token, and a pool block none of whose tokens is visible is never listed.
+struct VisibleList {
+  int lo;   // first window position
+  int s;    // sink positions below lo: [0, s)
+  int a;    // sink sub-blocks
+  int w0;   // first window sub-block (after the sink ones)
+  int nsb;  // listed sub-blocks
+  __device__ __forceinline__ VisibleList(int seq_len, int window, int n_sink) {
+    lo = window > 0 ? max(0, seq_len - window) : 0;
+    s = min(n_sink, lo);
+    a = (s + kSub - 1) / kSub;
+    w0 = max(lo / kSub, a);
+    nsb = a + max(0, (seq_len + kSub - 1) / kSub - w0);
+  }
+  // first token of listed sub-block u
+  __device__ __forceinline__ int token0(int u) const { return kSub * (u < a ? u : w0 + (u - a)); }
+  __device__ __forceinline__ bool visible(int t, int seq_len) const { return t < seq_len && (t >= lo || t < s); }
 };
 
 __device__ __forceinline__ void flag_status(int32_t* status, int bit) {
@@ -91,10 +126,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
 
   const int seq_len = p.seq_lens[b];
   if (seq_len < 1 || seq_len > p.max_seq_len) return;  // the merge kernel flags this row
-  const int t0 = split * p.chunk;
-  if (t0 >= seq_len) return;  // chunk past the end: the merge never reads it
-  const int t1 = min(t0 + p.chunk, seq_len);
-  const int nsub = (t1 - t0 + kSub - 1) / kSub;
+  const VisibleList vis(seq_len, p.window, p.n_sink);
+  const int u0 = split * (p.chunk / kSub);  // this split's listed sub-blocks [u0, u0 + nsub)
+  if (u0 >= vis.nsb) return;  // split past the end of the list: the merge never reads it
+  const int nsub = min(p.chunk / kSub, vis.nsb - u0);
   const int h0 = kvh * p.group + hc * 16;
   const int rows = min(16, p.group - hc * 16);
 
@@ -127,7 +162,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   bool bad = false;
 
   auto issue = [&](int j, int stage) {
-    const int t = t0 + (warp + j * kDecWarps) * kSub;  // first token of the sub-block
+    const int t = vis.token0(u0 + warp + j * kDecWarps);  // first token of the sub-block
     const int lblk = t / p.block_size;
     const int off = t - lblk * p.block_size;  // multiple of 16, off + 15 < block_size
     const int phys = __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks_per_seq + lblk);
@@ -137,7 +172,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
 #pragma unroll
     for (int x = lane; x < kSub * L::kChunks; x += 32) {
       const int r = x / L::kChunks, c = x % L::kChunks;
-      const bool valid = ok && (t + r < t1);  // slots past seq_len are zero-filled, never read
+      const bool valid = ok && vis.visible(t + r, seq_len);  // hidden slots are zero-filled, never read
       const size_t src = valid ? ((static_cast<size_t>(phys) * p.block_size + off + r) * p.Hkv + kvh) * D + c * 8
                                : 0;
       const uint32_t dst = kdst + swz(r, c, L::kRowBytes);
@@ -169,7 +204,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
 
     const uint32_t kb = smem_u32(my_ring + (j % kStages) * 2 * L::kTile);
     const uint32_t vb = kb + L::kTile;
-    const int tok0 = t0 + (warp + j * kDecWarps) * kSub;
+    const int tok0 = vis.token0(u0 + warp + j * kDecWarps);
 
     // S = Q K^T for 16 tokens: two n-tiles of 8 tokens.
     float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -182,14 +217,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
       mma_bf16_16816(s[0], qf[kk], b00, b01);
       mma_bf16_16816(s[1], qf[kk], b10, b11);
     }
-    // scale into base 2, mask slots past the sequence end
+    // scale into base 2, mask slots that are not visible
     float mx[2] = {neg_inf, neg_inf};
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int tok = tok0 + nt * 8 + 2 * tq + (e & 1);
-        const float x = (tok < t1) ? s[nt][e] * p.scale_log2 : neg_inf;
+        const float x = vis.visible(tok, seq_len) ? s[nt][e] * p.scale_log2 : neg_inf;
         s[nt][e] = x;
         mx[e >> 1] = fmaxf(mx[e >> 1], x);
       }
@@ -199,7 +234,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
       mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
       mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
     }
-    // the first token of a sub-block is always < t1, so mx is finite
+    // every listed sub-block holds a visible token, so mx is finite
     float alpha[2];
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
@@ -313,16 +348,18 @@ struct MergeParams {
   const float* o_part;
   const float* lse_part;
   const int32_t* seq_lens;
+  const float* sinks;  // [Hq] learned sink logits or nullptr
   __nv_bfloat16* o;
   float* lse;
   int32_t* status;
-  int B, Hq, splits, chunk, max_seq_len;
+  int B, Hq, splits, chunk, max_seq_len, window, n_sink;
 };
 
 // One CTA of 4 warps per (sequence, query head): lse = log sum_s exp(lse_s),
 // O = sum_s exp(lse_s - lse) O_s over the chunks that hold tokens. The warps
 // take every 4th chunk and combine their partial sums in shared memory, so a
-// single long sequence with hundreds of chunks still merges in parallel.
+// single long sequence with hundreds of chunks still merges in parallel. A
+// learned sink logit joins the normaliser last (it carries no value).
 constexpr int kMergeWarps = 4;
 
 template <int D>
@@ -347,7 +384,8 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
       for (int e = 0; e < PER; ++e) orow[e] = __float2bfloat16_rn(NAN);
     return;
   }
-  const int ns = (seq_len + p.chunk - 1) / p.chunk;
+  const int per_split = p.chunk / kSub;
+  const int ns = (VisibleList(seq_len, p.window, p.n_sink).nsb + per_split - 1) / per_split;
   const float* lrow = p.lse_part + row * p.splits;
   // global max over the chunks
   float M = -INFINITY;
@@ -397,7 +435,21 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
     float total = 0.f;
 #pragma unroll
     for (int w = 0; w < kMergeWarps; ++w) total += s_sum[w];
-    const float inv = 1.f / total;
+    float inv = 1.f / total;
+    float lse_out = M + __logf(total);
+    if (p.sinks != nullptr) {
+      // one more score column s_h with a zero value: log-add it to the
+      // normaliser and shrink the output by the tokens' share of the mass
+      const float sk = p.sinks[row % p.Hq];
+      if (!(fabsf(sk) <= 3.0e38f)) {  // NaN or infinite sink logit
+        any_nan = 1;
+        if (lane == 0) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
+      }
+      const float hi = fmaxf(lse_out, sk), lo = fminf(lse_out, sk);
+      const float lse_all = hi + log1pf(__expf(lo - hi));
+      inv *= __expf(lse_out - lse_all);
+      lse_out = lse_all;
+    }
     float out[PER];
 #pragma unroll
     for (int e = 0; e < PER; ++e) {
@@ -409,7 +461,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
 #pragma unroll
     for (int e = 0; e < PER; e += 2)
       *reinterpret_cast<__nv_bfloat162*>(orow + e) = __floats2bfloat162_rn(out[e], out[e + 1]);
-    if (lane == 0 && p.lse) p.lse[row] = any_nan ? NAN : M + __logf(total);
+    if (lane == 0 && p.lse) p.lse[row] = any_nan ? NAN : lse_out;
   }
 }
 
@@ -454,9 +506,10 @@ __global__ void paged_gather_kernel(const uint4* __restrict__ cache, const int32
 
 template <int D>
 cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
-                            const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int num_blocks,
-                            int block_size, int max_blocks_per_seq, int max_seq_len, float scale, void* workspace,
-                            const DecodePlan& plan, int32_t* status, cudaStream_t stream) {
+                            const int32_t* seq_lens, const float* sinks, void* o, float* lse, int B, int Hq, int Hkv,
+                            int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, int window,
+                            int n_sink, float scale, void* workspace, const DecodePlan& plan, int32_t* status,
+                            cudaStream_t stream) {
   DecodeParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
@@ -477,6 +530,8 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   p.max_seq_len = max_seq_len;
   p.chunk = plan.chunk;
   p.splits = plan.splits;
+  p.window = window;
+  p.n_sink = n_sink;
   p.scale_log2 = scale * kLog2e;
 
   const int smem = DecSmem<D>::kTotal;
@@ -491,6 +546,7 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   m.o_part = p.o_part;
   m.lse_part = p.lse_part;
   m.seq_lens = seq_lens;
+  m.sinks = sinks;
   m.o = static_cast<__nv_bfloat16*>(o);
   m.lse = lse;
   m.status = status;
@@ -499,6 +555,8 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   m.splits = plan.splits;
   m.chunk = plan.chunk;
   m.max_seq_len = max_seq_len;
+  m.window = window;
+  m.n_sink = n_sink;
   decode_merge_kernel<D><<<B * Hq, kMergeWarps * 32, 0, stream>>>(m);
   return cudaGetLastError();
 }
@@ -508,6 +566,14 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
 size_t decode_workspace_bytes(int B, int Hq, int d, const DecodePlan& plan) {
   const size_t rows = static_cast<size_t>(B) * Hq * plan.splits;
   return rows * d * sizeof(float) + rows * sizeof(float);
+}
+
+int decode_plan_length(int max_seq_len, int window, int n_sink) {
+  const long long whole = (static_cast<long long>(max_seq_len) + 15) / 16 * 16;
+  if (window <= 0) return max_seq_len;
+  // listed sub-blocks <= ceil(n_sink / 16) + ceil(window / 16) + 1
+  const long long listed = 16LL * ((n_sink + 15LL) / 16 + (window + 15LL) / 16 + 1);
+  return static_cast<int>(listed < whole ? listed : whole);
 }
 
 int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan* out) {
@@ -526,14 +592,17 @@ int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan
 }
 
 cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
-                          const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int d,
-                          int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, float scale,
-                          void* workspace, const DecodePlan& plan, int32_t* status, cudaStream_t stream) {
+                          const int32_t* seq_lens, const float* sinks, void* o, float* lse, int B, int Hq, int Hkv,
+                          int d, int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, int window,
+                          int n_sink, float scale, void* workspace, const DecodePlan& plan, int32_t* status,
+                          cudaStream_t stream) {
   if (d == 128)
-    return launch_decode_t<128>(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, num_blocks,
-                                block_size, max_blocks_per_seq, max_seq_len, scale, workspace, plan, status, stream);
-  return launch_decode_t<64>(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, num_blocks, block_size,
-                             max_blocks_per_seq, max_seq_len, scale, workspace, plan, status, stream);
+    return launch_decode_t<128>(q, k_cache, v_cache, block_table, seq_lens, sinks, o, lse, B, Hq, Hkv, num_blocks,
+                                block_size, max_blocks_per_seq, max_seq_len, window, n_sink, scale, workspace, plan,
+                                status, stream);
+  return launch_decode_t<64>(q, k_cache, v_cache, block_table, seq_lens, sinks, o, lse, B, Hq, Hkv, num_blocks,
+                             block_size, max_blocks_per_seq, max_seq_len, window, n_sink, scale, workspace, plan,
+                             status, stream);
 }
 
 cudaError_t launch_paged_gather(const void* cache, const int32_t* block_table, const int32_t* seq_lens, void* out,

@@ -27,13 +27,18 @@ struct DecodePlan {
 };
 
 int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan* out);
+// Length the split plan is made for: max_seq_len without a window, else the
+// most tokens a windowed query's visible sub-block list can span.
+int decode_plan_length(int max_seq_len, int window, int n_sink);
 size_t decode_workspace_bytes(int B, int Hq, int d, const DecodePlan& plan);
 
 // Kernel launchers (defined next to their kernels). Return cudaError_t.
+// window 0 = every cached token visible (n_sink must then be 0); sinks may be nullptr.
 cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
-                          const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int d,
-                          int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, float scale,
-                          void* workspace, const DecodePlan& plan, int32_t* status, cudaStream_t stream);
+                          const int32_t* seq_lens, const float* sinks, void* o, float* lse, int B, int Hq, int Hkv,
+                          int d, int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, int window,
+                          int n_sink, float scale, void* workspace, const DecodePlan& plan, int32_t* status,
+                          cudaStream_t stream);
 
 cudaError_t launch_paged_gather(const void* cache, const int32_t* block_table, const int32_t* seq_lens, void* out,
                                 int B, int Hkv, int d, int num_blocks, int block_size, int max_blocks_per_seq,

@@ -381,20 +381,34 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // partly filled block goes row by row (tm_row: one-row boxes) so that its
         // slots past seq_len arrive as zeros, never as stale pool contents: their
         // probabilities are 0, and 0 * NaN would still poison P.V.
-        auto load_kv = [&](const CUtensorMap* tm, const CUtensorMap* tm_row, uint32_t dst, uint32_t bar_full,
-                           int kt) {
+        //
+        // The table entries of a key tile are read one tile ahead (all of them in
+        // flight at once) and kept for the V copy of the same tile, so the
+        // producer never waits on a table read between two copies.
+        constexpr int kMaxBoxes = kBN / 16;
+        auto fetch_entries = [&](int kt, int (&ent)[kMaxBoxes]) {
+          if (!PAGED) return;
+          const int bs = p.block_size;
+#pragma unroll
+          for (int e = 0; e < kMaxBoxes; ++e) {
+            const int key = kt * kBN + e * bs;
+            ent[e] = p.num_blocks;
+            if (e * bs < kBN && !gm.bad && key < gm.nk)
+              ent[e] = __ldg(p.block_table + static_cast<size_t>(wi.b) * p.max_blocks + key / bs);
+          }
+        };
+        auto load_kv = [&](const CUtensorMap* tm, const CUtensorMap* tm_row, uint32_t dst, uint32_t bar_full, int kt,
+                           const int (&ent)[kMaxBoxes]) {
           if (!PAGED) {
             for (int hh = 0; hh < C::kHalves; ++hh)
               tma_load_3d(dst + hh * C::kHalf, tm, bar_full, hh * 64, kt * kBN, zkv);
           } else {
             const int bs = p.block_size;
-            for (int e = 0; e < kBN / bs; ++e) {
+#pragma unroll
+            for (int e = 0; e < kMaxBoxes; ++e) {
+              if (e * bs >= kBN) break;
               const int key = kt * kBN + e * bs;
-              int phys = p.num_blocks;
-              if (!gm.bad && key < gm.nk) {
-                const int entry = __ldg(p.block_table + static_cast<size_t>(wi.b) * p.max_blocks + key / bs);
-                if (entry >= 0 && entry < p.num_blocks) phys = entry;
-              }
+              const int phys = (ent[e] >= 0 && ent[e] < p.num_blocks) ? ent[e] : p.num_blocks;
               const uint32_t bdst = dst + e * bs * 128;
               if (key + bs <= gm.nk || phys == p.num_blocks) {
                 for (int hh = 0; hh < C::kHalves; ++hh)
@@ -409,6 +423,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             }
           }
         };
+        int ent_k[kMaxBoxes], ent_v[kMaxBoxes];  // entries of key tiles i and i - 1
+        fetch_entries(kt_lo, ent_k);
         // Q of this item once the previous item's last score MMA has read its Q
         if (it > 0 && !mbar_wait_bounded(bar(kBarQEmpty), (it - 1) & 1, budget, abort_flag)) {
           ok = false;
@@ -428,7 +444,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               break;
             }
             mbar_arrive_expect_tx(bar(kBarKFull + s), C::kTile);
-            load_kv(&tm_k, &tm_kr, sbase + C::kKOff + s * C::kTile, bar(kBarKFull + s), kt_lo + i);
+            load_kv(&tm_k, &tm_kr, sbase + C::kKOff + s * C::kTile, bar(kBarKFull + s), kt_lo + i, ent_k);
             k_issued = gi + 1;
           }
           if (i >= 1) {
@@ -438,8 +454,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               break;
             }
             mbar_arrive_expect_tx(bar(kBarVFull + s), C::kTile);
-            load_kv(&tm_v, &tm_vr, sbase + C::kVOff + s * C::kTile, bar(kBarVFull + s), kt_lo + i - 1);
+            load_kv(&tm_v, &tm_vr, sbase + C::kVOff + s * C::kTile, bar(kBarVFull + s), kt_lo + i - 1, ent_v);
             v_issued = gv + 1;
+          }
+          if (PAGED) {
+#pragma unroll
+            for (int e = 0; e < kMaxBoxes; ++e) ent_v[e] = ent_k[e];
+            if (i + 1 < T) fetch_entries(kt_lo + i + 1, ent_k);
           }
         }
         g += T;

@@ -15,6 +15,12 @@
  *                        ("Module 09: Efficient Attention", "The Block Table"),
  *                        split along the sequence and merged by log-sum-exp
  *                        ("Inference attention" post, section "FlashDecoding").
+ *   attn_decode_paged_window - the same decode with a sliding window, the
+ *                        StreamingLLM sink positions and gpt-oss's learned
+ *                        per-head sink logit ("Modern Attention Mechanisms",
+ *                        sections 9, 10 and 12).
+ *   attn_prefill_paged - the newest Nq positions of each sequence against its
+ *                        paged context (prefix / chunked prefill).
  *
  * Conventions shared by every entry point:
  *   - Pointers named q, k, v, o, lse, k_cache, v_cache, block_table, seq_lens,
@@ -187,6 +193,57 @@ ATTN_API int attn_decode_paged(const void* q, const void* k_cache, const void* v
                       const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int d,
                       int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, float scale,
                       void* workspace, size_t workspace_bytes, int32_t* status, attn_stream_t stream);
+
+/*
+ * attn_decode_window_workspace_bytes - bytes of device workspace
+ * attn_decode_paged_window needs for these sizes, window and n_sink (the split
+ * plan covers only the sub-blocks a windowed query can see). Equal to
+ * attn_decode_workspace_bytes when window == 0 or window >= max_seq_len.
+ * Returns 0 for invalid sizes.
+ */
+ATTN_API size_t attn_decode_window_workspace_bytes(int B, int Hq, int Hkv, int d, int max_seq_len, int block_size,
+                                                   int window, int n_sink);
+
+/*
+ * attn_decode_paged_window - attn_decode_paged with a sliding window, sink
+ * positions and learned sink logits.
+ *
+ * Defined by "Module 5. Modern Attention Mechanisms": section 4/9 (a window
+ * of W positions includes the current one: the query at position
+ * n - 1 = seq_lens[b] - 1 sees positions p with 0 <= n - 1 - p < W), section
+ * 10 and the mask builder of section 12 (StreamingLLM: the first n_sink
+ * positions stay visible beside a finite window), and section 10's gpt-oss
+ * sink: each query head h owns a logit sinks[h] that is appended to the row's
+ * scaled scores, normalised with them and dropped before the product with V
+ * (it takes probability mass and contributes no value).
+ *
+ * Arguments as for attn_decode_paged, plus
+ *   sinks        [Hq] fp32 device array of sink logits (natural-log units, the
+ *                same units as scale * q.k), or NULL for none. A non-finite
+ *                logit turns that head's rows into NaN and sets
+ *                ATTN_STATUS_BIT_DEVICE_CHECK.
+ *   window       W >= 1, or 0 for no window (every cached token visible).
+ *                W >= max_seq_len behaves as 0.
+ *   n_sink       0 <= n_sink <= max_seq_len; n_sink > 0 needs window > 0
+ *                (else ATTN_ERR_INVALID_ARG).
+ *   workspace    at least attn_decode_window_workspace_bytes(...) bytes.
+ *
+ *   o            softmax over the visible tokens and the sink column, times V.
+ *   lse          log(sum over visible tokens of exp(scale * q.k) + exp(sinks[h])):
+ *                the log of the full softmax denominator (without sinks, the
+ *                log-sum-exp over the visible tokens).
+ *
+ * Only table entries of blocks that hold a visible token are read: a rolling
+ * cache may leave the entries of evicted middle blocks as -1. Out-of-range
+ * entries that are read, and seq_lens outside [1, max_seq_len], are handled
+ * as in attn_decode_paged.
+ */
+ATTN_API int attn_decode_paged_window(const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* block_table, const int32_t* seq_lens, const float* sinks, void* o,
+                                      float* lse, int B, int Hq, int Hkv, int d, int num_blocks, int block_size,
+                                      int max_blocks_per_seq, int max_seq_len, int window, int n_sink, float scale,
+                                      void* workspace, size_t workspace_bytes, int32_t* status,
+                                      attn_stream_t stream);
 
 /*
  * attn_paged_gather - walk every sequence's block table into a contiguous

@@ -238,14 +238,15 @@ def gather_paged_ref(cache, block_table, seq_lens, max_seq_len: int):
 
 
 def _gather_one(cache, table_row, n: int) -> np.ndarray:
-    """Token-by-token gather of one sequence: [n, Hkv, d] float64."""
+    """Token-by-token gather of one sequence: [n, Hkv, d] float64. Each row is
+    widened as it is copied, so the pool itself is never converted whole."""
     num_blocks, bs = cache.shape[0], cache.shape[1]
-    rows = np.empty((n,) + cache.shape[2:], dtype=np.float64)
+    rows = np.empty((n,) + tuple(cache.shape[2:]), dtype=np.float64)
     for t in range(n):
         phys = int(table_row[t // bs])
         if phys < 0 or phys >= num_blocks:
             raise ValueError(f"block table entry {phys} outside the pool")
-        rows[t] = cache[phys, t % bs]
+        rows[t] = _as_f64(cache[phys, t % bs])
     return rows
 
 
@@ -271,11 +272,9 @@ def decode_rows_ref(q, k_cache, v_cache, block_table, seq_lens, b: int, heads, s
         raise ValueError("a decode row needs at least one cached token")
     kind = MASK_SLIDING_WINDOW if window > 0 else MASK_CAUSAL
     allowed = allowed_mask(1, n, kind, window, n_sink=min(int(n_sink), n))
-    kc = _as_f64(k_cache)
-    vc = _as_f64(v_cache)
     row = _as_int(block_table)[b]
-    k_seq = _gather_one(kc, row, n)
-    v_seq = _gather_one(vc, row, n)
+    k_seq = _gather_one(k_cache, row, n)
+    v_seq = _gather_one(v_cache, row, n)
     qb = _as_f64(q[b])
     sk = None if sinks is None else _as_f64(sinks)
     outs, lses = [], []

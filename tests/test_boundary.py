@@ -93,6 +93,39 @@ def test_decode_rejects_bad_arguments(kw, code):
     assert _decode(**kw) == code
 
 
+def _decode_window(**kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, sl=FAKE, sinks=NULL, o=FAKE, lse=NULL, B=2, Hq=8, Hkv=2, d=128, nb=10,
+             bs=16, mb=4, msl=64, window=16, n_sink=4, scale=0.1, ws=FAKE, wsb=1 << 20)
+    a.update(kw)
+    return _lib.lib().attn_decode_paged_window(a["q"], a["kc"], a["vc"], a["bt"], a["sl"], a["sinks"], a["o"],
+                                               a["lse"], a["B"], a["Hq"], a["Hkv"], a["d"], a["nb"], a["bs"], a["mb"],
+                                               a["msl"], a["window"], a["n_sink"], a["scale"], a["ws"], a["wsb"],
+                                               NULL, NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=NULL), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(window=-1), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(n_sink=-1), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(window=0, n_sink=1), _lib.ATTN_ERR_INVALID_ARG),  # sink positions only beside a finite window
+    (dict(n_sink=65), _lib.ATTN_ERR_INVALID_ARG),           # n_sink > max_seq_len
+    (dict(sinks=ctypes.c_void_p(0x10002)), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(mb=3), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(d=80), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(bs=8, mb=8), _lib.ATTN_ERR_UNSUPPORTED),
+])
+def test_decode_window_rejects_bad_arguments(kw, code):
+    assert _decode_window(**kw) == code
+
+
+def test_decode_window_workspace_rejects_bad_sizes():
+    lib = _lib.lib()
+    assert lib.attn_decode_window_workspace_bytes(2, 8, 2, 80, 64, 16, 16, 0) == 0
+    assert lib.attn_decode_window_workspace_bytes(2, 8, 2, 128, 64, 8, 16, 0) == 0
+    assert lib.attn_decode_window_workspace_bytes(2, 8, 2, 128, 64, 16, -1, 0) == 0
+
+
 def _prefill_paged(**kw):
     a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, sl=FAKE, o=FAKE, lse=NULL, B=2, Hq=8, Hkv=2, Nq=64, d=128, nb=10,
              bs=16, mb=8, msl=128, mask=1, window=0, scale=0.1)
