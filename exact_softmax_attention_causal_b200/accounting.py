@@ -79,3 +79,14 @@ def decode_visible_tokens(n: int, window: int = 0, n_sink: int = 0) -> int:
 
 def decode_window_kv_bytes(seq_lens, Hkv: int, d: int, window: int = 0, n_sink: int = 0) -> int:
     return sum(decode_visible_tokens(n, window, n_sink) for n in seq_lens) * Hkv * d * 2 * 2
+
+
+def mla_decode_bytes(seq_lens, d_latent: int, d_rope: int) -> int:
+    """Latent-cache bytes an absorbed MLA decode step must read: one
+    (d_c + d_R)-wide bf16 row per cached token, shared by every head."""
+    return sum(int(n) for n in seq_lens) * (d_latent + d_rope) * 2
+
+
+def mla_decode_flops(seq_lens, H: int, d_latent: int, d_rope: int) -> int:
+    """2 (d_c + d_R) for the logit plus 2 d_c for the latent output, per head per token."""
+    return sum(int(n) for n in seq_lens) * H * (2 * (d_latent + d_rope) + 2 * d_latent)

@@ -155,6 +155,37 @@ def paged_prefill_inputs(B: int, Hq: int, Hkv: int, Nq: int, d: int, *, seq_lens
     return PagedPrefillInputs(q, k_cache, v_cache, table, seq_lens, block_size, int(max_seq_len), seed)
 
 
+@dataclasses.dataclass
+class MlaDecodeInputs:
+    q: torch.Tensor            # [B, H, d_c + d_R] bf16: absorbed content query, then positional query
+    cache: torch.Tensor        # [num_blocks, block_size, d_c + d_R] bf16: latent, then positional key
+    block_table: torch.Tensor  # [B, max_blocks] int32
+    seq_lens: torch.Tensor     # [B] int32
+    d_latent: int
+    block_size: int
+    max_seq_len: int
+    seed: int
+
+
+def mla_decode_inputs(B: int, H: int, d_latent: int, d_rope: int, *, seq_lens=None, len_range=None,
+                      block_size: int = 16, max_seq_len: int | None = None, seed: int = 0,
+                      extra_blocks: int = 0) -> MlaDecodeInputs:
+    """Same recipe as paged_decode_inputs with one latent row per token: draw
+    seq_lens, lay out the pool, then Q and the cache as bf16-rounded normals."""
+    gen = torch.Generator("cpu").manual_seed(seed)
+    if seq_lens is None:
+        lo, hi = len_range
+        seq_lens = torch.randint(lo, hi + 1, (B,), generator=gen, dtype=torch.int64)
+    seq_lens = torch.as_tensor(seq_lens, dtype=torch.int32).reshape(B)
+    if max_seq_len is None:
+        max_seq_len = int(len_range[1]) if len_range is not None else int(seq_lens.max())
+    table, pool = paged_layout(seq_lens.tolist(), block_size, blocks_needed(max_seq_len, block_size), gen,
+                               extra_blocks)
+    q = _normal_bf16((B, H, d_latent + d_rope), gen)
+    cache = _normal_bf16((pool, block_size, d_latent + d_rope), gen)
+    return MlaDecodeInputs(q, cache, table, seq_lens, d_latent, block_size, int(max_seq_len), seed)
+
+
 # Named workloads. Sizes follow the pages' shapes: Llama-style GQA-8
 # ("USAAIO Lesson 90", GQA part), 131,072-token contexts ("Modern Attention
 # Mechanisms", section 1) and 16-token blocks ("Module 09", "The Block Table").
@@ -193,6 +224,18 @@ WINDOW_DECODE_WORKLOADS = {
                                   window=0, n_sink=0, learned_sinks=True),
     "streaming_window4096_nsink4_b64": dict(B=64, Hq=32, Hkv=8, d=128, len_range=(8192, 32768), block_size=16,
                                             window=4096, n_sink=4, learned_sinks=False),
+}
+
+
+# Absorbed MLA decode with DeepSeek-V2's shapes ("Module 09", MLA section: a
+# 512-wide latent and a 64-wide positional key per token, 128 heads of head
+# dim 128, so the logit scale is 1 / sqrt(128 + 64)); the second keeps 16 of
+# the 128 heads, as one GPU holds when the heads are split eight ways.
+MLA_DECODE_WORKLOADS = {
+    "deepseek_v2_mla_b64": dict(B=64, H=128, d_latent=512, d_rope=64, d_head=128, len_range=(1024, 32768),
+                                block_size=16),
+    "deepseek_v2_mla_h16_b64": dict(B=64, H=16, d_latent=512, d_rope=64, d_head=128, len_range=(1024, 32768),
+                                    block_size=16),
 }
 
 
