@@ -1,4 +1,4 @@
-"""fp64 CPU oracle for exact softmax attention (prefill, paged decode, MLA decode).
+"""fp64 CPU oracle for exact softmax attention (prefill, paged decode, MLA decode, backward).
 
 TEST INFRASTRUCTURE ONLY. This package is the slow, plain definition that the
 CUDA path is checked against. Only ``tests/``, ``__graft_entry__.smoke()`` and
@@ -28,3 +28,4 @@ from .attention import (  # noqa: F401
     kv_cache_bytes,
 )
 from .mla import mla_cache_bytes, mla_decode_ref, mla_decode_rows_ref  # noqa: F401
+from .backward import prefill_backward_ref, sdpa_backward_rows  # noqa: F401
