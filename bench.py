@@ -383,7 +383,8 @@ def run_single_op(args):
 
     prefill (TFLOP/s, tensor roofline), prefill_paged (TFLOP/s over the visible
     pairs of each chunk against its context), decode (KV GB/s, HBM roofline),
-    decode_window (GB/s of the K/V bytes of the visible tokens only).
+    decode_window (GB/s of the K/V bytes of the visible tokens only), mla_decode
+    (GB/s of the latent cache, with its tensor-core rate reported beside it).
     L2 is flushed before every timed launch; CUDA events on the launching stream.
     """
     import exact_softmax_attention_causal_b200 as attn
@@ -445,6 +446,24 @@ def run_single_op(args):
                                      workspace=ws)
         unit, bound, peak, scale_div = "GB/s", "hbm", peaks["hbm_gbs"], 1e9
         metric = "windowed paged-decode KV GB/s (visible tokens)"
+    elif args.op == "mla_decode":
+        cfg = dict(workloads.MLA_DECODE_WORKLOADS[name])
+        x = workloads.mla_decode_inputs(cfg["B"], cfg["H"], cfg["d_latent"], cfg["d_rope"], len_range=cfg["len_range"],
+                                        block_size=cfg["block_size"], seed=seed)
+        q, cache, bt, sl = x.q.to(dev), x.cache.to(dev), x.block_table.to(dev), x.seq_lens.to(dev)
+        o = torch.empty((cfg["B"], cfg["H"], cfg["d_latent"]), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((cfg["B"], cfg["H"]), dtype=torch.float32, device=dev)
+        ws = torch.empty(attn.mla_decode_workspace_bytes(cfg["B"], cfg["H"], x.max_seq_len), dtype=torch.uint8,
+                         device=dev)
+        work = accounting.mla_decode_bytes(x.seq_lens.tolist(), cfg["d_latent"], cfg["d_rope"])
+        mla_flops = accounting.mla_decode_flops(x.seq_lens.tolist(), cfg["H"], cfg["d_latent"], cfg["d_rope"])
+        msl = x.max_seq_len
+        mla_scale = 1.0 / math.sqrt(cfg["d_head"] + cfg["d_rope"])
+
+        def launch():
+            attn.mla_decode_paged(q, cache, bt, sl, msl, mla_scale, out=o, lse=lse, workspace=ws)
+        unit, bound, peak, scale_div = "GB/s", "hbm", peaks["hbm_gbs"], 1e9
+        metric = "absorbed MLA decode latent-cache GB/s"
     else:
         cfg = dict(workloads.DECODE_WORKLOADS[name])
         x = workloads.paged_decode_inputs(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"], len_range=cfg.get("len_range"),
@@ -491,9 +510,14 @@ def run_single_op(args):
                            l2="flushed (256 MiB write) before every timed launch"),
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                          "traffic": None, "peak_source": tag},
-            "work_per_launch": work, "gpu_launches": args.steps * (2 if args.op.startswith("decode") else 1),
+            "work_per_launch": work,
+            "gpu_launches": args.steps * (2 if args.op.startswith("decode") or args.op == "mla_decode" else 1),
             "clocks": clk.summary(),
         }
+        if args.op == "mla_decode":  # the same launches against the tensor roofline, for context
+            tf = mla_flops / (ms / args.steps / 1e3) / 1e12
+            line["tensor_context"] = {"achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                      "frac": tf / peaks["bf16_tflops"], "flops_per_launch": mla_flops}
         print(json.dumps(line), flush=True)
     return 0
 
@@ -510,11 +534,13 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["step", "prefill", "prefill_paged", "decode", "decode_window"], default="step",
+    ap.add_argument("--op", choices=["step", "prefill", "prefill_paged", "decode", "decode_window", "mla_decode"],
+                    default="step",
                     help="step: the full hot-path step (default); otherwise time one entry point on --workload")
     ap.add_argument("--workload", default=None,
                     choices=sorted(list(workloads.PREFILL_WORKLOADS) + list(workloads.PAGED_PREFILL_WORKLOADS) +
-                                   list(workloads.DECODE_WORKLOADS) + list(workloads.WINDOW_DECODE_WORKLOADS)))
+                                   list(workloads.DECODE_WORKLOADS) + list(workloads.WINDOW_DECODE_WORKLOADS) +
+                                   list(workloads.MLA_DECODE_WORKLOADS)))
     ap.add_argument("--decode-workload", default="paged_decode_b64", choices=sorted(workloads.DECODE_WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -525,10 +551,12 @@ def main(argv=None):
         ap.error("--warmup must be at least 3")
     if args.op != "step":
         defaults = {"prefill": "llama3_8b_causal_gqa", "prefill_paged": "chunked_prefill_b4_q512",
-                    "decode": "paged_decode_b64", "decode_window": "gptoss_window128_sinks_b64"}
+                    "decode": "paged_decode_b64", "decode_window": "gptoss_window128_sinks_b64",
+                    "mla_decode": "deepseek_v2_mla_b64"}
         args.workload = args.workload or defaults[args.op]
         table = {"prefill": workloads.PREFILL_WORKLOADS, "prefill_paged": workloads.PAGED_PREFILL_WORKLOADS,
-                 "decode": workloads.DECODE_WORKLOADS, "decode_window": workloads.WINDOW_DECODE_WORKLOADS}[args.op]
+                 "decode": workloads.DECODE_WORKLOADS, "decode_window": workloads.WINDOW_DECODE_WORKLOADS,
+                 "mla_decode": workloads.MLA_DECODE_WORKLOADS}[args.op]
         if args.workload not in table:
             ap.error(f"--workload {args.workload} is not a {args.op} workload")
         if args.impl == "reference":

@@ -24,7 +24,8 @@ from ._lib import AttnError, STATUS_BIT_DEVICE_CHECK, STATUS_BIT_TIMEOUT  # noqa
 MASKS = {"full": 0, "causal": 1, "window": 2, "sliding_window": 2}
 
 __all__ = ["prefill", "prefill_paged", "decode_paged", "decode_paged_window", "paged_gather", "decode_plan",
-           "decode_workspace_bytes", "decode_window_workspace_bytes", "AttnError", "version"]
+           "decode_workspace_bytes", "decode_window_workspace_bytes", "mla_decode_paged", "mla_decode_workspace_bytes",
+           "AttnError", "version"]
 
 
 def version() -> int:
@@ -218,6 +219,48 @@ def decode_paged_window(q, k_cache, v_cache, block_table, seq_lens, max_seq_len:
                                              workspace.numel() * workspace.element_size(), _ptr(status),
                                              _stream_handle(stream))
     _lib.check(rc, "attn_decode_paged_window")
+    return out, lse
+
+
+def mla_decode_workspace_bytes(B: int, H: int, max_seq_len: int, d_latent: int = 512, d_rope: int = 64) -> int:
+    n = int(_lib.lib().attn_mla_decode_workspace_bytes(B, H, d_latent, d_rope, max_seq_len))
+    if n == 0:
+        raise AttnError(_lib.ATTN_ERR_INVALID_ARG, "attn_mla_decode_workspace_bytes")
+    return n
+
+
+def mla_decode_paged(q, cache, block_table, seq_lens, max_seq_len: int, scale: float, d_latent: int = 512, out=None,
+                     lse=None, workspace=None, status=None, stream=None, return_lse: bool = True):
+    """Absorbed MLA decode: q [B, H, d_latent + d_rope] (absorbed content query,
+    then positional query), cache [num_blocks, block_size, d_latent + d_rope]
+    (latent, then positional key), both bf16. Returns the latent output
+    O [B, H, d_latent] bf16 (apply the value up-projection afterwards) and
+    LSE [B, H] fp32. `scale` is 1 / sqrt(d_head + d_rope).
+    """
+    _need(q, "q", torch.bfloat16, 3)
+    _need(cache, "cache", torch.bfloat16, 3)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    B, H, width = q.shape
+    num_blocks, block_size, width2 = cache.shape
+    if width2 != width or width <= d_latent:
+        raise ValueError("q and cache rows must both be d_latent + d_rope wide")
+    if block_table.shape[0] != B or seq_lens.shape[0] != B:
+        raise ValueError("block_table and seq_lens need one row per sequence")
+    d_rope = width - d_latent
+    if workspace is None:
+        workspace = torch.empty(mla_decode_workspace_bytes(B, H, max_seq_len, d_latent, d_rope), dtype=torch.uint8,
+                                device=q.device)
+    if out is None:
+        out = torch.empty((B, H, d_latent), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    rc = _lib.lib().attn_mla_decode_paged(_ptr(q), _ptr(cache), _ptr(block_table), _ptr(seq_lens), _ptr(out), _ptr(lse),
+                                          B, H, d_latent, d_rope, num_blocks, block_size, block_table.shape[1],
+                                          int(max_seq_len), float(scale), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _ptr(status),
+                                          _stream_handle(stream))
+    _lib.check(rc, "attn_mla_decode_paged")
     return out, lse
 
 

@@ -6,10 +6,24 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
+#include <mutex>
 
 #include "internal.h"
 
 namespace attn {
+
+void* tensor_map_encode_fn() {
+  static void* fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = f;
+  });
+  return fn;
+}
 
 long long wait_budget_cycles() {
   const char* s = std::getenv("ATTN_WAIT_BUDGET_CYCLES");
@@ -196,6 +210,43 @@ int attn_decode_paged_window(const void* q, const void* k_cache, const void* v_c
   return decode_common(q, k_cache, v_cache, block_table, seq_lens, sinks, o, lse, B, Hq, Hkv, d, num_blocks,
                        block_size, max_blocks_per_seq, max_seq_len, window, n_sink, scale, workspace,
                        workspace_bytes, status, stream);
+}
+
+size_t attn_mla_decode_workspace_bytes(int B, int H, int d_latent, int d_rope, int max_seq_len) {
+  if (d_latent != 512 || d_rope != 64) return 0;
+  int sms = 0;
+  if (current_sm_count(&sms) != ATTN_OK) return 0;
+  MlaPlan plan;
+  if (plan_mla(B, H, max_seq_len, sms, &plan) != ATTN_OK) return 0;
+  return mla_workspace_bytes(B, H, plan);
+}
+
+int attn_mla_decode_paged(const void* q, const void* cache, const int32_t* block_table, const int32_t* seq_lens,
+                          void* o, float* lse, int B, int H, int d_latent, int d_rope, int num_blocks, int block_size,
+                          int max_blocks_per_seq, int max_seq_len, float scale, void* workspace,
+                          size_t workspace_bytes, int32_t* status, attn_stream_t stream) {
+  if (!q || !cache || !block_table || !seq_lens || !o) return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || d_latent <= 0 || d_rope <= 0 || num_blocks <= 0 || block_size <= 0 ||
+      max_blocks_per_seq <= 0 || max_seq_len <= 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(max_blocks_per_seq) * block_size < max_seq_len) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(cache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_INVALID_ARG;
+  if (d_latent != 512 || d_rope != 64) return ATTN_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B > 65535 || (H + 63) / 64 > 65535) return ATTN_ERR_UNSUPPORTED;
+  int sms = 0;
+  if (current_sm_count(&sms) != ATTN_OK) return ATTN_ERR_CUDA;
+  MlaPlan plan;
+  if (plan_mla(B, H, max_seq_len, sms, &plan) != ATTN_OK) return ATTN_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < mla_workspace_bytes(B, H, plan))
+    return ATTN_ERR_WORKSPACE;
+  return launch_mla_decode(q, cache, block_table, seq_lens, o, lse, B, H, num_blocks, block_size,
+                           max_blocks_per_seq, max_seq_len, scale, workspace, plan, status,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 int attn_paged_gather(const void* cache, const int32_t* block_table, const int32_t* seq_lens, void* out, int B,

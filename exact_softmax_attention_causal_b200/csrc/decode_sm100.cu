@@ -58,6 +58,11 @@ struct DecodeParams {
   const int32_t* seq_lens;
   float* o_part;    // [B, Hq, splits, D]
   float* lse_part;  // [B, Hq, splits]
+  // One split per sequence: the split kernel writes the final output itself
+  // (normalised, learned sink folded in) and no merge runs.
+  __nv_bfloat16* o;  // [B, Hq, D]
+  float* lse;        // [B, Hq] or nullptr
+  const float* sinks;
   int32_t* status;
   int B, Hq, Hkv, group, hchunks;
   int num_blocks, block_size, max_blocks_per_seq, max_seq_len;
@@ -109,7 +114,23 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk, int row_bytes) {
   return static_cast<uint32_t>(row * row_bytes + ((chunk ^ (row & 7)) << 4));
 }
 
-template <int D>
+// Final output of one row from its unnormalised sum (already divided by the
+// token sum: `inv`) and the tokens' log-sum-exp; folds a learned sink logit
+// into the normaliser. Returns the natural-log LSE written for the row.
+__device__ __forceinline__ float sink_fold(const float* sinks, int h, float lse_tok, float& scale_out, bool& bad) {
+  if (sinks == nullptr) return lse_tok;
+  const float sk = sinks[h];
+  if (!(fabsf(sk) <= 3.0e38f)) bad = true;  // NaN or infinite sink logit
+  const float hi = fmaxf(lse_tok, sk), lo = fminf(lse_tok, sk);
+  const float lse_all = hi + log1pf(__expf(lo - hi));
+  scale_out *= __expf(lse_tok - lse_all);
+  return lse_all;
+}
+
+// WIN: the sequence is read through the visible-sub-block list (sliding window,
+// sink positions); without it every cached token is visible and the list
+// arithmetic folds away at compile time.
+template <int D, bool WIN>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeParams p) {
   using L = DecSmem<D>;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -125,8 +146,19 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   const int lane = threadIdx.x & 31;
 
   const int seq_len = p.seq_lens[b];
-  if (seq_len < 1 || seq_len > p.max_seq_len) return;  // the merge kernel flags this row
-  const VisibleList vis(seq_len, p.window, p.n_sink);
+  const bool direct = (p.splits == 1);
+  if (seq_len < 1 || seq_len > p.max_seq_len) {
+    // the merge kernel flags this row; without a merge this CTA writes its NaN rows
+    if (direct) {
+      const int h0 = kvh * p.group + hc * 16, rows = min(16, p.group - hc * 16);
+      for (int i = threadIdx.x; i < rows * D; i += kDecThreads)
+        p.o[(static_cast<size_t>(b) * p.Hq + h0 + i / D) * D + i % D] = __float2bfloat16_rn(NAN);
+      if (threadIdx.x < rows && p.lse != nullptr) p.lse[static_cast<size_t>(b) * p.Hq + h0 + threadIdx.x] = NAN;
+      if (threadIdx.x == 0) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
+    }
+    return;
+  }
+  const VisibleList vis(seq_len, WIN ? p.window : 0, WIN ? p.n_sink : 0);
   const int u0 = split * (p.chunk / kSub);  // this split's listed sub-blocks [u0, u0 + nsub)
   if (u0 >= vis.nsb) return;  // split past the end of the list: the merge never reads it
   const int nsub = min(p.chunk / kSub, vis.nsb - u0);
@@ -324,22 +356,44 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
         wsc[w] = (wm[w * 16 + r] == neg_inf) ? 0.f : fast_exp2(wm[w * 16 + r] - M);
         Lsum += wsc[w] * wl[w * 16 + r];
       }
-      const float inv = 1.f / Lsum;
-      const size_t prow = (static_cast<size_t>(b) * p.Hq + h0 + r) * p.splits + split;
-      float* dst = p.o_part + prow * D;
-      for (int c = part * (D / 8); c < (part + 1) * (D / 8); c += 4) {
-        float4 acc;
-        float* a = &acc.x;
+      float inv = 1.f / Lsum;
+      if (direct) {
+        bool bad_row = cta_is_bad;
+        const float lse_out = sink_fold(p.sinks, h0 + r, (M + __log2f(Lsum)) * kLn2, inv, bad_row);
+        if (bad_row && part == 0 && !cta_is_bad) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
+        __nv_bfloat16* dst = p.o + (static_cast<size_t>(b) * p.Hq + h0 + r) * D;
+        for (int c = part * (D / 8); c < (part + 1) * (D / 8); c += 8) {
+          uint32_t pk[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float v = 0.f;
+          for (int e = 0; e < 8; e += 2) {
+            float v0 = 0.f, v1 = 0.f;
 #pragma unroll
-          for (int w = 0; w < kDecWarps; ++w) v += wsc[w] * wo[(w * 16 + r) * D + c + e];
-          a[e] = cta_is_bad ? NAN : v * inv;
+            for (int w = 0; w < kDecWarps; ++w) {
+              v0 += wsc[w] * wo[(w * 16 + r) * D + c + e];
+              v1 += wsc[w] * wo[(w * 16 + r) * D + c + e + 1];
+            }
+            pk[e >> 1] = pack_bf16x2(bad_row ? NAN : v0 * inv, bad_row ? NAN : v1 * inv);
+          }
+          *reinterpret_cast<uint4*>(dst + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
-        *reinterpret_cast<float4*>(dst + c) = acc;
+        if (part == 0 && p.lse != nullptr) p.lse[static_cast<size_t>(b) * p.Hq + h0 + r] = bad_row ? NAN : lse_out;
+      } else {
+        const size_t prow = (static_cast<size_t>(b) * p.Hq + h0 + r) * p.splits + split;
+        float* dst = p.o_part + prow * D;
+        for (int c = part * (D / 8); c < (part + 1) * (D / 8); c += 4) {
+          float4 acc;
+          float* a = &acc.x;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kDecWarps; ++w) v += wsc[w] * wo[(w * 16 + r) * D + c + e];
+            a[e] = cta_is_bad ? NAN : v * inv;
+          }
+          *reinterpret_cast<float4*>(dst + c) = acc;
+        }
+        if (part == 0) p.lse_part[prow] = cta_is_bad ? NAN : (M + __log2f(Lsum)) * kLn2;
       }
-      if (part == 0) p.lse_part[prow] = cta_is_bad ? NAN : (M + __log2f(Lsum)) * kLn2;
     }
   }
 }
@@ -355,12 +409,15 @@ struct MergeParams {
   int B, Hq, splits, chunk, max_seq_len, window, n_sink;
 };
 
-// One CTA of 4 warps per (sequence, query head): lse = log sum_s exp(lse_s),
-// O = sum_s exp(lse_s - lse) O_s over the chunks that hold tokens. The warps
-// take every 4th chunk and combine their partial sums in shared memory, so a
-// single long sequence with hundreds of chunks still merges in parallel. A
-// learned sink logit joins the normaliser last (it carries no value).
-constexpr int kMergeWarps = 4;
+// One CTA of 8 warps per (sequence, query head): lse = log sum_s exp(lse_s),
+// O = sum_s exp(lse_s - lse) O_s over the chunks that hold tokens. Warp w
+// takes chunks w, w + 8, ... four at a time (their loads are all in flight
+// before the first is used) and the warps combine their partial sums in
+// shared memory, so a single long sequence with hundreds of chunks still
+// merges in parallel. A learned sink logit joins the normaliser last (it
+// carries no value).
+constexpr int kMergeWarps = 8;
+constexpr int kMergeUnroll = 4;
 
 template <int D>
 __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const MergeParams p) {
@@ -416,15 +473,32 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   const float* obase = p.o_part + row * p.splits * D + lane * PER;
-  for (int s = warp; s < ns; s += kMergeWarps) {
-    const float w = fast_exp2((lrow[s] - M) * kLog2e);
-    sum += w;
-    const float* src = obase + static_cast<size_t>(s) * D;
+  for (int base = warp; base < ns; base += kMergeUnroll * kMergeWarps) {
+    float ls[kMergeUnroll];
+    float v[kMergeUnroll][PER];
 #pragma unroll
-    for (int e = 0; e < PER; e += 2) {
-      const float2 v = *reinterpret_cast<const float2*>(src + e);
-      acc[e] += w * v.x;
-      acc[e + 1] += w * v.y;
+    for (int u = 0; u < kMergeUnroll; ++u) {
+      const int s = base + u * kMergeWarps;
+      ls[u] = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) v[u][e] = 0.f;
+      if (s < ns) {
+        ls[u] = lrow[s];
+        const float* src = obase + static_cast<size_t>(s) * D;
+#pragma unroll
+        for (int e = 0; e < PER; e += 2) {
+          const float2 x = *reinterpret_cast<const float2*>(src + e);
+          v[u][e] = x.x;
+          v[u][e + 1] = x.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kMergeUnroll; ++u) {
+      const float w = (ls[u] == -INFINITY) ? 0.f : fast_exp2((ls[u] - M) * kLog2e);
+      sum += w;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) acc[e] += w * v[u][e];
     }
   }
   if (lane == 0) s_sum[warp] = sum;
@@ -436,19 +510,13 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
 #pragma unroll
     for (int w = 0; w < kMergeWarps; ++w) total += s_sum[w];
     float inv = 1.f / total;
-    float lse_out = M + __logf(total);
-    if (p.sinks != nullptr) {
-      // one more score column s_h with a zero value: log-add it to the
-      // normaliser and shrink the output by the tokens' share of the mass
-      const float sk = p.sinks[row % p.Hq];
-      if (!(fabsf(sk) <= 3.0e38f)) {  // NaN or infinite sink logit
-        any_nan = 1;
-        if (lane == 0) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
-      }
-      const float hi = fmaxf(lse_out, sk), lo = fminf(lse_out, sk);
-      const float lse_all = hi + log1pf(__expf(lo - hi));
-      inv *= __expf(lse_out - lse_all);
-      lse_out = lse_all;
+    // a learned sink: one more score column s_h with a zero value, log-added to
+    // the normaliser; the output shrinks by the tokens' share of the mass
+    bool bad_sink = false;
+    const float lse_out = sink_fold(p.sinks, static_cast<int>(row % p.Hq), M + __logf(total), inv, bad_sink);
+    if (bad_sink) {
+      any_nan = 1;
+      if (lane == 0) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
     }
     float out[PER];
 #pragma unroll
@@ -518,6 +586,9 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   p.seq_lens = seq_lens;
   p.o_part = static_cast<float*>(workspace);
   p.lse_part = p.o_part + static_cast<size_t>(B) * Hq * plan.splits * D;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.sinks = sinks;
   p.status = status;
   p.B = B;
   p.Hq = Hq;
@@ -535,16 +606,26 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   p.scale_log2 = scale * kLog2e;
 
   const int smem = DecSmem<D>::kTotal;
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const auto kernel = window > 0 ? decode_split_kernel<D, true> : decode_split_kernel<D, false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.splits, Hkv * plan.hchunks, B);
-  decode_split_kernel<D><<<grid, kDecThreads, smem, stream>>>(p);
+  kernel<<<grid, kDecThreads, smem, stream>>>(p);
   e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || plan.splits == 1) return e;  // one split: the split kernel wrote the output
 
+  return launch_decode_merge(p.o_part, p.lse_part, seq_lens, sinks, o, lse, B, Hq, D, plan.splits, plan.chunk,
+                             max_seq_len, window, n_sink, status, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_decode_merge(const float* o_part, const float* lse_part, const int32_t* seq_lens,
+                                const float* sinks, void* o, float* lse, int B, int Hq, int d, int splits, int chunk,
+                                int max_seq_len, int window, int n_sink, int32_t* status, cudaStream_t stream) {
   MergeParams m;
-  m.o_part = p.o_part;
-  m.lse_part = p.lse_part;
+  m.o_part = o_part;
+  m.lse_part = lse_part;
   m.seq_lens = seq_lens;
   m.sinks = sinks;
   m.o = static_cast<__nv_bfloat16*>(o);
@@ -552,16 +633,22 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   m.status = status;
   m.B = B;
   m.Hq = Hq;
-  m.splits = plan.splits;
-  m.chunk = plan.chunk;
+  m.splits = splits;
+  m.chunk = chunk;
   m.max_seq_len = max_seq_len;
   m.window = window;
   m.n_sink = n_sink;
-  decode_merge_kernel<D><<<B * Hq, kMergeWarps * 32, 0, stream>>>(m);
+  const dim3 grid(static_cast<unsigned>(B) * static_cast<unsigned>(Hq));
+  if (d == 128)
+    decode_merge_kernel<128><<<grid, kMergeWarps * 32, 0, stream>>>(m);
+  else if (d == 64)
+    decode_merge_kernel<64><<<grid, kMergeWarps * 32, 0, stream>>>(m);
+  else if (d == 512)
+    decode_merge_kernel<512><<<grid, kMergeWarps * 32, 0, stream>>>(m);
+  else
+    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
-
-}  // namespace
 
 size_t decode_workspace_bytes(int B, int Hq, int d, const DecodePlan& plan) {
   const size_t rows = static_cast<size_t>(B) * Hq * plan.splits;
@@ -585,8 +672,11 @@ int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan
   const long long target = 4LL * num_sms;  // CTAs: enough to fill every SM a few times over
   int chunk = 2048;
   while (chunk > 256 && units * ((max_seq_len + chunk - 1) / chunk) < target) chunk >>= 1;
-  out->chunk = chunk;
-  out->splits = (max_seq_len + chunk - 1) / chunk;
+  // spread the 16-token sub-blocks evenly over the splits (no near-empty last split)
+  const int subs = (max_seq_len + 15) / 16;
+  const int nominal_splits = (max_seq_len + chunk - 1) / chunk;
+  out->chunk = 16 * ((subs + nominal_splits - 1) / nominal_splits);
+  out->splits = (max_seq_len + out->chunk - 1) / out->chunk;
   out->hchunks = hchunks;
   return ATTN_OK;
 }

@@ -20,9 +20,13 @@ long long wait_budget_cycles();
 // larger bound, so that a short pipeline budget never cuts a drain short.
 constexpr long long kDrainBudgetCycles = 4000000000LL;
 
+// The driver's cuTensorMapEncodeTiled, looked up once through the runtime
+// (no link against libcuda); nullptr when unavailable.
+void* tensor_map_encode_fn();
+
 struct DecodePlan {
-  int chunk;       // tokens per split (multiple of 16)
-  int splits;      // ceil(max_seq_len / chunk)
+  int chunk;       // tokens per split (multiple of 16, at most 2048)
+  int splits;      // ceil(planning length / chunk)
   int hchunks;     // query-head chunks of <= 16 per K/V head
 };
 
@@ -49,6 +53,22 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
                    int d, int mask_kind, int window, float scale, int32_t* status, cudaStream_t stream);
 
 // Prefill of the newest Nq positions of each sequence against its paged context.
+// Absorbed MLA decode: split kernel + log-sum-exp merge (mla_sm100.cu).
+struct MlaPlan {
+  int chunk;   // tokens per split (multiple of 128)
+  int splits;  // ceil(max_seq_len / chunk)
+};
+int plan_mla(int B, int H, int max_seq_len, int num_sms, MlaPlan* out);
+size_t mla_workspace_bytes(int B, int H, const MlaPlan& plan);
+int launch_mla_decode(const void* q, const void* cache, const int32_t* block_table, const int32_t* seq_lens, void* o,
+                      float* lse, int B, int H, int num_blocks, int block_size, int max_blocks_per_seq,
+                      int max_seq_len, float scale, void* workspace, const MlaPlan& plan, int32_t* status,
+                      cudaStream_t stream);
+// The split-merge kernel of the paged decode, for head widths 64, 128 and 512.
+cudaError_t launch_decode_merge(const float* o_part, const float* lse_part, const int32_t* seq_lens,
+                                const float* sinks, void* o, float* lse, int B, int Hq, int d, int splits, int chunk,
+                                int max_seq_len, int window, int n_sink, int32_t* status, cudaStream_t stream);
+
 int launch_prefill_paged(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
                          const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int d,
                          int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, int mask_kind,

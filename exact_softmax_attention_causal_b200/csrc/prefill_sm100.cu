@@ -57,7 +57,6 @@
 
 #include <cmath>
 #include <cstdint>
-#include <mutex>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -123,15 +122,6 @@ enum : int {
 };
 constexpr int kTmemSlotOff = 224;
 constexpr int kAbortOff = 228;
-
-// Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format: start
-// address, leading and stride byte offsets in 16-byte units, version 1,
-// layout type 2 = SWIZZLE_128B).
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
-         (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
-         (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
 
 // Instruction descriptor for kind::f16: fp32 accumulate, bf16 A and B, A
 // K-major, B K-major (0) or MN-major (1), N >> 3 at bit 17, M >> 4 at bit 24.
@@ -753,23 +743,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  });
-  return fn;
-}
-
 // [heads][n][d] bf16 viewed as a rank-3 tensor (d innermost); box = 64 columns
 // x 128 rows x 1 head, 128-byte swizzle. Rows past n read as zero.
 bool encode_bhnd(CUtensorMap* map, const void* base, int d, int n, int heads, int box_rows = 128) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  const auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encode_fn());
   if (enc == nullptr) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
                               static_cast<cuuint64_t>(heads)};
@@ -788,7 +765,7 @@ bool encode_bhnd(CUtensorMap* map, const void* base, int d, int n, int heads, in
 // box_slots = 1 one token row.
 bool encode_pool(CUtensorMap* map, const void* base, int d, int hkv, int block_size, int num_blocks,
                  int box_slots) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  const auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encode_fn());
   if (enc == nullptr) return false;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(hkv),
                               static_cast<cuuint64_t>(block_size), static_cast<cuuint64_t>(num_blocks)};

@@ -183,6 +183,18 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format: start
+// address, leading and stride byte offsets in 16-byte units, version 1,
+// layout type 2 = SWIZZLE_128B). K-major operands: rows of 128 bytes along K,
+// 8-row groups SBO apart. MN-major operands: rows of 128 bytes along M (or N),
+// one row per K index, 8-row groups SBO apart, 64-element groups along M (N)
+// LBO apart.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
+         (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
 // Arrive on an mbarrier once every tcgen05 op issued so far by this thread completes.
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)

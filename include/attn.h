@@ -21,6 +21,9 @@
  *                        sections 9, 10 and 12).
  *   attn_prefill_paged - the newest Nq positions of each sequence against its
  *                        paged context (prefix / chunked prefill).
+ *   attn_mla_decode_paged - absorbed Multi-head Latent Attention decode over a
+ *                        paged latent cache ("Modern Attention Mechanisms",
+ *                        section 7; "Module 09", the MLA section).
  *
  * Conventions shared by every entry point:
  *   - Pointers named q, k, v, o, lse, k_cache, v_cache, block_table, seq_lens,
@@ -244,6 +247,50 @@ ATTN_API int attn_decode_paged_window(const void* q, const void* k_cache, const 
                                       int max_blocks_per_seq, int max_seq_len, int window, int n_sink, float scale,
                                       void* workspace, size_t workspace_bytes, int32_t* status,
                                       attn_stream_t stream);
+
+/*
+ * attn_mla_decode_workspace_bytes - bytes of device workspace
+ * attn_mla_decode_paged needs (fp32 partial latent outputs [B, H, splits, 512]
+ * and partial log-sum-exps [B, H, splits]). Returns 0 for invalid or
+ * unsupported sizes.
+ */
+ATTN_API size_t attn_mla_decode_workspace_bytes(int B, int H, int d_latent, int d_rope, int max_seq_len);
+
+/*
+ * attn_mla_decode_paged - one new query token per sequence, H heads, against a
+ * paged cache of Multi-head Latent Attention rows, in the absorbed form.
+ *
+ * Defined by "Module 5. Modern Attention Mechanisms", section 7 (with
+ * k_t = A c_t and v_t = B c_t: q.k_t = (A^T q).c_t and
+ * sum_t p_t v_t = B (sum_t p_t c_t); a separate positional key whose term is
+ * added to the logit) and "Module 09: Efficient Attention", the MLA section
+ * (key and query are the concatenations [content ; rope], the logit is their
+ * dot product over sqrt(d_head + d_h^R), the cache holds d_c + d_h^R numbers
+ * per token). Token t of sequence b is row [c_t ; k^R_t] in slot
+ * t % block_size of block block_table[b][t / block_size]; head h's query is
+ * [A_h^T q^C_h ; q^R_h]; every cached token is visible. The output is the
+ * latent sum_t p_t c_t: the caller applies the value up-projection B_h.
+ *
+ *   q            [B, H, d_latent + d_rope] bf16                         read
+ *   cache        [num_blocks, block_size, d_latent + d_rope] bf16       read (only referenced rows)
+ *   block_table  [B, max_blocks_per_seq] int32, as for attn_decode_paged read
+ *   seq_lens     [B] int32, each in [1, max_seq_len]                     read
+ *   o            [B, H, d_latent] bf16                                   written
+ *   lse          [B, H] fp32, natural log, or NULL                      written
+ *   d_latent, d_rope   must be 512 and 64 (DeepSeek-V2's widths), else
+ *                ATTN_ERR_UNSUPPORTED
+ *   block_size   16, 32, 64 or 128
+ *   scale        the logit scale, 1 / sqrt(d_head + d_rope) per the pages
+ *   workspace    at least attn_mla_decode_workspace_bytes(...) bytes, 16-byte aligned
+ *
+ * Bad referenced table entries and seq_lens are handled as in
+ * attn_decode_paged (NaN rows, ATTN_STATUS_BIT_DEVICE_CHECK).
+ */
+ATTN_API int attn_mla_decode_paged(const void* q, const void* cache, const int32_t* block_table,
+                                   const int32_t* seq_lens, void* o, float* lse, int B, int H, int d_latent,
+                                   int d_rope, int num_blocks, int block_size, int max_blocks_per_seq,
+                                   int max_seq_len, float scale, void* workspace, size_t workspace_bytes,
+                                   int32_t* status, attn_stream_t stream);
 
 /*
  * attn_paged_gather - walk every sequence's block table into a contiguous

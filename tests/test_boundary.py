@@ -126,6 +126,33 @@ def test_decode_window_workspace_rejects_bad_sizes():
     assert lib.attn_decode_window_workspace_bytes(2, 8, 2, 128, 64, 16, -1, 0) == 0
 
 
+def _mla(**kw):
+    a = dict(q=FAKE, c=FAKE, bt=FAKE, sl=FAKE, o=FAKE, lse=NULL, B=2, H=128, dc=512, dr=64, nb=10, bs=16, mb=4, msl=64,
+             scale=0.07, ws=FAKE, wsb=1 << 20)
+    a.update(kw)
+    return _lib.lib().attn_mla_decode_paged(a["q"], a["c"], a["bt"], a["sl"], a["o"], a["lse"], a["B"], a["H"],
+                                            a["dc"], a["dr"], a["nb"], a["bs"], a["mb"], a["msl"], a["scale"],
+                                            a["ws"], a["wsb"], NULL, NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=NULL), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(c=ctypes.c_void_p(0x10008)), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(H=0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(mb=3), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(scale=0.0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(dc=256), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(dr=32), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(bs=48, mb=2), _lib.ATTN_ERR_UNSUPPORTED),
+])
+def test_mla_rejects_bad_arguments(kw, code):
+    assert _mla(**kw) == code
+
+
+def test_mla_workspace_rejects_unsupported_widths():
+    assert _lib.lib().attn_mla_decode_workspace_bytes(2, 128, 256, 64, 1024) == 0
+
+
 def _prefill_paged(**kw):
     a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, sl=FAKE, o=FAKE, lse=NULL, B=2, Hq=8, Hkv=2, Nq=64, d=128, nb=10,
              bs=16, mb=8, msl=128, mask=1, window=0, scale=0.1)
@@ -168,16 +195,21 @@ def _plan(B, Hq, Hkv, L, sms=148):
 def test_decode_plan_covers_the_sequence(B, Hq, Hkv, L):
     rc, chunk, splits = _plan(B, Hq, Hkv, L)
     assert rc == _lib.ATTN_OK
-    assert chunk % 16 == 0 and 256 <= chunk <= 2048
+    assert chunk % 16 == 0 and 16 <= chunk <= 2048
     assert splits == -(-L // chunk)
-    # enough (sequence, kv head, head chunk, split) units to fill 148 SMs, unless chunks are at their minimum
+    # the 16-token sub-blocks are spread evenly: no split holds less than a sub-block less than another
+    subs = -(-L // 16)
+    assert subs - (splits - 1) * (chunk // 16) >= max(1, chunk // 16 - splits)
+    # enough (sequence, kv head, head chunk, split) units for several waves on 148 SMs, unless chunks are small
     units = B * Hkv * -(-(Hq // Hkv) // 16) * splits
-    assert units >= 4 * 148 or chunk == 256
+    assert units >= 4 * 148 or chunk <= 256
 
 
 def test_decode_plan_examples():
     assert _plan(64, 32, 8, 32768)[1:] == (2048, 16)
     assert _plan(1, 32, 1, 131072)[1:] == (256, 512)  # 2 head chunks x 512 splits
+    assert _plan(1, 32, 8, 131072)[1:] == (1024, 128)
+    assert _plan(64, 32, 8, 4128)[1:] == (1376, 3)  # a 4096 window + 4 sinks: 258 sub-blocks in 3 even splits
     assert _plan(0, 32, 1, 131072)[0] == _lib.ATTN_ERR_INVALID_ARG
     assert _plan(1, 32, 3, 100)[0] == _lib.ATTN_ERR_INVALID_ARG
 
