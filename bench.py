@@ -384,7 +384,8 @@ def run_single_op(args):
     prefill (TFLOP/s, tensor roofline), prefill_paged (TFLOP/s over the visible
     pairs of each chunk against its context), decode (KV GB/s, HBM roofline),
     decode_window (GB/s of the K/V bytes of the visible tokens only), mla_decode
-    (GB/s of the latent cache, with its tensor-core rate reported beside it).
+    (GB/s of the latent cache, with its tensor-core rate reported beside it),
+    prefill_backward (TFLOP/s counting 5 products per visible pair).
     L2 is flushed before every timed launch; CUDA events on the launching stream.
     """
     import exact_softmax_attention_causal_b200 as attn
@@ -446,6 +447,23 @@ def run_single_op(args):
                                      workspace=ws)
         unit, bound, peak, scale_div = "GB/s", "hbm", peaks["hbm_gbs"], 1e9
         metric = "windowed paged-decode KV GB/s (visible tokens)"
+    elif args.op == "prefill_backward":
+        cfg = workloads.PREFILL_WORKLOADS[name]
+        x = workloads.prefill_inputs(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["N"], cfg["d"], seed)
+        q, k, v = x.q.to(dev), x.k.to(dev), x.v.to(dev)
+        gen = torch.Generator("cpu").manual_seed(10_000 + seed)
+        d_o = torch.randn(q.shape, generator=gen, dtype=torch.float32).to(torch.bfloat16).to(dev)
+        o, lse = attn.prefill(q, k, v, mask=cfg["mask"], window=cfg["window"])
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(attn.prefill_backward_workspace_bytes(cfg["B"], cfg["Hq"], cfg["N"]), dtype=torch.uint8,
+                         device=dev)
+        work = accounting.prefill_backward_flops(cfg["B"], cfg["Hq"], cfg["N"], cfg["d"], cfg["mask"], cfg["window"])
+
+        def launch():
+            attn.prefill_backward(q, k, v, o, lse, d_o, mask=cfg["mask"], window=cfg["window"], dq=dq, dk=dk, dv=dv,
+                                  workspace=ws)
+        unit, bound, peak, scale_div = "TFLOP/s", "tensor", peaks["bf16_tflops"], 1e12
+        metric = "attention backward TFLOP/s (5 products per visible pair)"
     elif args.op == "mla_decode":
         cfg = dict(workloads.MLA_DECODE_WORKLOADS[name])
         x = workloads.mla_decode_inputs(cfg["B"], cfg["H"], cfg["d_latent"], cfg["d_rope"], len_range=cfg["len_range"],
@@ -511,7 +529,8 @@ def run_single_op(args):
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                          "traffic": None, "peak_source": tag},
             "work_per_launch": work,
-            "gpu_launches": args.steps * (2 if args.op.startswith("decode") or args.op == "mla_decode" else 1),
+            "gpu_launches": args.steps * {"prefill_backward": 3, "mla_decode": 2, "decode": 2,
+                                          "decode_window": 2}.get(args.op, 1),
             "clocks": clk.summary(),
         }
         if args.op == "mla_decode":  # the same launches against the tensor roofline, for context
@@ -534,7 +553,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["step", "prefill", "prefill_paged", "decode", "decode_window", "mla_decode"],
+    ap.add_argument("--op", choices=["step", "prefill", "prefill_paged", "decode", "decode_window", "mla_decode",
+                                     "prefill_backward"],
                     default="step",
                     help="step: the full hot-path step (default); otherwise time one entry point on --workload")
     ap.add_argument("--workload", default=None,
@@ -552,11 +572,12 @@ def main(argv=None):
     if args.op != "step":
         defaults = {"prefill": "llama3_8b_causal_gqa", "prefill_paged": "chunked_prefill_b4_q512",
                     "decode": "paged_decode_b64", "decode_window": "gptoss_window128_sinks_b64",
-                    "mla_decode": "deepseek_v2_mla_b64"}
+                    "mla_decode": "deepseek_v2_mla_b64", "prefill_backward": "llama3_8b_causal_gqa"}
         args.workload = args.workload or defaults[args.op]
         table = {"prefill": workloads.PREFILL_WORKLOADS, "prefill_paged": workloads.PAGED_PREFILL_WORKLOADS,
                  "decode": workloads.DECODE_WORKLOADS, "decode_window": workloads.WINDOW_DECODE_WORKLOADS,
-                 "mla_decode": workloads.MLA_DECODE_WORKLOADS}[args.op]
+                 "mla_decode": workloads.MLA_DECODE_WORKLOADS,
+                 "prefill_backward": workloads.PREFILL_WORKLOADS}[args.op]
         if args.workload not in table:
             ap.error(f"--workload {args.workload} is not a {args.op} workload")
         if args.impl == "reference":

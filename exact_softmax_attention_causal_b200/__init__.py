@@ -25,6 +25,7 @@ MASKS = {"full": 0, "causal": 1, "window": 2, "sliding_window": 2}
 
 __all__ = ["prefill", "prefill_paged", "decode_paged", "decode_paged_window", "paged_gather", "decode_plan",
            "decode_workspace_bytes", "decode_window_workspace_bytes", "mla_decode_paged", "mla_decode_workspace_bytes",
+           "prefill_backward", "prefill_backward_workspace_bytes",
            "AttnError", "version"]
 
 
@@ -82,6 +83,43 @@ def prefill(q, k, v, mask: str = "causal", window: int = 0, scale: float | None 
                                  int(window), float(scale), _ptr(status), _stream_handle(stream))
     _lib.check(rc, "attn_prefill")
     return out, lse
+
+
+def prefill_backward_workspace_bytes(B: int, Hq: int, N: int) -> int:
+    n = int(_lib.lib().attn_prefill_backward_workspace_bytes(B, Hq, N))
+    if n == 0:
+        raise AttnError(_lib.ATTN_ERR_INVALID_ARG, "attn_prefill_backward_workspace_bytes")
+    return n
+
+
+def prefill_backward(q, k, v, o, lse, d_o, mask: str = "causal", window: int = 0, scale: float | None = None,
+                     dq=None, dk=None, dv=None, workspace=None, status=None, stream=None):
+    """Gradients (dQ, dK, dV) of prefill() for the output gradient d_o, from the
+    forward's inputs, output O and LSE. Shapes as in prefill(); bf16 results."""
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (d_o, "d_o")):
+        _need(t, name, torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape or o.shape != q.shape or d_o.shape != q.shape:
+        raise ValueError("k, v must be [B, Hkv, N, d]; o and d_o like q")
+    if lse.shape != (B, Hq, N):
+        raise ValueError("lse must be [B, Hq, N]")
+    if mask not in MASKS:
+        raise ValueError(f"mask must be one of {sorted(MASKS)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(prefill_backward_workspace_bytes(B, Hq, N), dtype=torch.uint8, device=q.device)
+    rc = _lib.lib().attn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(d_o), _ptr(lse), _ptr(dq), _ptr(dk),
+                                          _ptr(dv), B, Hq, Hkv, N, d, MASKS[mask], int(window), float(scale),
+                                          _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+                                          _stream_handle(stream))
+    _lib.check(rc, "attn_prefill_backward")
+    return dq, dk, dv
 
 
 def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int, mask: str = "causal",

@@ -22,6 +22,8 @@ SYMBOLS = (
     "attn_decode_paged_noalloc",
     "attn_decode_window_workspace_bytes",
     "attn_decode_paged_window",
+    "attn_prefill_backward_workspace_bytes",
+    "attn_prefill_backward",
     "attn_mla_decode_workspace_bytes",
     "attn_mla_decode_paged",
     "attn_paged_gather",
@@ -70,6 +72,11 @@ def _declare(lib):
     lib.attn_decode_paged_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
                                              _i, _i, _f, _vp, _sz, _vp, _vp]
     lib.attn_decode_paged_window.restype = _i
+    lib.attn_prefill_backward_workspace_bytes.argtypes = [_i, _i, _i]
+    lib.attn_prefill_backward_workspace_bytes.restype = _sz
+    lib.attn_prefill_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
+                                          _vp, _sz, _vp, _vp]
+    lib.attn_prefill_backward.restype = _i
     lib.attn_mla_decode_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
     lib.attn_mla_decode_workspace_bytes.restype = _sz
     lib.attn_mla_decode_paged.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _sz,

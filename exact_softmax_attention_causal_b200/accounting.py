@@ -90,3 +90,9 @@ def mla_decode_bytes(seq_lens, d_latent: int, d_rope: int) -> int:
 def mla_decode_flops(seq_lens, H: int, d_latent: int, d_rope: int) -> int:
     """2 (d_c + d_R) for the logit plus 2 d_c for the latent output, per head per token."""
     return sum(int(n) for n in seq_lens) * H * (2 * (d_latent + d_rope) + 2 * d_latent)
+
+
+def prefill_backward_flops(B: int, Hq: int, N: int, d: int, mask: str, window: int = 0) -> int:
+    """Five d-long products per visible (query, key) pair per query head (S
+    recomputed, dP, dV, dK, dQ): 10 d FLOPs per pair, 2.5 x the forward."""
+    return 10 * B * Hq * d * visible_pairs(N, mask, window)

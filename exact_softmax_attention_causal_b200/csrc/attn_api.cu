@@ -212,6 +212,35 @@ int attn_decode_paged_window(const void* q, const void* k_cache, const void* v_c
                        workspace_bytes, status, stream);
 }
 
+size_t attn_prefill_backward_workspace_bytes(int B, int Hq, int N) {
+  if (B <= 0 || Hq <= 0 || N <= 0) return 0;
+  return backward_workspace_bytes(B, Hq, N);
+}
+
+int attn_prefill_backward(const void* q, const void* k, const void* v, const void* o, const void* d_o,
+                          const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
+                          int mask_kind, int window, float scale, void* workspace, size_t workspace_bytes,
+                          int32_t* status, attn_stream_t stream) {
+  if (!q || !k || !v || !o || !d_o || !lse || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (mask_kind != ATTN_MASK_FULL && mask_kind != ATTN_MASK_CAUSAL && mask_kind != ATTN_MASK_SLIDING_WINDOW)
+    return ATTN_ERR_INVALID_ARG;
+  if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window < 1) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(d_o) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (B > 65535 || Hq > 65535 || static_cast<long long>(B) * Hq * N > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 15u) ||
+      workspace_bytes < backward_workspace_bytes(B, Hq, N))
+    return ATTN_ERR_WORKSPACE;
+  if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window >= N) mask_kind = ATTN_MASK_CAUSAL;
+  return launch_backward(q, k, v, o, d_o, lse, dq, dk, dv, B, Hq, Hkv, N, d, mask_kind, window, scale, workspace,
+                         status, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t attn_mla_decode_workspace_bytes(int B, int H, int d_latent, int d_rope, int max_seq_len) {
   if (d_latent != 512 || d_rope != 64) return 0;
   int sms = 0;

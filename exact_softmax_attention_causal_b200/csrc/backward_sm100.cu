@@ -1,0 +1,645 @@
+// Attention backward pass on the 5th-generation tensor cores (tcgen05 + TMEM
+// + TMA): dQ, dK, dV of prefill attention.
+//
+// What it computes: the derivative of O = softmax(scale Q K^T + M) V
+// ("Module 5. Modern Attention Mechanisms", section 4; grouped-query heads as
+// in section 6) for an upstream gradient dO, by the chain rule:
+//   P  = exp(scale S - LSE) (S = Q K^T, LSE the forward's log-sum-exp)
+//   dV = P^T dO,  dP = dO V^T,  dS = P (dP - D),  D = rowsum(dO * O)
+//   dQ = scale dS K,  dK = scale dS^T Q,
+// with dK and dV of a K/V head summed over the query heads of its group.
+// As the "Inference attention" post (section "FlashAttention") says of the
+// backward pass, S and P are recomputed tile by tile from the saved LSE
+// instead of being stored.
+//
+// How: three kernels, no atomics (the result does not depend on scheduling):
+//   bwd_rowdot_kernel  D = rowsum(dO * O), one warp per row, fp32.
+//   bwd_dkdv_kernel    one CTA per (batch, K/V head, 128-key tile): for every
+//                      query head of the group and every 128-row query tile
+//                      that sees the key tile, S^T = K Q^T and dP^T = V dO^T
+//                      into TMEM (M = keys), P^T and dS^T (bf16) written back
+//                      over them, then dV += P^T dO and dK += dS^T Q with the
+//                      probabilities read from TMEM.
+//   bwd_dq_kernel      one CTA per (batch, query head, 128-row query tile):
+//                      S = Q K^T and dP = dO V^T per key tile, dS (bf16) over
+//                      S, then dQ += dS K.
+// Each recomputes S once more than a single fused kernel would (seven
+// 128x128xd products per tile pair instead of five), in exchange for
+// deterministic sums without a dQ accumulator shared between CTAs.
+//
+// Roles in both tile kernels (192 threads): warps 0-3 compute P and dS (thread
+// i owns TMEM lane i = one key row (dK/dV) or query row (dQ)), warp 4 is the
+// TMA producer, warp 5 issues the MMAs and owns TMEM. Every pipeline wait is
+// bounded; on expiry the CTA records ATTN_STATUS_BIT_TIMEOUT, writes NaN, drains
+// and exits.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace attn {
+namespace {
+
+constexpr int kT = 128;             // rows per tile (TMEM lanes), keys per tile
+constexpr int kBwdThreads = 192;
+constexpr int kBwdTmaWarp = 4;
+constexpr int kBwdMmaWarp = 5;
+constexpr int kBox = 128 * 128;     // bytes of one 64-column, 128-row swizzled box
+
+struct BwdParams {
+  const __nv_bfloat16* o;
+  const __nv_bfloat16* d_o;
+  const float* lse;   // [B, Hq, N] natural log (forward output)
+  float* dvec;        // [B, Hq, N] D = rowsum(dO * O)
+  __nv_bfloat16* dq;  // [B, Hq, N, d]
+  __nv_bfloat16* dk;  // [B, Hkv, N, d]
+  __nv_bfloat16* dv;  // [B, Hkv, N, d]
+  int32_t* status;
+  int B, Hq, Hkv, N, group, mask_kind, window, ntiles;
+  float scale, scale_log2;
+  long long budget;
+};
+
+__device__ __forceinline__ void bwd_abort(volatile int* abort_flag, int32_t* status) {
+  *abort_flag = 1;
+  if (status != nullptr) atomicOr(status, ATTN_STATUS_BIT_TIMEOUT);
+}
+
+// key kpos visible to query qpos (both < N checked by the caller)
+__device__ __forceinline__ bool bwd_visible(const BwdParams& p, int qpos, int kpos) {
+  if (p.mask_kind == ATTN_MASK_FULL) return true;
+  if (kpos > qpos) return false;
+  return p.mask_kind != ATTN_MASK_SLIDING_WINDOW || qpos - kpos < p.window;
+}
+
+// Query tiles [lo, hi] that see key tile j, and key tiles that query tile i sees.
+__device__ __forceinline__ void q_tiles_of_key_tile(const BwdParams& p, int j, int& lo, int& hi) {
+  lo = 0;
+  hi = p.ntiles - 1;
+  if (p.mask_kind != ATTN_MASK_FULL) lo = j;
+  if (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) hi = min(hi, (j * kT + kT - 1 + p.window - 1) / kT);
+}
+__device__ __forceinline__ void k_tiles_of_q_tile(const BwdParams& p, int i, int& lo, int& hi) {
+  lo = 0;
+  hi = p.ntiles - 1;
+  if (p.mask_kind != ATTN_MASK_FULL) hi = i;
+  if (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) lo = max(0, i * kT - p.window + 1) / kT;
+}
+
+// kind::f16 instruction descriptor (fp32 accumulate, bf16 inputs).
+__host__ __device__ constexpr uint32_t idesc_bwd(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn) << 15) |
+         (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D x d/16 steps of a product with both operands K-major in shared memory
+// (K dimension = head dim: 64-column boxes of 16 KB hold 4 steps of 32 bytes).
+template <int D>
+__device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint64_t da, uint64_t db, uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kBox + (kk & 3) * 32) >> 4);
+    tc_mma_ss(d_tmem, da + off, db + off, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+// 128 / 16 steps of D (+)= A[tmem: bf16 pairs, 8 columns per step] * B[smem, MN-major, 16 rows per step].
+__device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t db, uint32_t idesc,
+                                           bool first) {
+#pragma unroll
+  for (int kk = 0; kk < kT / 16; ++kk)
+    tc_mma_ts(d_tmem, a_tmem + 8u * kk, db + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
+              (!first || kk > 0) ? 1u : 0u);
+}
+
+// ---------------------------------------------------------------------------
+// D = rowsum(dO * O): one warp per (batch, head, row)
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void bwd_rowdot_kernel(const BwdParams p) {
+  const size_t rows = static_cast<size_t>(p.B) * p.Hq * p.N;
+  const size_t row = blockIdx.x * static_cast<size_t>(blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  constexpr int PER = D / 32;
+  const __nv_bfloat16* a = p.o + row * D + lane * PER;
+  const __nv_bfloat16* g = p.d_o + row * D + lane * PER;
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < PER; e += 2) {
+    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(a + e));
+    const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(g + e));
+    s += x.x * y.x + x.y * y.y;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) p.dvec[row] = s;
+}
+
+// Shared-memory plan of the tile kernels (1024-byte aligned):
+template <int D>
+struct BwdCfg {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kTile = kHalves * kBox;  // one 128 x D bf16 tile
+  // dK/dV: K, V resident; two stages of (Q, dO) and their LSE / D rows.
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kKOff + kTile;
+  static constexpr int kQOff = kVOff + kTile;          // + stage * 2 * kTile
+  static constexpr int kStageBytes = 2 * kTile;        // Q then dO
+  static constexpr int kRowOff = kQOff + 2 * kStageBytes;  // [stage][LSE 128 | D 128] fp32
+  static constexpr int kBarOff = kRowOff + 2 * 2 * kT * 4;
+  static constexpr int kBytes = kBarOff + 256;
+  static constexpr int kAlloc = kBytes + 1024;
+  // TMEM columns: S^T (or S) 128, dP^T (or dP) 128, then the accumulators.
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 256 + D;
+};
+
+enum : int {
+  kBbKV = 0,       // K and V (dK/dV kernel) or Q and dO (dQ kernel) resident tiles landed
+  kBbFull = 1,     // + stage (2)
+  kBbEmpty = 3,    // + stage (2)
+  kBbS = 5,        // S and dP of the current pair are in TMEM
+  kBbP = 6,        // P / dS written back (4 softmax warps)
+  kBbAcc = 7,      // accumulators final
+  kBbDrain = 8,
+};
+constexpr int kBwdTmemSlot = 128;
+constexpr int kBwdAbort = 132;
+
+// ---------------------------------------------------------------------------
+// dK, dV: one CTA per (key tile, K/V head, batch)
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw_u32);
+  const int j = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int qlo, qhi;
+  q_tiles_of_key_tile(p, j, qlo, qhi);
+  const int nq = qhi - qlo + 1;
+  const int iters = p.group * nq;  // (query head of the group, query tile) pairs, head-major
+
+  const uint32_t bars = sbase + C::kBarOff;
+  auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + kBwdTmemSlot);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + kBwdAbort);
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBbKV), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBbFull + s), 1);
+      mbar_init(bar(kBbEmpty + s), 1);
+    }
+    mbar_init(bar(kBbS), 1);
+    mbar_init(bar(kBbP), 4);
+    mbar_init(bar(kBbAcc), 1);
+    mbar_init(bar(kBbDrain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const long long budget = p.budget;
+
+  if (warp == kBwdTmaWarp) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- TMA producer
+      const int zkv = b * p.Hkv + kvh;
+      mbar_arrive_expect_tx(bar(kBbKV), 2 * C::kTile);
+      for (int hh = 0; hh < C::kHalves; ++hh) {
+        tma_load_3d(sbase + C::kKOff + hh * kBox, &tm_k, bar(kBbKV), hh * 64, j * kT, zkv);
+        tma_load_3d(sbase + C::kVOff + hh * kBox, &tm_v, bar(kBbKV), hh * 64, j * kT, zkv);
+      }
+      int issued[2] = {0, 0};
+      bool ok = true;
+      for (int t = 0; t < iters && ok; ++t) {
+        const int s = t & 1;
+        if (t >= 2 && !mbar_wait_bounded(bar(kBbEmpty + s), ((t - 2) >> 1) & 1, budget, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int h = kvh * p.group + t / nq, i = qlo + t % nq;
+        const int zq = b * p.Hq + h;
+        const uint32_t st = sbase + C::kQOff + s * C::kStageBytes;
+        // the LSE and D rows of the tile travel by plain loads (softmax warps); only Q and dO by TMA
+        mbar_arrive_expect_tx(bar(kBbFull + s), 2 * C::kTile);
+        for (int hh = 0; hh < C::kHalves; ++hh) {
+          tma_load_3d(st + hh * kBox, &tm_q, bar(kBbFull + s), hh * 64, i * kT, zq);
+          tma_load_3d(st + C::kTile + hh * kBox, &tm_do, bar(kBbFull + s), hh * 64, i * kT, zq);
+        }
+        issued[s] = t / 2 + 1;
+      }
+      if (!ok) bwd_abort(abort_flag, p.status);
+      volatile int never = 0;
+      mbar_wait_bounded(bar(kBbKV), 0, kDrainBudgetCycles, &never);
+      for (int s = 0; s < 2; ++s)
+        if (issued[s] > 0) mbar_wait_bounded(bar(kBbFull + s), (issued[s] - 1) & 1, kDrainBudgetCycles, &never);
+    }
+  } else if (warp == kBwdMmaWarp) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      const uint64_t dk = desc_sw128(sbase + C::kKOff, 16, 1024);
+      const uint64_t dvv = desc_sw128(sbase + C::kVOff, 16, 1024);
+      constexpr uint32_t kIdS = idesc_bwd(kT, kT, 0, 0);   // S^T = K Q^T, dP^T = V dO^T
+      constexpr uint32_t kIdAcc = idesc_bwd(kT, D, 0, 1);  // dV += P^T dO, dK += dS^T Q (B MN-major)
+      bool ok = mbar_wait_bounded(bar(kBbKV), 0, budget, abort_flag);
+      for (int t = 0; t < iters && ok; ++t) {
+        const int s = t & 1;
+        const uint32_t st = sbase + C::kQOff + s * C::kStageBytes;
+        if (!mbar_wait_bounded(bar(kBbFull + s), (t >> 1) & 1, budget, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        mma_kmajor<D>(tmem + C::kColS, dk, desc_sw128(st, 16, 1024), kIdS);
+        mma_kmajor<D>(tmem + C::kColDP, dvv, desc_sw128(st + C::kTile, 16, 1024), kIdS);
+        tc_commit(bar(kBbS));
+        if (!mbar_wait_bounded(bar(kBbP), t & 1, budget, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // B = dO (then Q) as an MN-major operand: N = head dim (64-column boxes kBox apart),
+        // K = query rows (16 per step, 2 KB apart)
+        mma_tmem_a(tmem + C::kColAcc0, tmem + C::kColS, desc_sw128(st + C::kTile, kBox, 1024), kIdAcc, t == 0);
+        mma_tmem_a(tmem + C::kColAcc1, tmem + C::kColDP, desc_sw128(st, kBox, 1024), kIdAcc, t == 0);
+        tc_commit(bar(kBbEmpty + s));
+      }
+      if (!ok) bwd_abort(abort_flag, p.status);
+      tc_commit(bar(kBbAcc));
+      tc_commit(bar(kBbDrain));
+      volatile int never = 0;
+      mbar_wait_bounded(bar(kBbDrain), 0, kDrainBudgetCycles, &never);
+    }
+  } else {
+    // ------------------------------------------------------------ P / dS warps 0-3
+    const int r = threadIdx.x;  // key row of the tile = TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int kpos = j * kT + r;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int t = 0; t < iters; ++t) {
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbS), t & 1, budget, abort_flag));
+      if (!ok) break;  // no named barriers here: leaving early strands no other warp
+      tc_fence_after();
+      const int h = kvh * p.group + t / nq, i = qlo + t % nq;
+      const size_t rowbase = (static_cast<size_t>(b) * p.Hq + h) * p.N + static_cast<size_t>(i) * kT;
+      const bool full_tile = (p.mask_kind == ATTN_MASK_FULL || (i > j && (p.mask_kind == ATTN_MASK_CAUSAL ||
+                                                                          (i * kT + kT - 1) - j * kT < p.window))) &&
+                             (i * kT + kT <= p.N) && (j * kT + kT <= p.N);
+#pragma unroll 1
+      for (int c = 0; c < kT / 32; ++c) {
+        uint32_t sv[32], dpv[32];
+        tmem_ld_32x32b_x32(lane_base + C::kColS + 32u * c, sv);
+        tmem_ld_32x32b_x32(lane_base + C::kColDP + 32u * c, dpv);
+        // LSE (base 2) and D of the 32 query columns: the same addresses for every
+        // thread of the warp (one broadcast load each); rows past N see nothing
+        float l2[32], dd[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const bool in = (i * kT + 32 * c + e) < p.N;
+          l2[e] = in ? __ldg(p.lse + rowbase + 32 * c + e) * kLog2e : INFINITY;
+          dd[e] = in ? __ldg(p.dvec + rowbase + 32 * c + e) : 0.f;
+        }
+        tc_wait_ld();
+        uint32_t pk[16], dsk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float pr[2], ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int qpos = i * kT + 32 * c + e + u;
+            const bool vis = full_tile || (qpos < p.N && kpos < p.N && bwd_visible(p, qpos, kpos));
+            pr[u] = vis ? fast_exp2(__uint_as_float(sv[e + u]) * sl2 - l2[e + u]) : 0.f;
+            ds[u] = pr[u] * (__uint_as_float(dpv[e + u]) - dd[e + u]);
+          }
+          pk[e >> 1] = pack_bf16x2(pr[0], pr[1]);
+          dsk[e >> 1] = pack_bf16x2(ds[0], ds[1]);
+        }
+        // bf16 pairs over the columns already read: P^T at kColS + 16 c, dS^T at kColDP + 16 c
+        tmem_st_32x32b_x16(lane_base + C::kColS + 16u * c, pk);
+        tmem_st_32x32b_x16(lane_base + C::kColDP + 16u * c, dsk);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBbP));
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbAcc), 0, budget, abort_flag));
+    if (!ok) bwd_abort(abort_flag, p.status);
+    tc_fence_after();
+    // TMEM loads are warp-collective: every lane runs them, only rows < N are stored
+    const bool store = kpos < p.N;
+    __nv_bfloat16* dvrow = p.dv + ((static_cast<size_t>(b) * p.Hkv + kvh) * p.N + (store ? kpos : 0)) * D;
+    __nv_bfloat16* dkrow = p.dk + ((static_cast<size_t>(b) * p.Hkv + kvh) * p.N + (store ? kpos : 0)) * D;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t va[32], ka[32];
+      tmem_ld_32x32b_x32(lane_base + C::kColAcc0 + 32u * c, va);
+      tmem_ld_32x32b_x32(lane_base + C::kColAcc1 + 32u * c, ka);
+      tc_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; e += 8) {
+        uint32_t pv[4], pkk[4];
+#pragma unroll
+        for (int u = 0; u < 8; u += 2) {
+          pv[u >> 1] = pack_bf16x2(ok ? __uint_as_float(va[e + u]) : NAN, ok ? __uint_as_float(va[e + u + 1]) : NAN);
+          pkk[u >> 1] = pack_bf16x2(ok ? __uint_as_float(ka[e + u]) * p.scale : NAN,
+                                    ok ? __uint_as_float(ka[e + u + 1]) * p.scale : NAN);
+        }
+        if (store) {
+          *reinterpret_cast<uint4*>(dvrow + 32 * c + e) = make_uint4(pv[0], pv[1], pv[2], pv[3]);
+          *reinterpret_cast<uint4*>(dkrow + 32 * c + e) = make_uint4(pkk[0], pkk[1], pkk[2], pkk[3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dQ: one CTA per (query tile, query head, batch)
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const BwdParams p) {
+  using C = BwdCfg<D>;
+  // same plan as the dK/dV kernel with the roles swapped: Q and dO resident
+  // (kKOff / kVOff), two stages of (K, V)
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw_u32);
+  // with a causal or window mask the last query tiles see the most keys: launch them first
+  const int i = (p.mask_kind == ATTN_MASK_FULL) ? blockIdx.x : p.ntiles - 1 - blockIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int klo, khi;
+  k_tiles_of_q_tile(p, i, klo, khi);
+  const int iters = khi - klo + 1;
+  const int kvh = h / p.group;
+
+  const uint32_t bars = sbase + C::kBarOff;
+  auto bar = [&](int x) -> uint32_t { return bars + 8u * static_cast<uint32_t>(x); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + kBwdTmemSlot);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + kBwdAbort);
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBbKV), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBbFull + s), 1);
+      mbar_init(bar(kBbEmpty + s), 1);
+    }
+    mbar_init(bar(kBbS), 1);
+    mbar_init(bar(kBbP), 4);
+    mbar_init(bar(kBbAcc), 1);
+    mbar_init(bar(kBbDrain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const long long budget = p.budget;
+
+  if (warp == kBwdTmaWarp) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- TMA producer
+      const int zq = b * p.Hq + h, zkv = b * p.Hkv + kvh;
+      mbar_arrive_expect_tx(bar(kBbKV), 2 * C::kTile);
+      for (int hh = 0; hh < C::kHalves; ++hh) {
+        tma_load_3d(sbase + C::kKOff + hh * kBox, &tm_q, bar(kBbKV), hh * 64, i * kT, zq);
+        tma_load_3d(sbase + C::kVOff + hh * kBox, &tm_do, bar(kBbKV), hh * 64, i * kT, zq);
+      }
+      int issued[2] = {0, 0};
+      bool ok = true;
+      for (int t = 0; t < iters && ok; ++t) {
+        const int s = t & 1;
+        if (t >= 2 && !mbar_wait_bounded(bar(kBbEmpty + s), ((t - 2) >> 1) & 1, budget, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int jt = klo + t;
+        const uint32_t st = sbase + C::kQOff + s * C::kStageBytes;
+        mbar_arrive_expect_tx(bar(kBbFull + s), 2 * C::kTile);
+        for (int hh = 0; hh < C::kHalves; ++hh) {
+          tma_load_3d(st + hh * kBox, &tm_k, bar(kBbFull + s), hh * 64, jt * kT, zkv);
+          tma_load_3d(st + C::kTile + hh * kBox, &tm_v, bar(kBbFull + s), hh * 64, jt * kT, zkv);
+        }
+        issued[s] = t / 2 + 1;
+      }
+      if (!ok) bwd_abort(abort_flag, p.status);
+      volatile int never = 0;
+      mbar_wait_bounded(bar(kBbKV), 0, kDrainBudgetCycles, &never);
+      for (int s = 0; s < 2; ++s)
+        if (issued[s] > 0) mbar_wait_bounded(bar(kBbFull + s), (issued[s] - 1) & 1, kDrainBudgetCycles, &never);
+    }
+  } else if (warp == kBwdMmaWarp) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      const uint64_t dq = desc_sw128(sbase + C::kKOff, 16, 1024);
+      const uint64_t ddo = desc_sw128(sbase + C::kVOff, 16, 1024);
+      constexpr uint32_t kIdS = idesc_bwd(kT, kT, 0, 0);   // S = Q K^T, dP = dO V^T
+      constexpr uint32_t kIdAcc = idesc_bwd(kT, D, 0, 1);  // dQ += dS K (K as an MN-major B)
+      bool ok = mbar_wait_bounded(bar(kBbKV), 0, budget, abort_flag);
+      for (int t = 0; t < iters && ok; ++t) {
+        const int s = t & 1;
+        const uint32_t st = sbase + C::kQOff + s * C::kStageBytes;
+        if (!mbar_wait_bounded(bar(kBbFull + s), (t >> 1) & 1, budget, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        mma_kmajor<D>(tmem + C::kColS, dq, desc_sw128(st, 16, 1024), kIdS);
+        mma_kmajor<D>(tmem + C::kColDP, ddo, desc_sw128(st + C::kTile, 16, 1024), kIdS);
+        tc_commit(bar(kBbS));
+        if (!mbar_wait_bounded(bar(kBbP), t & 1, budget, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        mma_tmem_a(tmem + C::kColAcc0, tmem + C::kColS, desc_sw128(st, kBox, 1024), kIdAcc, t == 0);
+        tc_commit(bar(kBbEmpty + s));
+      }
+      if (!ok) bwd_abort(abort_flag, p.status);
+      tc_commit(bar(kBbAcc));
+      tc_commit(bar(kBbDrain));
+      volatile int never = 0;
+      mbar_wait_bounded(bar(kBbDrain), 0, kDrainBudgetCycles, &never);
+    }
+  } else {
+    // ------------------------------------------------------------ dS warps 0-3
+    const int r = threadIdx.x;  // query row of the tile = TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int qpos = i * kT + r;
+    const size_t row = (static_cast<size_t>(b) * p.Hq + h) * p.N + qpos;
+    const float l2 = qpos < p.N ? p.lse[row] * kLog2e : INFINITY;
+    const float dr = qpos < p.N ? p.dvec[row] : 0.f;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int t = 0; t < iters; ++t) {
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbS), t & 1, budget, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const int jt = klo + t;
+      const bool full_tile = (p.mask_kind == ATTN_MASK_FULL || (i > jt && (p.mask_kind == ATTN_MASK_CAUSAL ||
+                                                                           (i * kT + kT - 1) - jt * kT < p.window))) &&
+                             (i * kT + kT <= p.N) && (jt * kT + kT <= p.N);
+#pragma unroll 1
+      for (int c = 0; c < kT / 32; ++c) {
+        uint32_t sv[32], dpv[32];
+        tmem_ld_32x32b_x32(lane_base + C::kColS + 32u * c, sv);
+        tmem_ld_32x32b_x32(lane_base + C::kColDP + 32u * c, dpv);
+        tc_wait_ld();
+        uint32_t dsk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int kpos = jt * kT + 32 * c + e + u;
+            const bool vis = full_tile || (qpos < p.N && kpos < p.N && bwd_visible(p, qpos, kpos));
+            const float pr = vis ? fast_exp2(__uint_as_float(sv[e + u]) * sl2 - l2) : 0.f;
+            ds[u] = pr * (__uint_as_float(dpv[e + u]) - dr);
+          }
+          dsk[e >> 1] = pack_bf16x2(ds[0], ds[1]);
+        }
+        tmem_st_32x32b_x16(lane_base + C::kColS + 16u * c, dsk);  // dS as bf16 pairs over read columns
+      }
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBbP));
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbAcc), 0, budget, abort_flag));
+    if (!ok) bwd_abort(abort_flag, p.status);
+    tc_fence_after();
+    // TMEM loads are warp-collective: every lane runs them, only rows < N are stored
+    const bool store = qpos < p.N;
+    __nv_bfloat16* dqrow = p.dq + (store ? row : 0) * D;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t qa[32];
+      tmem_ld_32x32b_x32(lane_base + C::kColAcc0 + 32u * c, qa);
+      tc_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; e += 8) {
+        uint32_t pq[4];
+#pragma unroll
+        for (int u = 0; u < 8; u += 2)
+          pq[u >> 1] = pack_bf16x2(ok ? __uint_as_float(qa[e + u]) * p.scale : NAN,
+                                   ok ? __uint_as_float(qa[e + u + 1]) * p.scale : NAN);
+        if (store) *reinterpret_cast<uint4*>(dqrow + 32 * c + e) = make_uint4(pq[0], pq[1], pq[2], pq[3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// [heads][n][d] bf16 as a rank-3 tensor (d innermost), 64-column x 128-row boxes, 128-byte swizzle.
+bool encode_bwd(CUtensorMap* map, const void* base, int d, int n, int heads) {
+  const auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encode_fn());
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
+                              static_cast<cuuint64_t>(heads)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(n) * d * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kT), 1};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estride,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+int launch_backward_t(const void* q, const void* k, const void* v, const void* o, const void* d_o, const float* lse,
+                      void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int mask_kind, int window,
+                      float scale, void* workspace, int32_t* status, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_bwd(&tq, q, D, N, B * Hq) || !encode_bwd(&tk, k, D, N, B * Hkv) || !encode_bwd(&tv, v, D, N, B * Hkv) ||
+      !encode_bwd(&tdo, d_o, D, N, B * Hq))
+    return ATTN_ERR_CUDA;
+  BwdParams p;
+  p.o = static_cast<const __nv_bfloat16*>(o);
+  p.d_o = static_cast<const __nv_bfloat16*>(d_o);
+  p.lse = lse;
+  p.dvec = static_cast<float*>(workspace);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.status = status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.mask_kind = mask_kind;
+  p.window = window;
+  p.ntiles = (N + kT - 1) / kT;
+  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
+  p.budget = wait_budget_cycles();
+  const size_t rows = static_cast<size_t>(B) * Hq * N;
+  bwd_rowdot_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  constexpr int smem = BwdCfg<D>::kAlloc;
+  if (cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  bwd_dkdv_kernel<D><<<dim3(p.ntiles, Hkv, B), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  bwd_dq_kernel<D><<<dim3(p.ntiles, Hq, B), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(int B, int Hq, int N) { return static_cast<size_t>(B) * Hq * N * sizeof(float); }
+
+int launch_backward(const void* q, const void* k, const void* v, const void* o, const void* d_o, const float* lse,
+                    void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int mask_kind, int window,
+                    float scale, void* workspace, int32_t* status, cudaStream_t stream) {
+  if (d == 128)
+    return launch_backward_t<128>(q, k, v, o, d_o, lse, dq, dk, dv, B, Hq, Hkv, N, mask_kind, window, scale,
+                                  workspace, status, stream);
+  return launch_backward_t<64>(q, k, v, o, d_o, lse, dq, dk, dv, B, Hq, Hkv, N, mask_kind, window, scale, workspace,
+                               status, stream);
+}
+
+}  // namespace attn

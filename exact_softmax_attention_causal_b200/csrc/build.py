@@ -20,7 +20,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 PKG = os.path.dirname(HERE)
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libattn_b200.so")
-SOURCES = ["attn_api.cu", "prefill_sm100.cu", "decode_sm100.cu", "decode_noalloc.cu", "mla_sm100.cu"]
+SOURCES = ["attn_api.cu", "prefill_sm100.cu", "decode_sm100.cu", "decode_noalloc.cu", "mla_sm100.cu", "backward_sm100.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -69,6 +69,12 @@ cudaError_t launch_decode_merge(const float* o_part, const float* lse_part, cons
                                 const float* sinks, void* o, float* lse, int B, int Hq, int d, int splits, int chunk,
                                 int max_seq_len, int window, int n_sink, int32_t* status, cudaStream_t stream);
 
+// Backward pass (backward_sm100.cu): workspace = D = rowsum(dO * O), fp32 [B, Hq, N].
+size_t backward_workspace_bytes(int B, int Hq, int N);
+int launch_backward(const void* q, const void* k, const void* v, const void* o, const void* d_o, const float* lse,
+                    void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int mask_kind, int window,
+                    float scale, void* workspace, int32_t* status, cudaStream_t stream);
+
 int launch_prefill_paged(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
                          const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int d,
                          int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, int mask_kind,

@@ -21,6 +21,9 @@
  *                        sections 9, 10 and 12).
  *   attn_prefill_paged - the newest Nq positions of each sequence against its
  *                        paged context (prefix / chunked prefill).
+ *   attn_prefill_backward - dQ, dK, dV of attn_prefill for an output gradient
+ *                        dO, recomputing S and P tile by tile from the saved
+ *                        LSE ("Inference attention" post, "FlashAttention").
  *   attn_mla_decode_paged - absorbed Multi-head Latent Attention decode over a
  *                        paged latent cache ("Modern Attention Mechanisms",
  *                        section 7; "Module 09", the MLA section).
@@ -247,6 +250,41 @@ ATTN_API int attn_decode_paged_window(const void* q, const void* k_cache, const 
                                       int max_blocks_per_seq, int max_seq_len, int window, int n_sink, float scale,
                                       void* workspace, size_t workspace_bytes, int32_t* status,
                                       attn_stream_t stream);
+
+/*
+ * attn_prefill_backward_workspace_bytes - bytes of device workspace
+ * attn_prefill_backward needs: D = rowsum(dO * O), fp32 [B, Hq, N]. Returns 0
+ * for invalid sizes.
+ */
+ATTN_API size_t attn_prefill_backward_workspace_bytes(int B, int Hq, int N);
+
+/*
+ * attn_prefill_backward - gradients of attn_prefill.
+ *
+ * The pages say the backward pass recomputes S and P tile by tile instead of
+ * storing them ("Inference attention" post, section "FlashAttention"); the
+ * gradients are the chain rule of the forward definition ("Module 5. Modern
+ * Attention Mechanisms", section 4; head map of section 6):
+ *   P = exp(scale Q K^T - LSE) on visible pairs (0 elsewhere),
+ *   dV = P^T dO, dP = dO V^T, dS = P * (dP - D), D = rowsum(dO * O),
+ *   dQ = scale dS K, dK = scale dS^T Q,
+ * with dK and dV of a K/V head summed over the Hq / Hkv query heads that read it.
+ *
+ *   q, o, d_o    [B, Hq, N, d] bf16                          read (o, lse: attn_prefill's outputs)
+ *   k, v         [B, Hkv, N, d] bf16                         read
+ *   lse          [B, Hq, N] fp32, natural log                read
+ *   dq           [B, Hq, N, d] bf16                          written
+ *   dk, dv       [B, Hkv, N, d] bf16                         written
+ *   mask_kind, window, scale   as passed to attn_prefill
+ *   workspace    at least attn_prefill_backward_workspace_bytes(B, Hq, N)
+ *                bytes, 16-byte aligned
+ *   status       device int32 or NULL (bounded-wait expiry: NaN outputs and
+ *                ATTN_STATUS_BIT_TIMEOUT)
+ */
+ATTN_API int attn_prefill_backward(const void* q, const void* k, const void* v, const void* o, const void* d_o,
+                                   const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
+                                   int d, int mask_kind, int window, float scale, void* workspace,
+                                   size_t workspace_bytes, int32_t* status, attn_stream_t stream);
 
 /*
  * attn_mla_decode_workspace_bytes - bytes of device workspace

@@ -36,3 +36,28 @@ def assert_parity(o_gpu, o_ref, lse_gpu=None, lse_ref=None, what=""):
         assert lmax <= LSE_MAX_ABS, f"{what}: LSE max |err| {lmax:.3e} > {LSE_MAX_ABS}"
         out["lse_max_abs"] = lmax
     return out
+
+
+# Gradients (bf16 outputs of fp32 accumulations over bf16-rounded P and dS):
+# relative RMS <= 1e-2 and max |err| <= 2e-2 of the reference's largest
+# magnitude. P, dS and the outputs are each rounded to bf16 once (relative
+# 2^-9 = 0.2 % per element), which puts the RMS error near 0.5 %. Both scales
+# have a floor of 0.05: with unit-normal inputs the gradient entries are of
+# order 0.1 to 10, and where the exact gradient vanishes (a window of 1: P = 1,
+# D = dP, so dS = 0 and dQ = 0) what remains is rounding noise of order 1e-6.
+GRAD_REL_RMS = 1e-2
+GRAD_MAX_REL = 2e-2
+GRAD_FLOOR = 0.05
+
+
+def assert_grad_parity(g_gpu, g_ref, what=""):
+    g_gpu, g_ref = to64(g_gpu), to64(g_ref)
+    assert g_gpu.shape == g_ref.shape, (what, g_gpu.shape, g_ref.shape)
+    assert np.isfinite(g_gpu).all(), f"{what}: non-finite gradient"
+    scale = max(float(np.abs(g_ref).max()), GRAD_FLOOR)
+    rms_ref = max(float(np.sqrt(np.mean(g_ref ** 2))), GRAD_FLOOR)
+    max_abs = float(np.abs(g_gpu - g_ref).max())
+    rms_err = float(np.sqrt(np.mean((g_gpu - g_ref) ** 2)))
+    assert max_abs <= GRAD_MAX_REL * scale, f"{what}: max |err| {max_abs:.3e} > {GRAD_MAX_REL} x {scale:.3e}"
+    assert rms_err <= GRAD_REL_RMS * rms_ref, f"{what}: RMS err {rms_err:.3e} > {GRAD_REL_RMS} x {rms_ref:.3e}"
+    return {"max_abs": max_abs, "rel_rms": rms_err / rms_ref}

@@ -153,6 +153,34 @@ def test_mla_workspace_rejects_unsupported_widths():
     assert _lib.lib().attn_mla_decode_workspace_bytes(2, 128, 256, 64, 1024) == 0
 
 
+def _bwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, do=FAKE, lse=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, B=1, Hq=4, Hkv=2, N=256,
+             d=128, mask=1, window=0, scale=0.1, ws=FAKE, wsb=1 << 20)
+    a.update(kw)
+    return _lib.lib().attn_prefill_backward(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"],
+                                            a["dv"], a["B"], a["Hq"], a["Hkv"], a["N"], a["d"], a["mask"],
+                                            a["window"], a["scale"], a["ws"], a["wsb"], NULL, NULL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(do=NULL), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(lse=NULL), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(mask=2, window=0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(dk=ctypes.c_void_p(0x10008)), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(d=96), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(ws=NULL), _lib.ATTN_ERR_WORKSPACE),
+    (dict(wsb=100), _lib.ATTN_ERR_WORKSPACE),
+])
+def test_backward_rejects_bad_arguments(kw, code):
+    assert _bwd(**kw) == code
+
+
+def test_backward_workspace_is_one_float_per_row():
+    assert _lib.lib().attn_prefill_backward_workspace_bytes(2, 8, 300) == 2 * 8 * 300 * 4
+    assert _lib.lib().attn_prefill_backward_workspace_bytes(0, 8, 300) == 0
+
+
 def _prefill_paged(**kw):
     a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, sl=FAKE, o=FAKE, lse=NULL, B=2, Hq=8, Hkv=2, Nq=64, d=128, nb=10,
              bs=16, mb=8, msl=128, mask=1, window=0, scale=0.1)
