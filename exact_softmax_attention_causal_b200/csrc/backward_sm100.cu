@@ -27,9 +27,10 @@
 // 128x128xd products per tile pair instead of five), in exchange for
 // deterministic sums without a dQ accumulator shared between CTAs.
 //
-// Roles in both tile kernels (192 threads): warps 0-3 compute P and dS (thread
-// i owns TMEM lane i = one key row (dK/dV) or query row (dQ)), warp 4 is the
-// TMA producer, warp 5 issues the MMAs and owns TMEM. Every pipeline wait is
+// Roles in both tile kernels (320 threads): warps 0-7 compute P and dS (warp w
+// reads TMEM lanes 32 (w % 4) .. + 31, one key row (dK/dV) or query row (dQ)
+// per lane, over the column half 64 (w / 4) .. + 63), warp 8 is the TMA
+// producer, warp 9 issues the MMAs and owns TMEM. Every pipeline wait is
 // bounded; on expiry the CTA records ATTN_STATUS_BIT_TIMEOUT, writes NaN, drains
 // and exits.
 
@@ -48,21 +49,24 @@ namespace attn {
 namespace {
 
 constexpr int kT = 128;             // rows per tile (TMEM lanes), keys per tile
-constexpr int kBwdThreads = 192;
-constexpr int kBwdTmaWarp = 4;
-constexpr int kBwdMmaWarp = 5;
+constexpr int kBwdThreads = 320;
+constexpr int kBwdTmaWarp = 8;
+constexpr int kBwdMmaWarp = 9;
+constexpr int kBwdSoftWarps = 8;  // TMEM sub-partition (w % 4) x column half (w / 4)
 constexpr int kBox = 128 * 128;     // bytes of one 64-column, 128-row swizzled box
 
 struct BwdParams {
   const __nv_bfloat16* o;
   const __nv_bfloat16* d_o;
   const float* lse;   // [B, Hq, N] natural log (forward output)
-  float* dvec;        // [B, Hq, N] D = rowsum(dO * O)
+  // workspace, rows padded to whole tiles (npad = 128 * ntiles), 16-byte aligned:
+  float* lse2;        // [B, Hq, npad] LSE * log2(e), +inf past N
+  float* dvec;        // [B, Hq, npad] D = rowsum(dO * O), 0 past N
   __nv_bfloat16* dq;  // [B, Hq, N, d]
   __nv_bfloat16* dk;  // [B, Hkv, N, d]
   __nv_bfloat16* dv;  // [B, Hkv, N, d]
   int32_t* status;
-  int B, Hq, Hkv, N, group, mask_kind, window, ntiles;
+  int B, Hq, Hkv, N, group, mask_kind, window, ntiles, npad;
   float scale, scale_log2;
   long long budget;
 };
@@ -110,24 +114,36 @@ __device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint64_t da, uint64_
     tc_mma_ss(d_tmem, da + off, db + off, idesc, kk > 0 ? 1u : 0u);
   }
 }
-// 128 / 16 steps of D (+)= A[tmem: bf16 pairs, 8 columns per step] * B[smem, MN-major, 16 rows per step].
+// 128 / 16 steps of D (+)= A[tmem] * B[smem, MN-major, 16 rows per step]. A holds bf16 pairs
+// written by two warps per TMEM sub-partition, each over the first half of its own 64 columns:
+// K rows 16 kk .. 16 kk + 15 sit at column 64 (kk / 4) + 8 (kk % 4).
 __device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t db, uint32_t idesc,
                                            bool first) {
 #pragma unroll
   for (int kk = 0; kk < kT / 16; ++kk)
-    tc_mma_ts(d_tmem, a_tmem + 8u * kk, db + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
+    tc_mma_ts(d_tmem, a_tmem + 64u * (kk >> 2) + 8u * (kk & 3), db + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
               (!first || kk > 0) ? 1u : 0u);
 }
 
 // ---------------------------------------------------------------------------
-// D = rowsum(dO * O): one warp per (batch, head, row)
+// D = rowsum(dO * O) and LSE * log2(e), one warp per (batch, head, padded row)
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void bwd_rowdot_kernel(const BwdParams p) {
-  const size_t rows = static_cast<size_t>(p.B) * p.Hq * p.N;
-  const size_t row = blockIdx.x * static_cast<size_t>(blockDim.x / 32) + (threadIdx.x >> 5);
+  const size_t rows = static_cast<size_t>(p.B) * p.Hq * p.npad;
+  const size_t prow = blockIdx.x * static_cast<size_t>(blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
+  if (prow >= rows) return;
+  const size_t bh = prow / p.npad;
+  const int q = static_cast<int>(prow - bh * p.npad);
+  if (q >= p.N) {  // padding rows: no probability mass (exp2(x - inf) = 0) and D = 0
+    if (lane == 0) {
+      p.dvec[prow] = 0.f;
+      p.lse2[prow] = INFINITY;
+    }
+    return;
+  }
+  const size_t row = bh * p.N + q;
   constexpr int PER = D / 32;
   const __nv_bfloat16* a = p.o + row * D + lane * PER;
   const __nv_bfloat16* g = p.d_o + row * D + lane * PER;
@@ -140,7 +156,10 @@ __global__ void bwd_rowdot_kernel(const BwdParams p) {
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (lane == 0) p.dvec[row] = s;
+  if (lane == 0) {
+    p.dvec[prow] = s;
+    p.lse2[prow] = p.lse[row] * kLog2e;
+  }
 }
 
 // Shared-memory plan of the tile kernels (1024-byte aligned):
@@ -153,7 +172,7 @@ struct BwdCfg {
   static constexpr int kVOff = kKOff + kTile;
   static constexpr int kQOff = kVOff + kTile;          // + stage * 2 * kTile
   static constexpr int kStageBytes = 2 * kTile;        // Q then dO
-  static constexpr int kRowOff = kQOff + 2 * kStageBytes;  // [stage][LSE 128 | D 128] fp32
+  static constexpr int kRowOff = kQOff + 2 * kStageBytes;  // [stage][LSE*log2e 128 | D 128] fp32 (dK/dV)
   static constexpr int kBarOff = kRowOff + 2 * 2 * kT * 4;
   static constexpr int kBytes = kBarOff + 256;
   static constexpr int kAlloc = kBytes + 1024;
@@ -204,7 +223,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(kBbEmpty + s), 1);
     }
     mbar_init(bar(kBbS), 1);
-    mbar_init(bar(kBbP), 4);
+    mbar_init(bar(kBbP), kBwdSoftWarps);
     mbar_init(bar(kBbAcc), 1);
     mbar_init(bar(kBbDrain), 1);
     *abort_flag = 0;
@@ -240,12 +259,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int h = kvh * p.group + t / nq, i = qlo + t % nq;
         const int zq = b * p.Hq + h;
         const uint32_t st = sbase + C::kQOff + s * C::kStageBytes;
-        // the LSE and D rows of the tile travel by plain loads (softmax warps); only Q and dO by TMA
-        mbar_arrive_expect_tx(bar(kBbFull + s), 2 * C::kTile);
+        const uint32_t rows = sbase + C::kRowOff + s * (2 * kT * 4);
+        const size_t prow = static_cast<size_t>(zq) * p.npad + static_cast<size_t>(i) * kT;
+        mbar_arrive_expect_tx(bar(kBbFull + s), 2 * C::kTile + 2 * kT * 4);
         for (int hh = 0; hh < C::kHalves; ++hh) {
           tma_load_3d(st + hh * kBox, &tm_q, bar(kBbFull + s), hh * 64, i * kT, zq);
           tma_load_3d(st + C::kTile + hh * kBox, &tm_do, bar(kBbFull + s), hh * 64, i * kT, zq);
         }
+        bulk_load(rows, p.lse2 + prow, kT * 4, bar(kBbFull + s));
+        bulk_load(rows + kT * 4, p.dvec + prow, kT * 4, bar(kBbFull + s));
         issued[s] = t / 2 + 1;
       }
       if (!ok) bwd_abort(abort_flag, p.status);
@@ -291,34 +313,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_wait_bounded(bar(kBbDrain), 0, kDrainBudgetCycles, &never);
     }
   } else {
-    // ------------------------------------------------------------ P / dS warps 0-3
-    const int r = threadIdx.x;  // key row of the tile = TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    // ------------------------------------------------------------ P / dS warps 0-7
+    const int r = (warp & 3) * 32 + lane;  // key row of the tile = TMEM lane
+    const int ch = warp >> 2;              // query columns 64 ch .. 64 ch + 63
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int kpos = j * kT + r;
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int t = 0; t < iters; ++t) {
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbS), t & 1, budget, abort_flag));
+      // the staged rows: observe their own barrier too (already complete once the S MMAs ran)
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbFull + (t & 1)), (t >> 1) & 1, budget, abort_flag));
       if (!ok) break;  // no named barriers here: leaving early strands no other warp
       tc_fence_after();
-      const int h = kvh * p.group + t / nq, i = qlo + t % nq;
-      const size_t rowbase = (static_cast<size_t>(b) * p.Hq + h) * p.N + static_cast<size_t>(i) * kT;
+      const int i = qlo + t % nq;
+      // LSE * log2(e) and D of the pair's 128 query rows, staged in shared memory with Q and dO
+      // (the MMA warp consumed stage t & 1 only after the S MMAs, which precede this wait)
+      const float* srow = reinterpret_cast<const float*>(smem + C::kRowOff + (t & 1) * (2 * kT * 4));
       const bool full_tile = (p.mask_kind == ATTN_MASK_FULL || (i > j && (p.mask_kind == ATTN_MASK_CAUSAL ||
                                                                           (i * kT + kT - 1) - j * kT < p.window))) &&
                              (i * kT + kT <= p.N) && (j * kT + kT <= p.N);
 #pragma unroll 1
-      for (int c = 0; c < kT / 32; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * ch + cc;  // 32-column chunk of the tile
         uint32_t sv[32], dpv[32];
         tmem_ld_32x32b_x32(lane_base + C::kColS + 32u * c, sv);
         tmem_ld_32x32b_x32(lane_base + C::kColDP + 32u * c, dpv);
-        // LSE (base 2) and D of the 32 query columns: the same addresses for every
-        // thread of the warp (one broadcast load each); rows past N see nothing
+        // the 32 query columns' LSE (base 2) and D: broadcast shared-memory reads;
+        // rows past N carry +inf and 0
         float l2[32], dd[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const bool in = (i * kT + 32 * c + e) < p.N;
-          l2[e] = in ? __ldg(p.lse + rowbase + 32 * c + e) * kLog2e : INFINITY;
-          dd[e] = in ? __ldg(p.dvec + rowbase + 32 * c + e) : 0.f;
+        for (int e = 0; e < 32; e += 4) {
+          const float4 lv = *reinterpret_cast<const float4*>(srow + 32 * c + e);
+          const float4 dv4 = *reinterpret_cast<const float4*>(srow + kT + 32 * c + e);
+          l2[e] = lv.x;
+          l2[e + 1] = lv.y;
+          l2[e + 2] = lv.z;
+          l2[e + 3] = lv.w;
+          dd[e] = dv4.x;
+          dd[e + 1] = dv4.y;
+          dd[e + 2] = dv4.z;
+          dd[e + 3] = dv4.w;
         }
         tc_wait_ld();
         uint32_t pk[16], dsk[16];
@@ -335,9 +370,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pk[e >> 1] = pack_bf16x2(pr[0], pr[1]);
           dsk[e >> 1] = pack_bf16x2(ds[0], ds[1]);
         }
-        // bf16 pairs over the columns already read: P^T at kColS + 16 c, dS^T at kColDP + 16 c
-        tmem_st_32x32b_x16(lane_base + C::kColS + 16u * c, pk);
-        tmem_st_32x32b_x16(lane_base + C::kColDP + 16u * c, dsk);
+        // bf16 pairs over this warp's columns already read: 64 ch + 16 cc
+        tmem_st_32x32b_x16(lane_base + C::kColS + 64u * ch + 16u * cc, pk);
+        tmem_st_32x32b_x16(lane_base + C::kColDP + 64u * ch + 16u * cc, dsk);
       }
       tc_wait_st();
       tc_fence_before();
@@ -353,7 +388,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __nv_bfloat16* dvrow = p.dv + ((static_cast<size_t>(b) * p.Hkv + kvh) * p.N + (store ? kpos : 0)) * D;
     __nv_bfloat16* dkrow = p.dk + ((static_cast<size_t>(b) * p.Hkv + kvh) * p.N + (store ? kpos : 0)) * D;
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = ch * (D / 64); c < (ch + 1) * (D / 64); ++c) {  // this warp's half of the head dim
       uint32_t va[32], ka[32];
       tmem_ld_32x32b_x32(lane_base + C::kColAcc0 + 32u * c, va);
       tmem_ld_32x32b_x32(lane_base + C::kColAcc1 + 32u * c, ka);
@@ -417,7 +452,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(kBbEmpty + s), 1);
     }
     mbar_init(bar(kBbS), 1);
-    mbar_init(bar(kBbP), 4);
+    mbar_init(bar(kBbP), kBwdSoftWarps);
     mbar_init(bar(kBbAcc), 1);
     mbar_init(bar(kBbDrain), 1);
     *abort_flag = 0;
@@ -499,13 +534,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_wait_bounded(bar(kBbDrain), 0, kDrainBudgetCycles, &never);
     }
   } else {
-    // ------------------------------------------------------------ dS warps 0-3
-    const int r = threadIdx.x;  // query row of the tile = TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    // ------------------------------------------------------------ dS warps 0-7
+    const int r = (warp & 3) * 32 + lane;  // query row of the tile = TMEM lane
+    const int ch = warp >> 2;              // key columns 64 ch .. 64 ch + 63
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int qpos = i * kT + r;
     const size_t row = (static_cast<size_t>(b) * p.Hq + h) * p.N + qpos;
-    const float l2 = qpos < p.N ? p.lse[row] * kLog2e : INFINITY;
-    const float dr = qpos < p.N ? p.dvec[row] : 0.f;
+    const size_t prow = (static_cast<size_t>(b) * p.Hq + h) * p.npad + qpos;
+    const float l2 = p.lse2[prow];
+    const float dr = p.dvec[prow];
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int t = 0; t < iters; ++t) {
@@ -517,7 +554,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                                                            (i * kT + kT - 1) - jt * kT < p.window))) &&
                              (i * kT + kT <= p.N) && (jt * kT + kT <= p.N);
 #pragma unroll 1
-      for (int c = 0; c < kT / 32; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * ch + cc;  // 32-column chunk of the tile
         uint32_t sv[32], dpv[32];
         tmem_ld_32x32b_x32(lane_base + C::kColS + 32u * c, sv);
         tmem_ld_32x32b_x32(lane_base + C::kColDP + 32u * c, dpv);
@@ -535,7 +573,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           dsk[e >> 1] = pack_bf16x2(ds[0], ds[1]);
         }
-        tmem_st_32x32b_x16(lane_base + C::kColS + 16u * c, dsk);  // dS as bf16 pairs over read columns
+        tmem_st_32x32b_x16(lane_base + C::kColS + 64u * ch + 16u * cc, dsk);  // dS as bf16 pairs, own half
       }
       tc_wait_st();
       tc_fence_before();
@@ -550,7 +588,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool store = qpos < p.N;
     __nv_bfloat16* dqrow = p.dq + (store ? row : 0) * D;
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = ch * (D / 64); c < (ch + 1) * (D / 64); ++c) {  // this warp's half of the head dim
       uint32_t qa[32];
       tmem_ld_32x32b_x32(lane_base + C::kColAcc0 + 32u * c, qa);
       tc_wait_ld();
@@ -599,7 +637,10 @@ int launch_backward_t(const void* q, const void* k, const void* v, const void* o
   p.o = static_cast<const __nv_bfloat16*>(o);
   p.d_o = static_cast<const __nv_bfloat16*>(d_o);
   p.lse = lse;
+  p.ntiles = (N + kT - 1) / kT;
+  p.npad = p.ntiles * kT;
   p.dvec = static_cast<float*>(workspace);
+  p.lse2 = p.dvec + static_cast<size_t>(B) * Hq * p.npad;
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
@@ -611,11 +652,10 @@ int launch_backward_t(const void* q, const void* k, const void* v, const void* o
   p.group = Hq / Hkv;
   p.mask_kind = mask_kind;
   p.window = window;
-  p.ntiles = (N + kT - 1) / kT;
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
   p.budget = wait_budget_cycles();
-  const size_t rows = static_cast<size_t>(B) * Hq * N;
+  const size_t rows = static_cast<size_t>(B) * Hq * p.npad;
   bwd_rowdot_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   constexpr int smem = BwdCfg<D>::kAlloc;
@@ -630,7 +670,10 @@ int launch_backward_t(const void* q, const void* k, const void* v, const void* o
 
 }  // namespace
 
-size_t backward_workspace_bytes(int B, int Hq, int N) { return static_cast<size_t>(B) * Hq * N * sizeof(float); }
+size_t backward_workspace_bytes(int B, int Hq, int N) {
+  const size_t npad = static_cast<size_t>((N + kT - 1) / kT) * kT;
+  return 2 * static_cast<size_t>(B) * Hq * npad * sizeof(float);  // D, then LSE * log2(e)
+}
 
 int launch_backward(const void* q, const void* k, const void* v, const void* o, const void* d_o, const float* lse,
                     void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int mask_kind, int window,

@@ -253,8 +253,9 @@ ATTN_API int attn_decode_paged_window(const void* q, const void* k_cache, const 
 
 /*
  * attn_prefill_backward_workspace_bytes - bytes of device workspace
- * attn_prefill_backward needs: D = rowsum(dO * O), fp32 [B, Hq, N]. Returns 0
- * for invalid sizes.
+ * attn_prefill_backward needs: D = rowsum(dO * O) and LSE * log2(e), each fp32
+ * [B, Hq, Npad] with Npad = N rounded up to a multiple of 128. Returns 0 for
+ * invalid sizes.
  */
 ATTN_API size_t attn_prefill_backward_workspace_bytes(int B, int Hq, int N);
 

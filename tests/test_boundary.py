@@ -176,8 +176,8 @@ def test_backward_rejects_bad_arguments(kw, code):
     assert _bwd(**kw) == code
 
 
-def test_backward_workspace_is_one_float_per_row():
-    assert _lib.lib().attn_prefill_backward_workspace_bytes(2, 8, 300) == 2 * 8 * 300 * 4
+def test_backward_workspace_is_two_floats_per_padded_row():
+    assert _lib.lib().attn_prefill_backward_workspace_bytes(2, 8, 300) == 2 * (2 * 8 * 384 * 4)
     assert _lib.lib().attn_prefill_backward_workspace_bytes(0, 8, 300) == 0
 
 
