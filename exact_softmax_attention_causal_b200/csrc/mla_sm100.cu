@@ -33,7 +33,8 @@
 //              max exceeds it by more than 8 (base 2).
 //   warp 8     TMA producer: Q^T once (nine 8 KB chunks), then for every tile
 //              the nine 16 KB chunks of 128 cached rows, one box per pool
-//              block (block-table entries fetched a tile ahead). Rows past the
+//              block, lane e issuing block e's boxes (block-table entries
+//              fetched a tile ahead, one per lane). Rows past the
 //              sequence come in as zeros (one-row boxes for the partly filled
 //              last block, out-of-range block index for whole blocks).
 //   warp 9     MMA issuer; allocates and frees TMEM.
@@ -197,75 +198,80 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   const long long budget = p.budget;
 
   if (warp == kMlaTmaWarp) {
+    // ------------------------------------------------------------ TMA producer
+    // Lane 0 waits on the slots and arms their barriers; lane e then issues the
+    // boxes of the tile's e-th pool block, so the (up to 8) copies of a chunk go
+    // out from different threads at once.
+    const int bs = p.block_size;
+    const int boxes = kTok / bs;  // pool blocks per tile (block_size divides 128)
+    const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
     if (lane == 0) {
-      // ---------------------------------------------------------- TMA producer
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_c);
       prefetch_tmap(&tm_crow);
       mbar_arrive_expect_tx(bar(kMbQFull), kChunks * kQChunkBytes);
       for (int j = 0; j < kChunks; ++j)
         tma_load_3d(sbase + kQOff + j * kQChunkBytes, &tm_q, bar(kMbQFull), 64 * j, hb * kNH, b);
-      const int bs = p.block_size;
-      const int boxes = kTok / bs;  // pool blocks per tile (block_size divides 128)
-      const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
-      // Block-table entries of a tile: out-of-range or unneeded blocks become the
-      // out-of-range index num_blocks (TMA fills zeros); a bad referenced entry
-      // also marks the CTA's output as invalid.
-      auto fetch = [&](int tile, int (&ent)[8]) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          ent[e] = p.num_blocks;
-          const int key = t0 + tile * kTok + e * bs;
-          if (e < boxes && key < t1) ent[e] = __ldg(table + key / bs);
-        }
-      };
-      int ent[8], ent_next[8];
-      fetch(0, ent);
-      int issued[kChunks];  // tiles whose copy of chunk j was issued
-#pragma unroll
-      for (int j = 0; j < kChunks; ++j) issued[j] = 0;
-      bool ok = true;
-      for (int i = 0; i < ntiles && ok; ++i) {
-        if (i + 1 < ntiles) fetch(i + 1, ent_next);
-        const int tok0 = t0 + i * kTok;
-        for (int j = 0; j < kChunks; ++j) {
-          if (i > 0 && !mbar_wait_bounded(bar(kMbKEmpty + j), (i - 1) & 1, budget, abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar(kMbKFull + j), kKChunkBytes);
-          const uint32_t slot = sbase + kKOff + j * kKChunkBytes;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            if (e >= boxes) break;
-            const int key = tok0 + e * bs;
-            int phys = ent[e];
-            if (key < t1 && (phys < 0 || phys >= p.num_blocks)) {
-              *bad_flag = 1;
-              phys = p.num_blocks;
-            }
-            if (key >= t1) phys = p.num_blocks;
-            const uint32_t dst = slot + e * bs * 128;
-            if (key + bs <= t1 || phys == p.num_blocks) {
-              tma_load_3d(dst, &tm_c, bar(kMbKFull + j), 64 * j, 0, phys);
-            } else {
-              const int valid = t1 - key;  // 1 .. bs - 1 rows hold tokens of this split
-              for (int r = 0; r < bs; ++r)
-                tma_load_3d(dst + r * 128, &tm_crow, bar(kMbKFull + j), 64 * j, r, r < valid ? phys : p.num_blocks);
-            }
-          }
-          issued[j] = i + 1;
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ent[e] = ent_next[e];
+    }
+    // This lane's block of a tile: out-of-range or unneeded blocks become the
+    // out-of-range index num_blocks (TMA fills zeros); a bad referenced entry
+    // also marks the CTA's output as invalid.
+    auto fetch = [&](int tile) -> int {
+      const int key = t0 + tile * kTok + lane * bs;
+      return (lane < boxes && key < t1) ? __ldg(table + key / bs) : p.num_blocks;
+    };
+    int ent = fetch(0);
+    int issued = 0;  // lane 0: tiles whose copies were issued for every chunk
+    int last_j = -1;  // lane 0: chunks of the tile being issued when a wait gave up
+    bool ok = true;
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const int ent_next = (i + 1 < ntiles) ? fetch(i + 1) : p.num_blocks;
+      const int tok0 = t0 + i * kTok;
+      const int key = tok0 + lane * bs;
+      int phys = ent;
+      if (lane < boxes && key < t1 && (phys < 0 || phys >= p.num_blocks)) {
+        *bad_flag = 1;
+        phys = p.num_blocks;
       }
+      if (key >= t1) phys = p.num_blocks;
+      for (int j = 0; j < kChunks; ++j) {
+        bool armed = true;
+        if (lane == 0) {
+          armed = (i == 0) || mbar_wait_bounded(bar(kMbKEmpty + j), (i - 1) & 1, budget, abort_flag);
+          if (armed) {
+            mbar_arrive_expect_tx(bar(kMbKFull + j), kKChunkBytes);
+            last_j = j;
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, armed, 0);
+        if (!ok) break;
+        if (lane < boxes) {
+          const uint32_t dst = sbase + kKOff + j * kKChunkBytes + lane * bs * 128;
+          if (key + bs <= t1 || phys == p.num_blocks) {
+            tma_load_3d(dst, &tm_c, bar(kMbKFull + j), 64 * j, 0, phys);
+          } else {
+            const int valid = t1 - key;  // 1 .. bs - 1 rows hold tokens of this split
+            for (int r = 0; r < bs; ++r)
+              tma_load_3d(dst + r * 128, &tm_crow, bar(kMbKFull + j), 64 * j, r, r < valid ? phys : p.num_blocks);
+          }
+        }
+      }
+      if (ok) {
+        issued = i + 1;
+        last_j = -1;
+      }
+      ent = ent_next;
+    }
+    if (lane == 0) {
       if (!ok) mla_abort(abort_flag, p.status);
-      // Drain: Q and the newest copy of every chunk slot landed before the CTA may exit.
+      // Drain: Q and the newest copy of every chunk slot landed before the CTA may exit
+      // (chunks 0 .. last_j of an interrupted tile belong to tile `issued`).
       volatile int never = 0;
       mbar_wait_bounded(bar(kMbQFull), 0, kDrainBudgetCycles, &never);
-#pragma unroll
-      for (int j = 0; j < kChunks; ++j)
-        if (issued[j] > 0) mbar_wait_bounded(bar(kMbKFull + j), (issued[j] - 1) & 1, kDrainBudgetCycles, &never);
+      for (int j = 0; j < kChunks; ++j) {
+        const int n = (j <= last_j) ? issued + 1 : issued;
+        if (n > 0) mbar_wait_bounded(bar(kMbKFull + j), (n - 1) & 1, kDrainBudgetCycles, &never);
+      }
     }
   } else if (warp == kMlaMmaWarp) {
     if (lane == 0) {
