@@ -97,8 +97,13 @@ struct PfCfg {
   static constexpr int kStageOff = kVOff + kVStages * kTile;
   static constexpr int kStageBytes = 8 * 32 * 128;
   static constexpr int kBarOff = kStageOff + kStageBytes;
-  static constexpr int kBytes = kBarOff + 256;
+  // Paged contexts: work classes (query tile pair, sequence) sorted by their
+  // key-tile count, heaviest first (at most kOrderMax classes; else the fixed order).
+  static constexpr int kOrderOff = kBarOff + 256;
+  static constexpr int kOrderMax = 256;
+  static constexpr int kBytes = kOrderOff + kOrderMax * 4;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
+  static_assert(kAlloc <= 232448, "shared memory per CTA");
   // TMEM columns (512 allocated): scores of A and B (128 fp32 columns each;
   // the bf16 probabilities overwrite their first 64 columns), then outputs.
   __host__ __device__ static constexpr uint32_t col_s(int x) { return x ? 128u : 0u; }
@@ -136,6 +141,7 @@ struct PrefillParams {
   int32_t* status;
   int B, Hq, Hkv, N, group, mask_kind, window, num_cta_tiles;  // N = query rows per sequence
   int num_items;  // num_cta_tiles * Hq * B
+  int ordered;    // paged: items follow the per-launch cost order in shared memory
   float scale_log2;
   long long budget;
   // Paged context (prefix prefill): the keys of sequence b are its seq_lens[b]
@@ -153,12 +159,13 @@ struct PrefillParams {
 struct WorkItem {
   int q0, h, b;
 };
-__device__ __forceinline__ WorkItem item_at(const PrefillParams& p, int w) {
-  const int per = p.Hq * p.B;
-  const int rank = w / per;
-  const int rem = w - rank * per;
+// Item w belongs to class w / Hq = rank * B + b (fixed order) or to class
+// order[w / Hq] (paged, costs sorted at launch); head w % Hq.
+__device__ __forceinline__ WorkItem item_at(const PrefillParams& p, int w, const int* order, bool use_order) {
+  const int cls = use_order ? order[w / p.Hq] : w / p.Hq;
+  const int rank = cls / p.B;
   const int ct = (p.mask_kind == ATTN_MASK_FULL) ? rank : (p.num_cta_tiles - 1 - rank);
-  return WorkItem{ct * kRowsPerCta, rem % p.Hq, rem / p.Hq};
+  return WorkItem{ct * kRowsPerCta, w % p.Hq, cls - rank * p.B};
 }
 // Snake assignment of the heaviest-first list over the persistent CTAs:
 // round r hands item r * G + c (r even) or r * G + G - 1 - c (r odd) to CTA c.
@@ -338,6 +345,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
+  // Paged contexts: every CTA sorts the work classes by key-tile count (the
+  // same order everywhere), so the snake deal starts from the heaviest items
+  // of the longest contexts. The key ring, not yet written, holds the costs.
+  int* order = reinterpret_cast<int*>(smem + C::kOrderOff);
+  const bool use_order = PAGED && p.ordered;
+  if (use_order && warp == 0) {
+    const int classes = p.num_cta_tiles * p.B;
+    int* cost = reinterpret_cast<int*>(smem + C::kKOff);
+    for (int c = lane; c < classes; c += 32) {
+      const int rank = c / p.B;
+      const int ct = (p.mask_kind == ATTN_MASK_FULL) ? rank : (p.num_cta_tiles - 1 - rank);
+      cost[c] = item_geom<PAGED>(p, WorkItem{ct * kRowsPerCta, 0, c - rank * p.B}).T;
+    }
+    __syncwarp();
+    for (int c = lane; c < classes; c += 32) {
+      int r = 0;
+      for (int c2 = 0; c2 < classes; ++c2) r += (cost[c2] > cost[c]) || (cost[c2] == cost[c] && c2 < c);
+      order[r] = c;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -346,18 +373,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   if (warp >= kTmaWarp) {
     regs_dec<kRegsControl>();
-    if (warp == kTmaWarp && lane == 0) {
+    if (warp == kTmaWarp && (PAGED || lane == 0)) {
       // ---------------------------------------------------------- TMA producer
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
+      // Lane 0 waits on the ring and arms the barriers; the copies of a paged
+      // key tile (one box per pool block) go out from lanes 0 .. 128 / block_size - 1
+      // at once, lane e issuing block e. The contiguous kernel runs lane 0 alone.
+      if (lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+      }
       int g = 0;             // key tiles issued before this item (K and V alike)
       int k_issued = 0, v_issued = 0, it = 0;
       bool ok = true;
       for (int round = 0; ok; ++round) {
         const int w = item_index(round, cta, G);
         if (w >= p.num_items) break;
-        const WorkItem wi = item_at(p, w);
+        const WorkItem wi = item_at(p, w, order, use_order);
         const ItemGeom gm = item_geom<PAGED>(p, wi);
         const int kt_lo = gm.lo, T = gm.T;
         const int zq = wi.b * p.Hq + wi.h;
@@ -372,98 +404,96 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // slots past seq_len arrive as zeros, never as stale pool contents: their
         // probabilities are 0, and 0 * NaN would still poison P.V.
         //
-        // The table entries of a key tile are read one tile ahead (all of them in
-        // flight at once) and kept for the V copy of the same tile, so the
-        // producer never waits on a table read between two copies.
-        constexpr int kMaxBoxes = kBN / 16;
-        auto fetch_entries = [&](int kt, int (&ent)[kMaxBoxes]) {
-          if (!PAGED) return;
-          const int bs = p.block_size;
-#pragma unroll
-          for (int e = 0; e < kMaxBoxes; ++e) {
-            const int key = kt * kBN + e * bs;
-            ent[e] = p.num_blocks;
-            if (e * bs < kBN && !gm.bad && key < gm.nk)
-              ent[e] = __ldg(p.block_table + static_cast<size_t>(wi.b) * p.max_blocks + key / bs);
-          }
+        // Each lane reads its block's table entry one key tile ahead and keeps it
+        // for the V copy of the same tile, so no copy waits on a table read.
+        const int bs = PAGED ? p.block_size : kBN;
+        const int boxes = kBN / bs;
+        auto fetch = [&](int kt) -> int {
+          if (!PAGED) return 0;
+          const int key = kt * kBN + lane * bs;
+          return (lane < boxes && !gm.bad && key < gm.nk)
+                     ? __ldg(p.block_table + static_cast<size_t>(wi.b) * p.max_blocks + key / bs)
+                     : p.num_blocks;
         };
         auto load_kv = [&](const CUtensorMap* tm, const CUtensorMap* tm_row, uint32_t dst, uint32_t bar_full, int kt,
-                           const int (&ent)[kMaxBoxes]) {
+                           int ent) {
           if (!PAGED) {
-            for (int hh = 0; hh < C::kHalves; ++hh)
-              tma_load_3d(dst + hh * C::kHalf, tm, bar_full, hh * 64, kt * kBN, zkv);
-          } else {
-            const int bs = p.block_size;
-#pragma unroll
-            for (int e = 0; e < kMaxBoxes; ++e) {
-              if (e * bs >= kBN) break;
-              const int key = kt * kBN + e * bs;
-              const int phys = (ent[e] >= 0 && ent[e] < p.num_blocks) ? ent[e] : p.num_blocks;
-              const uint32_t bdst = dst + e * bs * 128;
-              if (key + bs <= gm.nk || phys == p.num_blocks) {
+            if (lane == 0)
+              for (int hh = 0; hh < C::kHalves; ++hh)
+                tma_load_3d(dst + hh * C::kHalf, tm, bar_full, hh * 64, kt * kBN, zkv);
+          } else if (lane < boxes) {
+            const int key = kt * kBN + lane * bs;
+            const int phys = (ent >= 0 && ent < p.num_blocks) ? ent : p.num_blocks;
+            const uint32_t bdst = dst + lane * bs * 128;
+            if (key + bs <= gm.nk || phys == p.num_blocks) {
+              for (int hh = 0; hh < C::kHalves; ++hh)
+                tma_load_4d(bdst + hh * C::kHalf, tm, bar_full, hh * 64, kvh, 0, phys);
+            } else {
+              const int valid = gm.nk - key;  // 1 .. bs - 1 rows hold tokens
+              for (int slot = 0; slot < bs; ++slot)
                 for (int hh = 0; hh < C::kHalves; ++hh)
-                  tma_load_4d(bdst + hh * C::kHalf, tm, bar_full, hh * 64, kvh, 0, phys);
-              } else {
-                const int valid = gm.nk - key;  // 1 .. bs - 1 rows hold tokens
-                for (int slot = 0; slot < bs; ++slot)
-                  for (int hh = 0; hh < C::kHalves; ++hh)
-                    tma_load_4d(bdst + hh * C::kHalf + slot * 128, tm_row, bar_full, hh * 64, kvh, slot,
-                                slot < valid ? phys : p.num_blocks);
-              }
+                  tma_load_4d(bdst + hh * C::kHalf + slot * 128, tm_row, bar_full, hh * 64, kvh, slot,
+                              slot < valid ? phys : p.num_blocks);
             }
           }
         };
-        int ent_k[kMaxBoxes], ent_v[kMaxBoxes];  // entries of key tiles i and i - 1
-        fetch_entries(kt_lo, ent_k);
+        int ent_k = fetch(kt_lo), ent_v = p.num_blocks;  // entries of key tiles i and i - 1
         // Q of this item once the previous item's last score MMA has read its Q
-        if (it > 0 && !mbar_wait_bounded(bar(kBarQEmpty), (it - 1) & 1, budget, abort_flag)) {
-          ok = false;
-          break;
+        bool armed = true;
+        if (lane == 0) {
+          armed = (it == 0) || mbar_wait_bounded(bar(kBarQEmpty), (it - 1) & 1, budget, abort_flag);
+          if (armed) {
+            mbar_arrive_expect_tx(bar(kBarQFull), kTilesPerCta * C::kTile);
+            for (int x = 0; x < kTilesPerCta; ++x)
+              for (int hh = 0; hh < C::kHalves; ++hh)
+                tma_load_3d(sbase + C::kQOff + x * C::kTile + hh * C::kHalf, &tm_q, bar(kBarQFull), hh * 64,
+                            wi.q0 + x * kBM, zq);
+          }
         }
-        mbar_arrive_expect_tx(bar(kBarQFull), kTilesPerCta * C::kTile);
-        for (int x = 0; x < kTilesPerCta; ++x)
-          for (int hh = 0; hh < C::kHalves; ++hh)
-            tma_load_3d(sbase + C::kQOff + x * C::kTile + hh * C::kHalf, &tm_q, bar(kBarQFull), hh * 64,
-                        wi.q0 + x * kBM, zq);
+        ok = PAGED ? __shfl_sync(0xffffffffu, armed, 0) : armed;
+        if (!ok) break;
         // K_i is issued before V_{i-1}: the score MMA needs K one tile earlier than P.V needs V.
         for (int i = 0; i <= T; ++i) {
           if (i < T) {
             const int gi = g + i, s = gi % C::kKStages, rnd = gi / C::kKStages;
-            if (rnd > 0 && !mbar_wait_bounded(bar(kBarKEmpty + s), (rnd - 1) & 1, budget, abort_flag)) {
-              ok = false;
-              break;
+            if (lane == 0) {
+              armed = (rnd == 0) || mbar_wait_bounded(bar(kBarKEmpty + s), (rnd - 1) & 1, budget, abort_flag);
+              if (armed) mbar_arrive_expect_tx(bar(kBarKFull + s), C::kTile);
             }
-            mbar_arrive_expect_tx(bar(kBarKFull + s), C::kTile);
+            ok = PAGED ? __shfl_sync(0xffffffffu, armed, 0) : armed;
+            if (!ok) break;
             load_kv(&tm_k, &tm_kr, sbase + C::kKOff + s * C::kTile, bar(kBarKFull + s), kt_lo + i, ent_k);
             k_issued = gi + 1;
           }
           if (i >= 1) {
             const int gv = g + i - 1, s = gv % C::kVStages, rnd = gv / C::kVStages;
-            if (rnd > 0 && !mbar_wait_bounded(bar(kBarVEmpty + s), (rnd - 1) & 1, budget, abort_flag)) {
-              ok = false;
-              break;
+            if (lane == 0) {
+              armed = (rnd == 0) || mbar_wait_bounded(bar(kBarVEmpty + s), (rnd - 1) & 1, budget, abort_flag);
+              if (armed) mbar_arrive_expect_tx(bar(kBarVFull + s), C::kTile);
             }
-            mbar_arrive_expect_tx(bar(kBarVFull + s), C::kTile);
+            ok = PAGED ? __shfl_sync(0xffffffffu, armed, 0) : armed;
+            if (!ok) break;
             load_kv(&tm_v, &tm_vr, sbase + C::kVOff + s * C::kTile, bar(kBarVFull + s), kt_lo + i - 1, ent_v);
             v_issued = gv + 1;
           }
           if (PAGED) {
-#pragma unroll
-            for (int e = 0; e < kMaxBoxes; ++e) ent_v[e] = ent_k[e];
-            if (i + 1 < T) fetch_entries(kt_lo + i + 1, ent_k);
+            ent_v = ent_k;
+            if (i + 1 < T) ent_k = fetch(kt_lo + i + 1);
           }
         }
         g += T;
         ++it;
       }
-      if (!ok) raise_abort(abort_flag, p.status);
-      // Drain: the newest copy of every stage and of Q has landed before the CTA may exit.
-      volatile int never = 0;
-      if (it > 0) mbar_wait_bounded(bar(kBarQFull), (it - 1) & 1, kDrainBudgetCycles, &never);
-      for (int j = (k_issued > C::kKStages ? k_issued - C::kKStages : 0); j < k_issued; ++j)
-        mbar_wait_bounded(bar(kBarKFull + j % C::kKStages), (j / C::kKStages) & 1, kDrainBudgetCycles, &never);
-      for (int j = (v_issued > C::kVStages ? v_issued - C::kVStages : 0); j < v_issued; ++j)
-        mbar_wait_bounded(bar(kBarVFull + j % C::kVStages), (j / C::kVStages) & 1, kDrainBudgetCycles, &never);
+      if (lane == 0) {
+        if (!ok) raise_abort(abort_flag, p.status);
+        // Drain: the newest copy of every stage and of Q has landed before the CTA may exit.
+        volatile int never = 0;
+        if (it > 0) mbar_wait_bounded(bar(kBarQFull), (it - 1) & 1, kDrainBudgetCycles, &never);
+        for (int j = (k_issued > C::kKStages ? k_issued - C::kKStages : 0); j < k_issued; ++j)
+          mbar_wait_bounded(bar(kBarKFull + j % C::kKStages), (j / C::kKStages) & 1, kDrainBudgetCycles, &never);
+        for (int j = (v_issued > C::kVStages ? v_issued - C::kVStages : 0); j < v_issued; ++j)
+          mbar_wait_bounded(bar(kBarVFull + j % C::kVStages), (j / C::kVStages) & 1, kDrainBudgetCycles, &never);
+      }
     } else if (warp == kMmaWarp && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       // Descriptors are built once; an operand at byte offset o from its base has
@@ -496,7 +526,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int round = 0; ok; ++round) {
         const int w = item_index(round, cta, G);
         if (w >= p.num_items) break;
-        const WorkItem wi = item_at(p, w);
+        const WorkItem wi = item_at(p, w, order, use_order);
         const int T = item_geom<PAGED>(p, wi).T;
         if (!mbar_wait_bounded(bar(kBarQFull), it & 1, budget, abort_flag) ||
             !mbar_wait_bounded(bar(kBarKFull + g % C::kKStages), (g / C::kKStages) & 1, budget, abort_flag)) {
@@ -564,7 +594,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     for (int round = 0;; ++round) {
       const int w = item_index(round, cta, G);
       if (w >= p.num_items) break;
-      const WorkItem wi = item_at(p, w);
+      const WorkItem wi = item_at(p, w, order, use_order);
       const ItemGeom gm = item_geom<PAGED>(p, wi);
       const int kt_lo = gm.lo, T = gm.T;
       const int qr0 = wi.q0 + x * kBM;  // first query row of the tile
@@ -818,6 +848,7 @@ int launch_prefill_t(const void* q, const void* k, const void* v, void* o, float
   p.window = window;
   p.num_cta_tiles = (N + kRowsPerCta - 1) / kRowsPerCta;
   p.num_items = p.num_cta_tiles * Hq * B;
+  p.ordered = (PAGED && p.num_cta_tiles * B <= PfCfg<D>::kOrderMax) ? 1 : 0;
   p.scale_log2 = scale * kLog2e;
   p.budget = wait_budget_cycles();
   p.block_table = PAGED ? ctx->block_table : nullptr;
