@@ -419,20 +419,25 @@ struct MergeParams {
 constexpr int kMergeWarps = 8;
 constexpr int kMergeUnroll = 4;
 
-template <int D>
+// COLS < D: the row's columns are shared out over D / COLS CTAs (blockIdx.y),
+// for rows with many splits; each reads every split's log-sum-exp and its
+// own columns of the partial outputs.
+template <int D, int COLS>
 __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const MergeParams p) {
-  constexpr int PER = D / 32;  // columns per lane
+  constexpr int PER = COLS / 32;  // columns per lane
   __shared__ float s_max[kMergeWarps];
   __shared__ int s_nan[kMergeWarps];
   __shared__ float s_sum[kMergeWarps];
-  __shared__ float s_acc[kMergeWarps][D];
+  __shared__ float s_acc[kMergeWarps][COLS];
   const size_t row = blockIdx.x;  // b * Hq + h
+  const int c0 = static_cast<int>(blockIdx.y) * COLS;
+  const bool lead = (blockIdx.y == 0);  // writes the row's LSE and status bits
   const int b = static_cast<int>(row / p.Hq);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int seq_len = p.seq_lens[b];
-  __nv_bfloat16* orow = p.o + row * D + lane * PER;
+  __nv_bfloat16* orow = p.o + row * D + c0 + lane * PER;
   if (seq_len < 1 || seq_len > p.max_seq_len) {
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && lead) {
       flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
       if (p.lse) p.lse[row] = NAN;
     }
@@ -472,7 +477,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  const float* obase = p.o_part + row * p.splits * D + lane * PER;
+  const float* obase = p.o_part + row * p.splits * D + c0 + lane * PER;
   for (int base = warp; base < ns; base += kMergeUnroll * kMergeWarps) {
     float ls[kMergeUnroll];
     float v[kMergeUnroll][PER];
@@ -485,11 +490,16 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
       if (s < ns) {
         ls[u] = lrow[s];
         const float* src = obase + static_cast<size_t>(s) * D;
+        if constexpr (PER % 2 == 0) {
 #pragma unroll
-        for (int e = 0; e < PER; e += 2) {
-          const float2 x = *reinterpret_cast<const float2*>(src + e);
-          v[u][e] = x.x;
-          v[u][e + 1] = x.y;
+          for (int e = 0; e < PER; e += 2) {
+            const float2 x = *reinterpret_cast<const float2*>(src + e);
+            v[u][e] = x.x;
+            v[u][e + 1] = x.y;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < PER; ++e) v[u][e] = src[e];
         }
       }
     }
@@ -516,7 +526,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
     const float lse_out = sink_fold(p.sinks, static_cast<int>(row % p.Hq), M + __logf(total), inv, bad_sink);
     if (bad_sink) {
       any_nan = 1;
-      if (lane == 0) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
+      if (lane == 0 && lead) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
     }
     float out[PER];
 #pragma unroll
@@ -526,10 +536,15 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
       for (int w = 0; w < kMergeWarps; ++w) v += s_acc[w][lane * PER + e];
       out[e] = any_nan ? NAN : v * inv;
     }
+    if constexpr (PER % 2 == 0) {
 #pragma unroll
-    for (int e = 0; e < PER; e += 2)
-      *reinterpret_cast<__nv_bfloat162*>(orow + e) = __floats2bfloat162_rn(out[e], out[e + 1]);
-    if (lane == 0 && p.lse) p.lse[row] = any_nan ? NAN : lse_out;
+      for (int e = 0; e < PER; e += 2)
+        *reinterpret_cast<__nv_bfloat162*>(orow + e) = __floats2bfloat162_rn(out[e], out[e + 1]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < PER; ++e) orow[e] = __float2bfloat16_rn(out[e]);
+    }
+    if (lane == 0 && lead && p.lse) p.lse[row] = any_nan ? NAN : lse_out;
   }
 }
 
@@ -638,13 +653,20 @@ cudaError_t launch_decode_merge(const float* o_part, const float* lse_part, cons
   m.max_seq_len = max_seq_len;
   m.window = window;
   m.n_sink = n_sink;
-  const dim3 grid(static_cast<unsigned>(B) * static_cast<unsigned>(Hq));
+  // rows with many splits: 32 columns per CTA, so a single long sequence still
+  // spreads its merge over many SMs
+  const bool wide = splits >= 32;
+  const unsigned rows = static_cast<unsigned>(B) * static_cast<unsigned>(Hq);
+  const dim3 grid(rows, wide ? static_cast<unsigned>(d / 32) : 1u);
   if (d == 128)
-    decode_merge_kernel<128><<<grid, kMergeWarps * 32, 0, stream>>>(m);
+    wide ? decode_merge_kernel<128, 32><<<grid, kMergeWarps * 32, 0, stream>>>(m)
+         : decode_merge_kernel<128, 128><<<grid, kMergeWarps * 32, 0, stream>>>(m);
   else if (d == 64)
-    decode_merge_kernel<64><<<grid, kMergeWarps * 32, 0, stream>>>(m);
+    wide ? decode_merge_kernel<64, 32><<<grid, kMergeWarps * 32, 0, stream>>>(m)
+         : decode_merge_kernel<64, 64><<<grid, kMergeWarps * 32, 0, stream>>>(m);
   else if (d == 512)
-    decode_merge_kernel<512><<<grid, kMergeWarps * 32, 0, stream>>>(m);
+    wide ? decode_merge_kernel<512, 32><<<grid, kMergeWarps * 32, 0, stream>>>(m)
+         : decode_merge_kernel<512, 512><<<grid, kMergeWarps * 32, 0, stream>>>(m);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();
