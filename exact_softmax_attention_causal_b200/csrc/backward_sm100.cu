@@ -176,8 +176,9 @@ struct BwdCfg {
   static constexpr int kBarOff = kRowOff + 2 * 2 * kT * 4;
   static constexpr int kBytes = kBarOff + 256;
   static constexpr int kAlloc = kBytes + 1024;
-  // TMEM columns: S^T (or S) 128, dP^T (or dP) 128, then the accumulators.
-  static constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 256 + D;
+  // TMEM columns: S^T (or S) 128, dP^T (or dP) 128, then the accumulators; the dQ
+  // kernel keeps a second S buffer in the last 128 columns.
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 256 + D, kColS2 = 384;
 };
 
 enum : int {
@@ -507,25 +508,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t ddo = desc_sw128(sbase + C::kVOff, 16, 1024);
       constexpr uint32_t kIdS = idesc_bwd(kT, kT, 0, 0);   // S = Q K^T, dP = dO V^T
       constexpr uint32_t kIdAcc = idesc_bwd(kT, D, 0, 1);  // dQ += dS K (K as an MN-major B)
-      bool ok = mbar_wait_bounded(bar(kBbKV), 0, budget, abort_flag);
-      for (int t = 0; t < iters && ok; ++t) {
-        const int s = t & 1;
-        const uint32_t st = sbase + C::kQOff + s * C::kStageBytes;
-        if (!mbar_wait_bounded(bar(kBbFull + s), (t >> 1) & 1, budget, abort_flag)) {
-          ok = false;
-          break;
-        }
+      // Two S buffers (columns kColS and kColS2): S of key tile t + 1 is computed
+      // while the dS warps work on tile t; dP has one buffer, refilled once they
+      // are done with it.
+      auto col_s = [&](int t) -> uint32_t { return (t & 1) ? C::kColS2 : C::kColS; };
+      auto stage = [&](int t) -> uint32_t { return sbase + C::kQOff + (t & 1) * C::kStageBytes; };
+      auto wait_stage = [&](int t) -> bool {
+        if (!mbar_wait_bounded(bar(kBbFull + (t & 1)), (t >> 1) & 1, budget, abort_flag)) return false;
         tc_fence_after();
-        mma_kmajor<D>(tmem + C::kColS, dq, desc_sw128(st, 16, 1024), kIdS);
-        mma_kmajor<D>(tmem + C::kColDP, ddo, desc_sw128(st + C::kTile, 16, 1024), kIdS);
+        return true;
+      };
+      bool ok = mbar_wait_bounded(bar(kBbKV), 0, budget, abort_flag) && wait_stage(0);
+      if (ok) {
+        mma_kmajor<D>(tmem + col_s(0), dq, desc_sw128(stage(0), 16, 1024), kIdS);
+        mma_kmajor<D>(tmem + C::kColDP, ddo, desc_sw128(stage(0) + C::kTile, 16, 1024), kIdS);
         tc_commit(bar(kBbS));
+      }
+      for (int t = 0; t < iters && ok; ++t) {
+        const bool next = t + 1 < iters;
+        // S of the next key tile into the other buffer (its previous dS was consumed by
+        // the dQ MMA issued in the last iteration, in order)
+        if (next) {
+          if (!wait_stage(t + 1)) {
+            ok = false;
+            break;
+          }
+          mma_kmajor<D>(tmem + col_s(t + 1), dq, desc_sw128(stage(t + 1), 16, 1024), kIdS);
+        }
         if (!mbar_wait_bounded(bar(kBbP), t & 1, budget, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        mma_tmem_a(tmem + C::kColAcc0, tmem + C::kColS, desc_sw128(st, kBox, 1024), kIdAcc, t == 0);
-        tc_commit(bar(kBbEmpty + s));
+        mma_tmem_a(tmem + C::kColAcc0, tmem + col_s(t), desc_sw128(stage(t), kBox, 1024), kIdAcc, t == 0);
+        tc_commit(bar(kBbEmpty + (t & 1)));
+        if (next) {  // dP of the next key tile, now that the dS warps have read this one
+          mma_kmajor<D>(tmem + C::kColDP, ddo, desc_sw128(stage(t + 1) + C::kTile, 16, 1024), kIdS);
+          tc_commit(bar(kBbS));
+        }
       }
       if (!ok) bwd_abort(abort_flag, p.status);
       tc_commit(bar(kBbAcc));
@@ -550,6 +570,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int jt = klo + t;
+      const uint32_t colS = (t & 1) ? C::kColS2 : C::kColS;  // this key tile's S buffer
       const bool full_tile = (p.mask_kind == ATTN_MASK_FULL || (i > jt && (p.mask_kind == ATTN_MASK_CAUSAL ||
                                                                            (i * kT + kT - 1) - jt * kT < p.window))) &&
                              (i * kT + kT <= p.N) && (jt * kT + kT <= p.N);
@@ -557,7 +578,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int cc = 0; cc < 2; ++cc) {
         const int c = 2 * ch + cc;  // 32-column chunk of the tile
         uint32_t sv[32], dpv[32];
-        tmem_ld_32x32b_x32(lane_base + C::kColS + 32u * c, sv);
+        tmem_ld_32x32b_x32(lane_base + colS + 32u * c, sv);
         tmem_ld_32x32b_x32(lane_base + C::kColDP + 32u * c, dpv);
         tc_wait_ld();
         uint32_t dsk[16];
@@ -573,7 +594,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           dsk[e >> 1] = pack_bf16x2(ds[0], ds[1]);
         }
-        tmem_st_32x32b_x16(lane_base + C::kColS + 64u * ch + 16u * cc, dsk);  // dS as bf16 pairs, own half
+        tmem_st_32x32b_x16(lane_base + colS + 64u * ch + 16u * cc, dsk);  // dS as bf16 pairs, own half
       }
       tc_wait_st();
       tc_fence_before();
