@@ -691,7 +691,9 @@ int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan
   const int group = Hq / Hkv;
   const int hchunks = (group + 15) / 16;
   const long long units = static_cast<long long>(B) * Hkv * hchunks;
-  const long long target = 4LL * num_sms;  // CTAs: enough to fill every SM a few times over
+  // CTAs: at least one per SM. More, shorter splits were measured slower on
+  // single long sequences (per-CTA latency and merge work outweigh the fill).
+  const long long target = 1LL * num_sms;
   int chunk = 2048;
   while (chunk > 256 && units * ((max_seq_len + chunk - 1) / chunk) < target) chunk >>= 1;
   // spread the 16-token sub-blocks evenly over the splits (no near-empty last split)

@@ -228,15 +228,15 @@ def test_decode_plan_covers_the_sequence(B, Hq, Hkv, L):
     # the 16-token sub-blocks are spread evenly: no split holds less than a sub-block less than another
     subs = -(-L // 16)
     assert subs - (splits - 1) * (chunk // 16) >= max(1, chunk // 16 - splits)
-    # enough (sequence, kv head, head chunk, split) units for several waves on 148 SMs, unless chunks are small
+    # at least one (sequence, kv head, head chunk, split) CTA per SM of 148, unless chunks are small
     units = B * Hkv * -(-(Hq // Hkv) // 16) * splits
-    assert units >= 4 * 148 or chunk <= 256
+    assert units >= 148 or chunk <= 256
 
 
 def test_decode_plan_examples():
     assert _plan(64, 32, 8, 32768)[1:] == (2048, 16)
-    assert _plan(1, 32, 1, 131072)[1:] == (256, 512)  # 2 head chunks x 512 splits
-    assert _plan(1, 32, 8, 131072)[1:] == (1024, 128)
+    assert _plan(1, 32, 1, 131072)[1:] == (1024, 128)  # 2 head chunks x 128 splits
+    assert _plan(1, 32, 8, 131072)[1:] == (2048, 64)
     assert _plan(64, 32, 8, 4128)[1:] == (1376, 3)  # a 4096 window + 4 sinks: 258 sub-blocks in 3 even splits
     assert _plan(0, 32, 1, 131072)[0] == _lib.ATTN_ERR_INVALID_ARG
     assert _plan(1, 32, 3, 100)[0] == _lib.ATTN_ERR_INVALID_ARG
