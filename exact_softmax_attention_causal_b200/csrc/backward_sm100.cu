@@ -30,7 +30,8 @@
 // Roles in both tile kernels (320 threads): warps 0-7 compute P and dS (warp w
 // reads TMEM lanes 32 (w % 4) .. + 31, one key row (dK/dV) or query row (dQ)
 // per lane, over the column half 64 (w / 4) .. + 63), warp 8 is the TMA
-// producer, warp 9 issues the MMAs and owns TMEM. Every pipeline wait is
+// producer, warp 9 issues the MMAs and owns TMEM (the whole warp runs the issue
+// loop and one elected lane issues each MMA and commit). Every pipeline wait is
 // bounded; on expiry the CTA records ATTN_STATUS_BIT_TIMEOUT, writes NaN, drains
 // and exits.
 
@@ -104,6 +105,7 @@ __host__ __device__ constexpr uint32_t idesc_bwd(int M, int N, int a_mn, int b_m
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Both product helpers are warp-collective (the MMA warp runs them converged).
 // D x d/16 steps of a product with both operands K-major in shared memory
 // (K dimension = head dim: 64-column boxes of 16 KB hold 4 steps of 32 bytes).
 template <int D>
@@ -111,7 +113,7 @@ __device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint64_t da, uint64_
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kBox + (kk & 3) * 32) >> 4);
-    tc_mma_ss(d_tmem, da + off, db + off, idesc, kk > 0 ? 1u : 0u);
+    tc_mma_ss_w(d_tmem, da + off, db + off, idesc, kk > 0 ? 1u : 0u);
   }
 }
 // 128 / 16 steps of D (+)= A[tmem] * B[smem, MN-major, 16 rows per step]. A holds bf16 pairs
@@ -121,8 +123,8 @@ __device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uin
                                            bool first) {
 #pragma unroll
   for (int kk = 0; kk < kT / 16; ++kk)
-    tc_mma_ts(d_tmem, a_tmem + 64u * (kk >> 2) + 8u * (kk & 3), db + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
-              (!first || kk > 0) ? 1u : 0u);
+    tc_mma_ts_w(d_tmem, a_tmem + 64u * (kk >> 2) + 8u * (kk & 3), db + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
+                (!first || kk > 0) ? 1u : 0u);
 }
 
 // ---------------------------------------------------------------------------
@@ -278,41 +280,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (issued[s] > 0) mbar_wait_bounded(bar(kBbFull + s), (issued[s] - 1) & 1, kDrainBudgetCycles, &never);
     }
   } else if (warp == kBwdMmaWarp) {
-    if (lane == 0) {
-      // ---------------------------------------------------------- MMA issuer
-      const uint64_t dk = desc_sw128(sbase + C::kKOff, 16, 1024);
-      const uint64_t dvv = desc_sw128(sbase + C::kVOff, 16, 1024);
-      constexpr uint32_t kIdS = idesc_bwd(kT, kT, 0, 0);   // S^T = K Q^T, dP^T = V dO^T
-      constexpr uint32_t kIdAcc = idesc_bwd(kT, D, 0, 1);  // dV += P^T dO, dK += dS^T Q (B MN-major)
-      bool ok = mbar_wait_bounded(bar(kBbKV), 0, budget, abort_flag);
-      for (int t = 0; t < iters && ok; ++t) {
-        const int s = t & 1;
-        const uint32_t st = sbase + C::kQOff + s * C::kStageBytes;
-        if (!mbar_wait_bounded(bar(kBbFull + s), (t >> 1) & 1, budget, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        mma_kmajor<D>(tmem + C::kColS, dk, desc_sw128(st, 16, 1024), kIdS);
-        mma_kmajor<D>(tmem + C::kColDP, dvv, desc_sw128(st + C::kTile, 16, 1024), kIdS);
-        tc_commit(bar(kBbS));
-        if (!mbar_wait_bounded(bar(kBbP), t & 1, budget, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // B = dO (then Q) as an MN-major operand: N = head dim (64-column boxes kBox apart),
-        // K = query rows (16 per step, 2 KB apart)
-        mma_tmem_a(tmem + C::kColAcc0, tmem + C::kColS, desc_sw128(st + C::kTile, kBox, 1024), kIdAcc, t == 0);
-        mma_tmem_a(tmem + C::kColAcc1, tmem + C::kColDP, desc_sw128(st, kBox, 1024), kIdAcc, t == 0);
-        tc_commit(bar(kBbEmpty + s));
+    // ------------------------------------------------------------ MMA issuer (whole warp)
+    const uint64_t dk = desc_sw128(sbase + C::kKOff, 16, 1024);
+    const uint64_t dvv = desc_sw128(sbase + C::kVOff, 16, 1024);
+    constexpr uint32_t kIdS = idesc_bwd(kT, kT, 0, 0);   // S^T = K Q^T, dP^T = V dO^T
+    constexpr uint32_t kIdAcc = idesc_bwd(kT, D, 0, 1);  // dV += P^T dO, dK += dS^T Q (B MN-major)
+    auto wait = [&](uint32_t b_, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait_bounded(b_, parity, budget, abort_flag));
+    };
+    bool ok = wait(bar(kBbKV), 0);
+    for (int t = 0; t < iters && ok; ++t) {
+      const int s = t & 1;
+      const uint32_t st = sbase + C::kQOff + s * C::kStageBytes;
+      if (!wait(bar(kBbFull + s), (t >> 1) & 1)) {
+        ok = false;
+        break;
       }
-      if (!ok) bwd_abort(abort_flag, p.status);
-      tc_commit(bar(kBbAcc));
-      tc_commit(bar(kBbDrain));
-      volatile int never = 0;
-      mbar_wait_bounded(bar(kBbDrain), 0, kDrainBudgetCycles, &never);
+      tc_fence_after();
+      mma_kmajor<D>(tmem + C::kColS, dk, desc_sw128(st, 16, 1024), kIdS);
+      mma_kmajor<D>(tmem + C::kColDP, dvv, desc_sw128(st + C::kTile, 16, 1024), kIdS);
+      tc_commit_w(bar(kBbS));
+      if (!wait(bar(kBbP), t & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // B = dO (then Q) as an MN-major operand: N = head dim (64-column boxes kBox apart),
+      // K = query rows (16 per step, 2 KB apart)
+      mma_tmem_a(tmem + C::kColAcc0, tmem + C::kColS, desc_sw128(st + C::kTile, kBox, 1024), kIdAcc, t == 0);
+      mma_tmem_a(tmem + C::kColAcc1, tmem + C::kColDP, desc_sw128(st, kBox, 1024), kIdAcc, t == 0);
+      tc_commit_w(bar(kBbEmpty + s));
     }
+    if (!ok && lane == 0) bwd_abort(abort_flag, p.status);
+    tc_commit_w(bar(kBbAcc));
+    tc_commit_w(bar(kBbDrain));
+    volatile int never = 0;
+    mbar_wait_bounded(bar(kBbDrain), 0, kDrainBudgetCycles, &never);
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ P / dS warps 0-7
     const int r = (warp & 3) * 32 + lane;  // key row of the tile = TMEM lane
@@ -321,13 +325,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int kpos = j * kT + r;
     const float sl2 = p.scale_log2;
     bool ok = true;
-    for (int t = 0; t < iters; ++t) {
+    int i = qlo;  // query tile of pair t: pairs run head-major, so i cycles through qlo .. qhi
+    for (int t = 0; t < iters; ++t, i = (i == qhi) ? qlo : i + 1) {
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbS), t & 1, budget, abort_flag));
       // the staged rows: observe their own barrier too (already complete once the S MMAs ran)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbFull + (t & 1)), (t >> 1) & 1, budget, abort_flag));
       if (!ok) break;  // no named barriers here: leaving early strands no other warp
       tc_fence_after();
-      const int i = qlo + t % nq;
       // LSE * log2(e) and D of the pair's 128 query rows, staged in shared memory with Q and dO
       // (the MMA warp consumed stage t & 1 only after the S MMAs, which precede this wait)
       const float* srow = reinterpret_cast<const float*>(smem + C::kRowOff + (t & 1) * (2 * kT * 4));
@@ -356,20 +360,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           dd[e + 2] = dv4.z;
           dd[e + 3] = dv4.w;
         }
+        if (!full_tile) {
+          // hidden (query, key) entries: LSE +inf makes the exponent -inf and P exactly 0
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int qpos = i * kT + 32 * c + e;
+            if (!(qpos < p.N && kpos < p.N && bwd_visible(p, qpos, kpos))) l2[e] = INFINITY;
+          }
+        }
         tc_wait_ld();
         uint32_t pk[16], dsk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          float pr[2], ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int qpos = i * kT + 32 * c + e + u;
-            const bool vis = full_tile || (qpos < p.N && kpos < p.N && bwd_visible(p, qpos, kpos));
-            pr[u] = vis ? fast_exp2(__uint_as_float(sv[e + u]) * sl2 - l2[e + u]) : 0.f;
-            ds[u] = pr[u] * (__uint_as_float(dpv[e + u]) - dd[e + u]);
-          }
-          pk[e >> 1] = pack_bf16x2(pr[0], pr[1]);
-          dsk[e >> 1] = pack_bf16x2(ds[0], ds[1]);
+          const float p0 = exp2_approx(fmaf(__uint_as_float(sv[e]), sl2, -l2[e]));
+          const float p1 = exp2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -l2[e + 1]));
+          pk[e >> 1] = pack_bf16x2(p0, p1);
+          dsk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(dpv[e]) - dd[e]), p1 * (__uint_as_float(dpv[e + 1]) - dd[e + 1]));
         }
         // bf16 pairs over this warp's columns already read: 64 ch + 16 cc
         tmem_st_32x32b_x16(lane_base + C::kColS + 64u * ch + 16u * cc, pk);
@@ -502,57 +508,59 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (issued[s] > 0) mbar_wait_bounded(bar(kBbFull + s), (issued[s] - 1) & 1, kDrainBudgetCycles, &never);
     }
   } else if (warp == kBwdMmaWarp) {
-    if (lane == 0) {
-      // ---------------------------------------------------------- MMA issuer
-      const uint64_t dq = desc_sw128(sbase + C::kKOff, 16, 1024);
-      const uint64_t ddo = desc_sw128(sbase + C::kVOff, 16, 1024);
-      constexpr uint32_t kIdS = idesc_bwd(kT, kT, 0, 0);   // S = Q K^T, dP = dO V^T
-      constexpr uint32_t kIdAcc = idesc_bwd(kT, D, 0, 1);  // dQ += dS K (K as an MN-major B)
-      // Two S buffers (columns kColS and kColS2): S of key tile t + 1 is computed
-      // while the dS warps work on tile t; dP has one buffer, refilled once they
-      // are done with it.
-      auto col_s = [&](int t) -> uint32_t { return (t & 1) ? C::kColS2 : C::kColS; };
-      auto stage = [&](int t) -> uint32_t { return sbase + C::kQOff + (t & 1) * C::kStageBytes; };
-      auto wait_stage = [&](int t) -> bool {
-        if (!mbar_wait_bounded(bar(kBbFull + (t & 1)), (t >> 1) & 1, budget, abort_flag)) return false;
-        tc_fence_after();
-        return true;
-      };
-      bool ok = mbar_wait_bounded(bar(kBbKV), 0, budget, abort_flag) && wait_stage(0);
-      if (ok) {
-        mma_kmajor<D>(tmem + col_s(0), dq, desc_sw128(stage(0), 16, 1024), kIdS);
-        mma_kmajor<D>(tmem + C::kColDP, ddo, desc_sw128(stage(0) + C::kTile, 16, 1024), kIdS);
-        tc_commit(bar(kBbS));
-      }
-      for (int t = 0; t < iters && ok; ++t) {
-        const bool next = t + 1 < iters;
-        // S of the next key tile into the other buffer (its previous dS was consumed by
-        // the dQ MMA issued in the last iteration, in order)
-        if (next) {
-          if (!wait_stage(t + 1)) {
-            ok = false;
-            break;
-          }
-          mma_kmajor<D>(tmem + col_s(t + 1), dq, desc_sw128(stage(t + 1), 16, 1024), kIdS);
-        }
-        if (!mbar_wait_bounded(bar(kBbP), t & 1, budget, abort_flag)) {
+    // ------------------------------------------------------------ MMA issuer (whole warp)
+    const uint64_t dq = desc_sw128(sbase + C::kKOff, 16, 1024);
+    const uint64_t ddo = desc_sw128(sbase + C::kVOff, 16, 1024);
+    constexpr uint32_t kIdS = idesc_bwd(kT, kT, 0, 0);   // S = Q K^T, dP = dO V^T
+    constexpr uint32_t kIdAcc = idesc_bwd(kT, D, 0, 1);  // dQ += dS K (K as an MN-major B)
+    // Two S buffers (columns kColS and kColS2): S of key tile t + 1 is computed
+    // while the dS warps work on tile t; dP has one buffer, refilled once they
+    // are done with it.
+    auto col_s = [&](int t) -> uint32_t { return (t & 1) ? C::kColS2 : C::kColS; };
+    auto stage = [&](int t) -> uint32_t { return sbase + C::kQOff + (t & 1) * C::kStageBytes; };
+    auto wait = [&](uint32_t b_, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait_bounded(b_, parity, budget, abort_flag));
+    };
+    auto wait_stage = [&](int t) -> bool {
+      if (!wait(bar(kBbFull + (t & 1)), (t >> 1) & 1)) return false;
+      tc_fence_after();
+      return true;
+    };
+    bool ok = wait(bar(kBbKV), 0) && wait_stage(0);
+    if (ok) {
+      mma_kmajor<D>(tmem + col_s(0), dq, desc_sw128(stage(0), 16, 1024), kIdS);
+      mma_kmajor<D>(tmem + C::kColDP, ddo, desc_sw128(stage(0) + C::kTile, 16, 1024), kIdS);
+      tc_commit_w(bar(kBbS));
+    }
+    for (int t = 0; t < iters && ok; ++t) {
+      const bool next = t + 1 < iters;
+      // S of the next key tile into the other buffer (its previous dS was consumed by
+      // the dQ MMA issued in the last iteration, in order)
+      if (next) {
+        if (!wait_stage(t + 1)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        mma_tmem_a(tmem + C::kColAcc0, tmem + col_s(t), desc_sw128(stage(t), kBox, 1024), kIdAcc, t == 0);
-        tc_commit(bar(kBbEmpty + (t & 1)));
-        if (next) {  // dP of the next key tile, now that the dS warps have read this one
-          mma_kmajor<D>(tmem + C::kColDP, ddo, desc_sw128(stage(t + 1) + C::kTile, 16, 1024), kIdS);
-          tc_commit(bar(kBbS));
-        }
+        mma_kmajor<D>(tmem + col_s(t + 1), dq, desc_sw128(stage(t + 1), 16, 1024), kIdS);
       }
-      if (!ok) bwd_abort(abort_flag, p.status);
-      tc_commit(bar(kBbAcc));
-      tc_commit(bar(kBbDrain));
-      volatile int never = 0;
-      mbar_wait_bounded(bar(kBbDrain), 0, kDrainBudgetCycles, &never);
+      if (!wait(bar(kBbP), t & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      mma_tmem_a(tmem + C::kColAcc0, tmem + col_s(t), desc_sw128(stage(t), kBox, 1024), kIdAcc, t == 0);
+      tc_commit_w(bar(kBbEmpty + (t & 1)));
+      if (next) {  // dP of the next key tile, now that the dS warps have read this one
+        mma_kmajor<D>(tmem + C::kColDP, ddo, desc_sw128(stage(t + 1) + C::kTile, 16, 1024), kIdS);
+        tc_commit_w(bar(kBbS));
+      }
     }
+    if (!ok && lane == 0) bwd_abort(abort_flag, p.status);
+    tc_commit_w(bar(kBbAcc));
+    tc_commit_w(bar(kBbDrain));
+    volatile int never = 0;
+    mbar_wait_bounded(bar(kBbDrain), 0, kDrainBudgetCycles, &never);
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ dS warps 0-7
     const int r = (warp & 3) * 32 + lane;  // query row of the tile = TMEM lane
@@ -581,18 +589,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld_32x32b_x32(lane_base + colS + 32u * c, sv);
         tmem_ld_32x32b_x32(lane_base + C::kColDP + 32u * c, dpv);
         tc_wait_ld();
+        if (!full_tile) {
+          // hidden (query, key) entries: a score of -inf makes P exactly 0 (scale_log2 > 0)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int kpos = jt * kT + 32 * c + e;
+            if (!(qpos < p.N && kpos < p.N && bwd_visible(p, qpos, kpos))) sv[e] = __float_as_uint(-INFINITY);
+          }
+        }
         uint32_t dsk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          float ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int kpos = jt * kT + 32 * c + e + u;
-            const bool vis = full_tile || (qpos < p.N && kpos < p.N && bwd_visible(p, qpos, kpos));
-            const float pr = vis ? fast_exp2(__uint_as_float(sv[e + u]) * sl2 - l2) : 0.f;
-            ds[u] = pr * (__uint_as_float(dpv[e + u]) - dr);
-          }
-          dsk[e >> 1] = pack_bf16x2(ds[0], ds[1]);
+          const float p0 = exp2_approx(fmaf(__uint_as_float(sv[e]), sl2, -l2));
+          const float p1 = exp2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -l2));
+          dsk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(dpv[e]) - dr), p1 * (__uint_as_float(dpv[e + 1]) - dr));
         }
         tmem_st_32x32b_x16(lane_base + colS + 64u * ch + 16u * cc, dsk);  // dS as bf16 pairs, own half
       }
