@@ -16,20 +16,25 @@
 //   bwd_rowdot_kernel  D = rowsum(dO * O), one warp per row, fp32.
 //   bwd_dkdv_kernel    one CTA per (batch, K/V head, 128-key tile): for every
 //                      query head of the group and every 128-row query tile
-//                      that sees the key tile, S^T = K Q^T and dP^T = V dO^T
-//                      into TMEM (M = keys), P^T and dS^T (bf16) written back
-//                      over them, then dV += P^T dO and dK += dS^T Q with the
-//                      probabilities read from TMEM.
+//                      that sees the key tile, in two halves of 64 query rows,
+//                      S^T = K Q^T and dP^T = V dO^T into TMEM (M = keys),
+//                      P^T and dS^T (bf16) written back over them, then
+//                      dV += P^T dO and dK += dS^T Q with the probabilities
+//                      read from TMEM. The halves alternate between two TMEM
+//                      regions, so the P / dS warps work on one half while the
+//                      tensor cores run the other's products.
 //   bwd_dq_kernel      one CTA per (batch, query head, 128-row query tile):
 //                      S = Q K^T and dP = dO V^T per key tile, dS (bf16) over
-//                      S, then dQ += dS K.
+//                      S, then dQ += dS K. S is double-buffered and dP is
+//                      released as soon as the dS warps have loaded it, so
+//                      the next tile's scores are ready when they finish.
 // Each recomputes S once more than a single fused kernel would (seven
 // 128x128xd products per tile pair instead of five), in exchange for
 // deterministic sums without a dQ accumulator shared between CTAs.
 //
 // Roles in both tile kernels (320 threads): warps 0-7 compute P and dS (warp w
 // reads TMEM lanes 32 (w % 4) .. + 31, one key row (dK/dV) or query row (dQ)
-// per lane, over the column half 64 (w / 4) .. + 63), warp 8 is the TMA
+// per lane, over the column half w / 4 of the tile or half-tile), warp 8 is the TMA
 // producer, warp 9 issues the MMAs and owns TMEM (the whole warp runs the issue
 // loop and one elected lane issues each MMA and commit). Every pipeline wait is
 // bounded; on expiry the CTA records ATTN_STATUS_BIT_TIMEOUT, writes NaN, drains
@@ -116,6 +121,16 @@ __device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint64_t da, uint64_
     tc_mma_ss_w(d_tmem, da + off, db + off, idesc, kk > 0 ? 1u : 0u);
   }
 }
+// 64 / 16 steps of the same product over half a tile (dK/dV kernel): A holds the bf16 pairs of
+// 64 K rows, written by two warps per TMEM sub-partition, each over the first half of its own
+// 32 columns: K rows 16 kk .. 16 kk + 15 sit at column 32 (kk / 2) + 8 (kk % 2).
+__device__ __forceinline__ void mma_tmem_a_half(uint32_t d_tmem, uint32_t a_tmem, uint64_t db, uint32_t idesc,
+                                                bool first) {
+#pragma unroll
+  for (int kk = 0; kk < kT / 32; ++kk)
+    tc_mma_ts_w(d_tmem, a_tmem + 32u * (kk >> 1) + 8u * (kk & 1), db + static_cast<uint64_t>((kk * 2048) >> 4),
+                idesc, (!first || kk > 0) ? 1u : 0u);
+}
 // 128 / 16 steps of D (+)= A[tmem] * B[smem, MN-major, 16 rows per step]. A holds bf16 pairs
 // written by two warps per TMEM sub-partition, each over the first half of its own 64 columns:
 // K rows 16 kk .. 16 kk + 15 sit at column 64 (kk / 4) + 8 (kk % 4).
@@ -178,19 +193,22 @@ struct BwdCfg {
   static constexpr int kBarOff = kRowOff + 2 * 2 * kT * 4;
   static constexpr int kBytes = kBarOff + 256;
   static constexpr int kAlloc = kBytes + 1024;
-  // TMEM columns: S^T (or S) 128, dP^T (or dP) 128, then the accumulators; the dQ
-  // kernel keeps a second S buffer in the last 128 columns.
+  // TMEM columns. dQ kernel: S 128, dP 128, the dQ accumulator, a second S buffer in the
+  // last 128 columns. dK/dV kernel: two regions of 128 columns, each holding one half-tile's
+  // S^T (64 columns) and dP^T (64 columns), then the dV and dK accumulators.
   static constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 256 + D, kColS2 = 384;
+  static constexpr uint32_t kRegion = 128, kRegionDP = 64;
 };
 
 enum : int {
   kBbKV = 0,       // K and V (dK/dV kernel) or Q and dO (dQ kernel) resident tiles landed
   kBbFull = 1,     // + stage (2)
   kBbEmpty = 3,    // + stage (2)
-  kBbS = 5,        // S and dP of the current pair are in TMEM
-  kBbP = 6,        // P / dS written back (4 softmax warps)
-  kBbAcc = 7,      // accumulators final
-  kBbDrain = 8,
+  kBbS = 5,        // S and dP in TMEM (dQ kernel: one; dK/dV kernel: + region (2))
+  kBbP = 7,        // P / dS written back by the 8 softmax warps (dQ: one; dK/dV: + region (2))
+  kBbAcc = 9,      // accumulators final
+  kBbDrain = 10,
+  kBbDPFree = 11,  // dQ kernel: the softmax warps have loaded dP (8 arrivals)
 };
 constexpr int kBwdTmemSlot = 128;
 constexpr int kBwdAbort = 132;
@@ -225,10 +243,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(kBbFull + s), 1);
       mbar_init(bar(kBbEmpty + s), 1);
     }
-    mbar_init(bar(kBbS), 1);
-    mbar_init(bar(kBbP), kBwdSoftWarps);
+    for (int r = 0; r < 2; ++r) {
+      mbar_init(bar(kBbS + r), 1);
+      mbar_init(bar(kBbP + r), kBwdSoftWarps);
+    }
     mbar_init(bar(kBbAcc), 1);
     mbar_init(bar(kBbDrain), 1);
+    mbar_init(bar(kBbDPFree), kBwdSoftWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -283,33 +304,55 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ------------------------------------------------------------ MMA issuer (whole warp)
     const uint64_t dk = desc_sw128(sbase + C::kKOff, 16, 1024);
     const uint64_t dvv = desc_sw128(sbase + C::kVOff, 16, 1024);
-    constexpr uint32_t kIdS = idesc_bwd(kT, kT, 0, 0);   // S^T = K Q^T, dP^T = V dO^T
-    constexpr uint32_t kIdAcc = idesc_bwd(kT, D, 0, 1);  // dV += P^T dO, dK += dS^T Q (B MN-major)
+    constexpr uint32_t kIdS = idesc_bwd(kT, kT / 2, 0, 0);  // S^T = K Q^T, dP^T = V dO^T (64 query rows)
+    constexpr uint32_t kIdAcc = idesc_bwd(kT, D, 0, 1);     // dV += P^T dO, dK += dS^T Q (B MN-major)
+    constexpr uint32_t kHalfRows = (kT / 2) * 128;          // bytes of 64 rows in a 128-byte-swizzled box
     auto wait = [&](uint32_t b_, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait_bounded(b_, parity, budget, abort_flag));
     };
-    bool ok = wait(bar(kBbKV), 0);
-    for (int t = 0; t < iters && ok; ++t) {
-      const int s = t & 1;
-      const uint32_t st = sbase + C::kQOff + s * C::kStageBytes;
-      if (!wait(bar(kBbFull + s), (t >> 1) & 1)) {
-        ok = false;
-        break;
-      }
+    // Half u covers query rows 64 (u % 2) .. + 63 of pair u / 2 and uses TMEM region u % 2.
+    auto half_stage = [&](int u) -> uint32_t {
+      return sbase + C::kQOff + ((u >> 1) & 1) * C::kStageBytes + (u & 1) * kHalfRows;
+    };
+    auto issue_s = [&](int u) {
+      const uint32_t st = half_stage(u);
+      const uint32_t reg = tmem + C::kRegion * (u & 1);
+      mma_kmajor<D>(reg, dk, desc_sw128(st, 16, 1024), kIdS);
+      mma_kmajor<D>(reg + C::kRegionDP, dvv, desc_sw128(st + C::kTile, 16, 1024), kIdS);
+      tc_commit_w(bar(kBbS + (u & 1)));
+    };
+    const int halves = 2 * iters;
+    bool ok = wait(bar(kBbKV), 0) && wait(bar(kBbFull), 0);
+    if (ok) {
       tc_fence_after();
-      mma_kmajor<D>(tmem + C::kColS, dk, desc_sw128(st, 16, 1024), kIdS);
-      mma_kmajor<D>(tmem + C::kColDP, dvv, desc_sw128(st + C::kTile, 16, 1024), kIdS);
-      tc_commit_w(bar(kBbS));
-      if (!wait(bar(kBbP), t & 1)) {
+      issue_s(0);
+      issue_s(1);
+    }
+    for (int u = 0; u < halves && ok; ++u) {
+      const int r = u & 1, t = u >> 1;
+      if (!wait(bar(kBbP + r), (u >> 1) & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
       // B = dO (then Q) as an MN-major operand: N = head dim (64-column boxes kBox apart),
       // K = query rows (16 per step, 2 KB apart)
-      mma_tmem_a(tmem + C::kColAcc0, tmem + C::kColS, desc_sw128(st + C::kTile, kBox, 1024), kIdAcc, t == 0);
-      mma_tmem_a(tmem + C::kColAcc1, tmem + C::kColDP, desc_sw128(st, kBox, 1024), kIdAcc, t == 0);
-      tc_commit_w(bar(kBbEmpty + s));
+      const uint32_t st = half_stage(u);
+      const uint32_t reg = tmem + C::kRegion * r;
+      mma_tmem_a_half(tmem + C::kColAcc0, reg, desc_sw128(st + C::kTile, kBox, 1024), kIdAcc, u == 0);
+      mma_tmem_a_half(tmem + C::kColAcc1, reg + C::kRegionDP, desc_sw128(st, kBox, 1024), kIdAcc, u == 0);
+      if (r == 1) tc_commit_w(bar(kBbEmpty + (t & 1)));  // the pair's last read of its stage
+      if (u + 2 < halves) {
+        // the next half in this region, issued behind the products that read the region
+        if (r == 0) {  // it opens pair t + 1
+          if (!wait(bar(kBbFull + ((t + 1) & 1)), ((t + 1) >> 1) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        issue_s(u + 2);
+      }
     }
     if (!ok && lane == 0) bwd_abort(abort_flag, p.status);
     tc_commit_w(bar(kBbAcc));
@@ -320,30 +363,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else {
     // ------------------------------------------------------------ P / dS warps 0-7
     const int r = (warp & 3) * 32 + lane;  // key row of the tile = TMEM lane
-    const int ch = warp >> 2;              // query columns 64 ch .. 64 ch + 63
+    const int ch = warp >> 2;              // query rows 32 ch .. 32 ch + 31 of each half-tile
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int kpos = j * kT + r;
     const float sl2 = p.scale_log2;
     bool ok = true;
     int i = qlo;  // query tile of pair t: pairs run head-major, so i cycles through qlo .. qhi
-    for (int t = 0; t < iters; ++t, i = (i == qhi) ? qlo : i + 1) {
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbS), t & 1, budget, abort_flag));
+    const int halves = 2 * iters;
+    for (int u = 0; u < halves; ++u) {
+      const int hf = u & 1, t = u >> 1;  // half-tile (= TMEM region) and pair
+      if (u > 0 && hf == 0) i = (i == qhi) ? qlo : i + 1;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbS + hf), (u >> 1) & 1, budget, abort_flag));
       // the staged rows: observe their own barrier too (already complete once the S MMAs ran)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbFull + (t & 1)), (t >> 1) & 1, budget, abort_flag));
       if (!ok) break;  // no named barriers here: leaving early strands no other warp
       tc_fence_after();
       // LSE * log2(e) and D of the pair's 128 query rows, staged in shared memory with Q and dO
-      // (the MMA warp consumed stage t & 1 only after the S MMAs, which precede this wait)
+      // (the MMA warp releases stage t & 1 only after the pair's last products, which wait for
+      // this half's P / dS)
       const float* srow = reinterpret_cast<const float*>(smem + C::kRowOff + (t & 1) * (2 * kT * 4));
       const bool full_tile = (p.mask_kind == ATTN_MASK_FULL || (i > j && (p.mask_kind == ATTN_MASK_CAUSAL ||
                                                                           (i * kT + kT - 1) - j * kT < p.window))) &&
                              (i * kT + kT <= p.N) && (j * kT + kT <= p.N);
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * ch + cc;  // 32-column chunk of the tile
+      const uint32_t reg = lane_base + C::kRegion * hf;
+      {
+        const int c = 2 * hf + ch;  // 32-column chunk of the tile: query rows 32 c .. 32 c + 31
         uint32_t sv[32], dpv[32];
-        tmem_ld_32x32b_x32(lane_base + C::kColS + 32u * c, sv);
-        tmem_ld_32x32b_x32(lane_base + C::kColDP + 32u * c, dpv);
+        tmem_ld_32x32b_x32(reg + 32u * ch, sv);
+        tmem_ld_32x32b_x32(reg + C::kRegionDP + 32u * ch, dpv);
         // the 32 query columns' LSE (base 2) and D: broadcast shared-memory reads;
         // rows past N carry +inf and 0
         float l2[32], dd[32];
@@ -377,14 +424,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pk[e >> 1] = pack_bf16x2(p0, p1);
           dsk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(dpv[e]) - dd[e]), p1 * (__uint_as_float(dpv[e + 1]) - dd[e + 1]));
         }
-        // bf16 pairs over this warp's columns already read: 64 ch + 16 cc
-        tmem_st_32x32b_x16(lane_base + C::kColS + 64u * ch + 16u * cc, pk);
-        tmem_st_32x32b_x16(lane_base + C::kColDP + 64u * ch + 16u * cc, dsk);
+        // bf16 pairs over the first half of this warp's own (already read) columns
+        tmem_st_32x32b_x16(reg + 32u * ch, pk);
+        tmem_st_32x32b_x16(reg + C::kRegionDP + 32u * ch, dsk);
       }
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBbP));
+      if (lane == 0) mbar_arrive(bar(kBbP + hf));
     }
     // ------------------------------------------------------------ epilogue
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbAcc), 0, budget, abort_flag));
@@ -458,10 +505,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(kBbFull + s), 1);
       mbar_init(bar(kBbEmpty + s), 1);
     }
-    mbar_init(bar(kBbS), 1);
-    mbar_init(bar(kBbP), kBwdSoftWarps);
+    for (int r = 0; r < 2; ++r) {
+      mbar_init(bar(kBbS + r), 1);
+      mbar_init(bar(kBbP + r), kBwdSoftWarps);
+    }
     mbar_init(bar(kBbAcc), 1);
     mbar_init(bar(kBbDrain), 1);
+    mbar_init(bar(kBbDPFree), kBwdSoftWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -543,6 +593,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mma_kmajor<D>(tmem + col_s(t + 1), dq, desc_sw128(stage(t + 1), 16, 1024), kIdS);
       }
+      if (next) {  // dP of the next key tile, as soon as the dS warps have loaded this one
+        if (!wait(bar(kBbDPFree), t & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        mma_kmajor<D>(tmem + C::kColDP, ddo, desc_sw128(stage(t + 1) + C::kTile, 16, 1024), kIdS);
+        tc_commit_w(bar(kBbS));
+      }
       if (!wait(bar(kBbP), t & 1)) {
         ok = false;
         break;
@@ -550,10 +609,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       mma_tmem_a(tmem + C::kColAcc0, tmem + col_s(t), desc_sw128(stage(t), kBox, 1024), kIdAcc, t == 0);
       tc_commit_w(bar(kBbEmpty + (t & 1)));
-      if (next) {  // dP of the next key tile, now that the dS warps have read this one
-        mma_kmajor<D>(tmem + C::kColDP, ddo, desc_sw128(stage(t + 1) + C::kTile, 16, 1024), kIdS);
-        tc_commit_w(bar(kBbS));
-      }
     }
     if (!ok && lane == 0) bwd_abort(abort_flag, p.status);
     tc_commit_w(bar(kBbAcc));
@@ -582,12 +637,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool full_tile = (p.mask_kind == ATTN_MASK_FULL || (i > jt && (p.mask_kind == ATTN_MASK_CAUSAL ||
                                                                            (i * kT + kT - 1) - jt * kT < p.window))) &&
                              (i * kT + kT <= p.N) && (jt * kT + kT <= p.N);
-#pragma unroll 1
+      // both chunks of dP first: once they are in registers the MMA warp may refill dP
+      uint32_t dpa[2][32];
+      tmem_ld_32x32b_x32(lane_base + C::kColDP + 32u * (2 * ch), dpa[0]);
+      tmem_ld_32x32b_x32(lane_base + C::kColDP + 32u * (2 * ch + 1), dpa[1]);
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBbDPFree));
+#pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         const int c = 2 * ch + cc;  // 32-column chunk of the tile
-        uint32_t sv[32], dpv[32];
+        uint32_t sv[32];
+        const uint32_t* dpv = dpa[cc];
         tmem_ld_32x32b_x32(lane_base + colS + 32u * c, sv);
-        tmem_ld_32x32b_x32(lane_base + C::kColDP + 32u * c, dpv);
         tc_wait_ld();
         if (!full_tile) {
           // hidden (query, key) entries: a score of -inf makes P exactly 0 (scale_log2 > 0)
