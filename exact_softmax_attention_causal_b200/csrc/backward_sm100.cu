@@ -34,7 +34,8 @@
 //
 // Roles in both tile kernels (320 threads): warps 0-7 compute P and dS (warp w
 // reads TMEM lanes 32 (w % 4) .. + 31, one key row (dK/dV) or query row (dQ)
-// per lane, over the column half w / 4 of the tile or half-tile), warp 8 is the TMA
+// per lane; in the dQ kernel over the column half w / 4 of each tile, in the
+// dK/dV kernel over the half-tiles of TMEM region w / 4), warp 8 is the TMA
 // producer, warp 9 issues the MMAs and owns TMEM (the whole warp runs the issue
 // loop and one elected lane issues each MMA and commit). Every pipeline wait is
 // bounded; on expiry the CTA records ATTN_STATUS_BIT_TIMEOUT, writes NaN, drains
@@ -122,8 +123,8 @@ __device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint64_t da, uint64_
   }
 }
 // 64 / 16 steps of the same product over half a tile (dK/dV kernel): A holds the bf16 pairs of
-// 64 K rows, written by two warps per TMEM sub-partition, each over the first half of its own
-// 32 columns: K rows 16 kk .. 16 kk + 15 sit at column 32 (kk / 2) + 8 (kk % 2).
+// 64 K rows, written in two 32-row chunks, each over the first half of its own 32 columns:
+// K rows 16 kk .. 16 kk + 15 sit at column 32 (kk / 2) + 8 (kk % 2).
 __device__ __forceinline__ void mma_tmem_a_half(uint32_t d_tmem, uint32_t a_tmem, uint64_t db, uint32_t idesc,
                                                 bool first) {
 #pragma unroll
@@ -179,7 +180,8 @@ __global__ void bwd_rowdot_kernel(const BwdParams p) {
   }
 }
 
-// Shared-memory plan of the tile kernels (1024-byte aligned):
+// Shared-memory plan of the dK/dV kernel (1024-byte aligned) and the TMEM columns of both
+// tile kernels:
 template <int D>
 struct BwdCfg {
   static constexpr int kHalves = D / 64;
@@ -200,18 +202,49 @@ struct BwdCfg {
   static constexpr uint32_t kRegion = 128, kRegionDP = 64;
 };
 
+// Barriers of the dK/dV kernel.
 enum : int {
-  kBbKV = 0,       // K and V (dK/dV kernel) or Q and dO (dQ kernel) resident tiles landed
+  kBbKV = 0,       // K and V resident tiles landed
   kBbFull = 1,     // + stage (2)
   kBbEmpty = 3,    // + stage (2)
-  kBbS = 5,        // S and dP in TMEM (dQ kernel: one; dK/dV kernel: + region (2))
-  kBbP = 7,        // P / dS written back by the 8 softmax warps (dQ: one; dK/dV: + region (2))
+  kBbS = 5,        // S^T and dP^T of a half-tile in TMEM, + region (2)
+  kBbP = 7,        // P^T / dS^T written back by the region's 4 softmax warps, + region (2)
   kBbAcc = 9,      // accumulators final
   kBbDrain = 10,
-  kBbDPFree = 11,  // dQ kernel: the softmax warps have loaded dP (8 arrivals)
 };
 constexpr int kBwdTmemSlot = 128;
 constexpr int kBwdAbort = 132;
+
+// Shared-memory plan of the dQ kernel: Q and dO resident, K in a ring of three
+// stages and V in a ring of two. V of key tile t is released once dP(t) has read
+// it, K only after dQ(t), so the ring that is released later is the deeper one.
+template <int D>
+struct DqCfg {
+  static constexpr int kTile = BwdCfg<D>::kTile;
+  static constexpr int kKStages = 3, kVStages = 2;
+  static constexpr int kQOff = 0;
+  static constexpr int kDoOff = kTile;
+  static constexpr int kKOff = 2 * kTile;                 // + stage * kTile
+  static constexpr int kVOff = kKOff + kKStages * kTile;  // + stage * kTile
+  static constexpr int kBarOff = kVOff + kVStages * kTile;
+  static constexpr int kBytes = kBarOff + 256;
+  static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 227 * 1024, "dQ kernel shared memory");
+};
+enum : int {
+  kDqQ = 0,                 // Q and dO landed
+  kDqFullK = 1,             // + stage (3)
+  kDqEmptyK = 4,            // + stage (3)
+  kDqFullV = 7,             // + stage (2)
+  kDqEmptyV = 9,            // + stage (2)
+  kDqS = 11,                // S and dP of the current key tile are in TMEM
+  kDqP = 12,                // dS written back (8 arrivals)
+  kDqAcc = 13,
+  kDqDrain = 14,
+  kDqDPFree = 15,           // the dS warps have loaded dP (8 arrivals)
+};
+constexpr int kDqTmemSlot = 192;
+constexpr int kDqAbort = 196;
 
 // ---------------------------------------------------------------------------
 // dK, dV: one CTA per (key tile, K/V head, batch)
@@ -245,11 +278,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     for (int r = 0; r < 2; ++r) {
       mbar_init(bar(kBbS + r), 1);
-      mbar_init(bar(kBbP + r), kBwdSoftWarps);
+      mbar_init(bar(kBbP + r), kBwdSoftWarps / 2);  // the warp group of region r
     }
     mbar_init(bar(kBbAcc), 1);
     mbar_init(bar(kBbDrain), 1);
-    mbar_init(bar(kBbDPFree), kBwdSoftWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -362,35 +394,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ P / dS warps 0-7
+    // Two warp groups in ping-pong: group g = w / 4 takes the half-tiles g, g + 2, ... (TMEM
+    // region g), all 64 query rows of each, so one group computes while the other waits.
     const int r = (warp & 3) * 32 + lane;  // key row of the tile = TMEM lane
-    const int ch = warp >> 2;              // query rows 32 ch .. 32 ch + 31 of each half-tile
+    const int ch = warp >> 2;              // warp group: TMEM region, and D-column half in the epilogue
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t reg = lane_base + C::kRegion * ch;
     const int kpos = j * kT + r;
     const float sl2 = p.scale_log2;
     bool ok = true;
     int i = qlo;  // query tile of pair t: pairs run head-major, so i cycles through qlo .. qhi
-    const int halves = 2 * iters;
-    for (int u = 0; u < halves; ++u) {
-      const int hf = u & 1, t = u >> 1;  // half-tile (= TMEM region) and pair
-      if (u > 0 && hf == 0) i = (i == qhi) ? qlo : i + 1;
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbS + hf), (u >> 1) & 1, budget, abort_flag));
-      // the staged rows: observe their own barrier too (already complete once the S MMAs ran)
+    for (int t = 0; t < iters; ++t, i = (i == qhi) ? qlo : i + 1) {
+      // the staged LSE / D rows first (the MMA warp releases stage t & 1 only after the pair's
+      // last products, which wait for this group's P / dS), then this half's S^T and dP^T
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbFull + (t & 1)), (t >> 1) & 1, budget, abort_flag));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbS + ch), t & 1, budget, abort_flag));
       if (!ok) break;  // no named barriers here: leaving early strands no other warp
       tc_fence_after();
-      // LSE * log2(e) and D of the pair's 128 query rows, staged in shared memory with Q and dO
-      // (the MMA warp releases stage t & 1 only after the pair's last products, which wait for
-      // this half's P / dS)
       const float* srow = reinterpret_cast<const float*>(smem + C::kRowOff + (t & 1) * (2 * kT * 4));
       const bool full_tile = (p.mask_kind == ATTN_MASK_FULL || (i > j && (p.mask_kind == ATTN_MASK_CAUSAL ||
                                                                           (i * kT + kT - 1) - j * kT < p.window))) &&
                              (i * kT + kT <= p.N) && (j * kT + kT <= p.N);
-      const uint32_t reg = lane_base + C::kRegion * hf;
-      {
-        const int c = 2 * hf + ch;  // 32-column chunk of the tile: query rows 32 c .. 32 c + 31
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * ch + cc;  // 32-column chunk of the tile: query rows 32 c .. 32 c + 31
         uint32_t sv[32], dpv[32];
-        tmem_ld_32x32b_x32(reg + 32u * ch, sv);
-        tmem_ld_32x32b_x32(reg + C::kRegionDP + 32u * ch, dpv);
+        tmem_ld_32x32b_x32(reg + 32u * cc, sv);
+        tmem_ld_32x32b_x32(reg + C::kRegionDP + 32u * cc, dpv);
         // the 32 query columns' LSE (base 2) and D: broadcast shared-memory reads;
         // rows past N carry +inf and 0
         float l2[32], dd[32];
@@ -424,14 +454,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pk[e >> 1] = pack_bf16x2(p0, p1);
           dsk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(dpv[e]) - dd[e]), p1 * (__uint_as_float(dpv[e + 1]) - dd[e + 1]));
         }
-        // bf16 pairs over the first half of this warp's own (already read) columns
-        tmem_st_32x32b_x16(reg + 32u * ch, pk);
-        tmem_st_32x32b_x16(reg + C::kRegionDP + 32u * ch, dsk);
+        // bf16 pairs over the first half of this chunk's own (already read) columns
+        tmem_st_32x32b_x16(reg + 32u * cc, pk);
+        tmem_st_32x32b_x16(reg + C::kRegionDP + 32u * cc, dsk);
       }
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBbP + hf));
+      if (lane == 0) mbar_arrive(bar(kBbP + ch));
     }
     // ------------------------------------------------------------ epilogue
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbAcc), 0, budget, abort_flag));
@@ -479,9 +509,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const BwdParams p) {
-  using C = BwdCfg<D>;
-  // same plan as the dK/dV kernel with the roles swapped: Q and dO resident
-  // (kKOff / kVOff), two stages of (K, V)
+  using C = BwdCfg<D>;  // TMEM columns
+  using Q = DqCfg<D>;   // shared memory and barriers
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
@@ -495,23 +524,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int iters = khi - klo + 1;
   const int kvh = h / p.group;
 
-  const uint32_t bars = sbase + C::kBarOff;
+  const uint32_t bars = sbase + Q::kBarOff;
   auto bar = [&](int x) -> uint32_t { return bars + 8u * static_cast<uint32_t>(x); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + kBwdTmemSlot);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + kBwdAbort);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Q::kBarOff + kDqTmemSlot);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Q::kBarOff + kDqAbort);
   if (threadIdx.x == 0) {
-    mbar_init(bar(kBbKV), 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(kBbFull + s), 1);
-      mbar_init(bar(kBbEmpty + s), 1);
+    mbar_init(bar(kDqQ), 1);
+    for (int s = 0; s < Q::kKStages; ++s) {
+      mbar_init(bar(kDqFullK + s), 1);
+      mbar_init(bar(kDqEmptyK + s), 1);
     }
-    for (int r = 0; r < 2; ++r) {
-      mbar_init(bar(kBbS + r), 1);
-      mbar_init(bar(kBbP + r), kBwdSoftWarps);
+    for (int s = 0; s < Q::kVStages; ++s) {
+      mbar_init(bar(kDqFullV + s), 1);
+      mbar_init(bar(kDqEmptyV + s), 1);
     }
-    mbar_init(bar(kBbAcc), 1);
-    mbar_init(bar(kBbDrain), 1);
-    mbar_init(bar(kBbDPFree), kBwdSoftWarps);
+    mbar_init(bar(kDqS), 1);
+    mbar_init(bar(kDqP), kBwdSoftWarps);
+    mbar_init(bar(kDqAcc), 1);
+    mbar_init(bar(kDqDrain), 1);
+    mbar_init(bar(kDqDPFree), kBwdSoftWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -529,92 +560,111 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       // ---------------------------------------------------------- TMA producer
       const int zq = b * p.Hq + h, zkv = b * p.Hkv + kvh;
-      mbar_arrive_expect_tx(bar(kBbKV), 2 * C::kTile);
+      mbar_arrive_expect_tx(bar(kDqQ), 2 * C::kTile);
       for (int hh = 0; hh < C::kHalves; ++hh) {
-        tma_load_3d(sbase + C::kKOff + hh * kBox, &tm_q, bar(kBbKV), hh * 64, i * kT, zq);
-        tma_load_3d(sbase + C::kVOff + hh * kBox, &tm_do, bar(kBbKV), hh * 64, i * kT, zq);
+        tma_load_3d(sbase + Q::kQOff + hh * kBox, &tm_q, bar(kDqQ), hh * 64, i * kT, zq);
+        tma_load_3d(sbase + Q::kDoOff + hh * kBox, &tm_do, bar(kDqQ), hh * 64, i * kT, zq);
       }
-      int issued[2] = {0, 0};
+      int nk[Q::kKStages] = {}, nv[Q::kVStages] = {};  // loads issued per stage
       bool ok = true;
       for (int t = 0; t < iters && ok; ++t) {
-        const int s = t & 1;
-        if (t >= 2 && !mbar_wait_bounded(bar(kBbEmpty + s), ((t - 2) >> 1) & 1, budget, abort_flag)) {
+        const int jt = klo + t;
+        const int sk = t % Q::kKStages, sv = t % Q::kVStages;
+        // K of key tile t: its stage held K(t - 3), released after dQ(t - 3)
+        if (nk[sk] > 0 && !mbar_wait_bounded(bar(kDqEmptyK + sk), (nk[sk] - 1) & 1, budget, abort_flag)) {
           ok = false;
           break;
         }
-        const int jt = klo + t;
-        const uint32_t st = sbase + C::kQOff + s * C::kStageBytes;
-        mbar_arrive_expect_tx(bar(kBbFull + s), 2 * C::kTile);
-        for (int hh = 0; hh < C::kHalves; ++hh) {
-          tma_load_3d(st + hh * kBox, &tm_k, bar(kBbFull + s), hh * 64, jt * kT, zkv);
-          tma_load_3d(st + C::kTile + hh * kBox, &tm_v, bar(kBbFull + s), hh * 64, jt * kT, zkv);
+        mbar_arrive_expect_tx(bar(kDqFullK + sk), C::kTile);
+        for (int hh = 0; hh < C::kHalves; ++hh)
+          tma_load_3d(sbase + Q::kKOff + sk * C::kTile + hh * kBox, &tm_k, bar(kDqFullK + sk), hh * 64, jt * kT, zkv);
+        ++nk[sk];
+        // V of key tile t: its stage held V(t - 2), released after dP(t - 2)
+        if (nv[sv] > 0 && !mbar_wait_bounded(bar(kDqEmptyV + sv), (nv[sv] - 1) & 1, budget, abort_flag)) {
+          ok = false;
+          break;
         }
-        issued[s] = t / 2 + 1;
+        mbar_arrive_expect_tx(bar(kDqFullV + sv), C::kTile);
+        for (int hh = 0; hh < C::kHalves; ++hh)
+          tma_load_3d(sbase + Q::kVOff + sv * C::kTile + hh * kBox, &tm_v, bar(kDqFullV + sv), hh * 64, jt * kT, zkv);
+        ++nv[sv];
       }
       if (!ok) bwd_abort(abort_flag, p.status);
+      // every issued copy has landed before the CTA can exit
       volatile int never = 0;
-      mbar_wait_bounded(bar(kBbKV), 0, kDrainBudgetCycles, &never);
-      for (int s = 0; s < 2; ++s)
-        if (issued[s] > 0) mbar_wait_bounded(bar(kBbFull + s), (issued[s] - 1) & 1, kDrainBudgetCycles, &never);
+      mbar_wait_bounded(bar(kDqQ), 0, kDrainBudgetCycles, &never);
+      for (int s = 0; s < Q::kKStages; ++s)
+        if (nk[s] > 0) mbar_wait_bounded(bar(kDqFullK + s), (nk[s] - 1) & 1, kDrainBudgetCycles, &never);
+      for (int s = 0; s < Q::kVStages; ++s)
+        if (nv[s] > 0) mbar_wait_bounded(bar(kDqFullV + s), (nv[s] - 1) & 1, kDrainBudgetCycles, &never);
     }
   } else if (warp == kBwdMmaWarp) {
     // ------------------------------------------------------------ MMA issuer (whole warp)
-    const uint64_t dq = desc_sw128(sbase + C::kKOff, 16, 1024);
-    const uint64_t ddo = desc_sw128(sbase + C::kVOff, 16, 1024);
+    const uint64_t dq = desc_sw128(sbase + Q::kQOff, 16, 1024);
+    const uint64_t ddo = desc_sw128(sbase + Q::kDoOff, 16, 1024);
     constexpr uint32_t kIdS = idesc_bwd(kT, kT, 0, 0);   // S = Q K^T, dP = dO V^T
     constexpr uint32_t kIdAcc = idesc_bwd(kT, D, 0, 1);  // dQ += dS K (K as an MN-major B)
     // Two S buffers (columns kColS and kColS2): S of key tile t + 1 is computed
     // while the dS warps work on tile t; dP has one buffer, refilled once they
-    // are done with it.
+    // have loaded it.
     auto col_s = [&](int t) -> uint32_t { return (t & 1) ? C::kColS2 : C::kColS; };
-    auto stage = [&](int t) -> uint32_t { return sbase + C::kQOff + (t & 1) * C::kStageBytes; };
+    auto k_at = [&](int t) -> uint32_t { return sbase + Q::kKOff + (t % Q::kKStages) * C::kTile; };
+    auto v_at = [&](int t) -> uint32_t { return sbase + Q::kVOff + (t % Q::kVStages) * C::kTile; };
     auto wait = [&](uint32_t b_, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait_bounded(b_, parity, budget, abort_flag));
     };
-    auto wait_stage = [&](int t) -> bool {
-      if (!wait(bar(kBbFull + (t & 1)), (t >> 1) & 1)) return false;
+    auto wait_k = [&](int t) -> bool {
+      if (!wait(bar(kDqFullK + t % Q::kKStages), (t / Q::kKStages) & 1)) return false;
       tc_fence_after();
       return true;
     };
-    bool ok = wait(bar(kBbKV), 0) && wait_stage(0);
+    auto wait_v = [&](int t) -> bool {
+      if (!wait(bar(kDqFullV + t % Q::kVStages), (t / Q::kVStages) & 1)) return false;
+      tc_fence_after();
+      return true;
+    };
+    // dP of key tile t, then release its V stage
+    auto issue_dp = [&](int t) {
+      mma_kmajor<D>(tmem + C::kColDP, ddo, desc_sw128(v_at(t), 16, 1024), kIdS);
+      tc_commit_w(bar(kDqEmptyV + t % Q::kVStages));
+      tc_commit_w(bar(kDqS));
+    };
+    bool ok = wait(bar(kDqQ), 0) && wait_k(0) && wait_v(0);
     if (ok) {
-      mma_kmajor<D>(tmem + col_s(0), dq, desc_sw128(stage(0), 16, 1024), kIdS);
-      mma_kmajor<D>(tmem + C::kColDP, ddo, desc_sw128(stage(0) + C::kTile, 16, 1024), kIdS);
-      tc_commit_w(bar(kBbS));
+      mma_kmajor<D>(tmem + col_s(0), dq, desc_sw128(k_at(0), 16, 1024), kIdS);
+      issue_dp(0);
     }
     for (int t = 0; t < iters && ok; ++t) {
       const bool next = t + 1 < iters;
       // S of the next key tile into the other buffer (its previous dS was consumed by
       // the dQ MMA issued in the last iteration, in order)
       if (next) {
-        if (!wait_stage(t + 1)) {
+        if (!wait_k(t + 1)) {
           ok = false;
           break;
         }
-        mma_kmajor<D>(tmem + col_s(t + 1), dq, desc_sw128(stage(t + 1), 16, 1024), kIdS);
+        mma_kmajor<D>(tmem + col_s(t + 1), dq, desc_sw128(k_at(t + 1), 16, 1024), kIdS);
       }
       if (next) {  // dP of the next key tile, as soon as the dS warps have loaded this one
-        if (!wait(bar(kBbDPFree), t & 1)) {
+        if (!wait(bar(kDqDPFree), t & 1) || !wait_v(t + 1)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        mma_kmajor<D>(tmem + C::kColDP, ddo, desc_sw128(stage(t + 1) + C::kTile, 16, 1024), kIdS);
-        tc_commit_w(bar(kBbS));
+        issue_dp(t + 1);
       }
-      if (!wait(bar(kBbP), t & 1)) {
+      if (!wait(bar(kDqP), t & 1)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      mma_tmem_a(tmem + C::kColAcc0, tmem + col_s(t), desc_sw128(stage(t), kBox, 1024), kIdAcc, t == 0);
-      tc_commit_w(bar(kBbEmpty + (t & 1)));
+      mma_tmem_a(tmem + C::kColAcc0, tmem + col_s(t), desc_sw128(k_at(t), kBox, 1024), kIdAcc, t == 0);
+      tc_commit_w(bar(kDqEmptyK + t % Q::kKStages));
     }
     if (!ok && lane == 0) bwd_abort(abort_flag, p.status);
-    tc_commit_w(bar(kBbAcc));
-    tc_commit_w(bar(kBbDrain));
+    tc_commit_w(bar(kDqAcc));
+    tc_commit_w(bar(kDqDrain));
     volatile int never = 0;
-    mbar_wait_bounded(bar(kBbDrain), 0, kDrainBudgetCycles, &never);
+    mbar_wait_bounded(bar(kDqDrain), 0, kDrainBudgetCycles, &never);
     __syncwarp();
   } else {
     // ------------------------------------------------------------ dS warps 0-7
@@ -629,7 +679,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int t = 0; t < iters; ++t) {
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbS), t & 1, budget, abort_flag));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kDqS), t & 1, budget, abort_flag));
       if (!ok) break;
       tc_fence_after();
       const int jt = klo + t;
@@ -644,7 +694,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBbDPFree));
+      if (lane == 0) mbar_arrive(bar(kDqDPFree));
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         const int c = 2 * ch + cc;  // 32-column chunk of the tile
@@ -672,10 +722,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBbP));
+      if (lane == 0) mbar_arrive(bar(kDqP));
     }
     // ------------------------------------------------------------ epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBbAcc), 0, budget, abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kDqAcc), 0, budget, abort_flag));
     if (!ok) bwd_abort(abort_flag, p.status);
     tc_fence_after();
     // TMEM loads are warp-collective: every lane runs them, only rows < N are stored
@@ -752,13 +802,13 @@ int launch_backward_t(const void* q, const void* k, const void* v, const void* o
   const size_t rows = static_cast<size_t>(B) * Hq * p.npad;
   bwd_rowdot_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  constexpr int smem = BwdCfg<D>::kAlloc;
-  if (cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-      cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  constexpr int smem_dkdv = BwdCfg<D>::kAlloc, smem_dq = DqCfg<D>::kAlloc;
+  if (cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dkdv) != cudaSuccess ||
+      cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dq) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  bwd_dkdv_kernel<D><<<dim3(p.ntiles, Hkv, B), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
+  bwd_dkdv_kernel<D><<<dim3(p.ntiles, Hkv, B), kBwdThreads, smem_dkdv, stream>>>(tq, tk, tv, tdo, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  bwd_dq_kernel<D><<<dim3(p.ntiles, Hq, B), kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
+  bwd_dq_kernel<D><<<dim3(p.ntiles, Hq, B), kBwdThreads, smem_dq, stream>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
