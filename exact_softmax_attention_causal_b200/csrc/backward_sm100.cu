@@ -46,6 +46,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 
@@ -74,6 +75,7 @@ struct BwdParams {
   __nv_bfloat16* dv;  // [B, Hkv, N, d]
   int32_t* status;
   int B, Hq, Hkv, N, group, mask_kind, window, ntiles, npad;
+  int chunk_kv, chunk_q;  // heads per scheduling chunk (dK/dV kernel: batch x K/V head; dQ: batch x query head)
   float scale, scale_log2;
   long long budget;
 };
@@ -88,6 +90,20 @@ __device__ __forceinline__ bool bwd_visible(const BwdParams& p, int qpos, int kp
   if (p.mask_kind == ATTN_MASK_FULL) return true;
   if (kpos > qpos) return false;
   return p.mask_kind != ATTN_MASK_SLIDING_WINDOW || qpos - kpos < p.window;
+}
+
+// Block order of both tile kernels: the (head, tile) blocks are taken in chunks of `chunk`
+// heads whose shared operands fit in L2 together; inside a chunk the tile of rank 0 (the one
+// with the most work under a causal or window mask) comes first for every head, then rank 1, ...
+// Blocks are dispatched roughly in index order, so the longest run first (less idle time at the
+// end) while the blocks in flight read the tiles of a few heads only.
+__device__ __forceinline__ void block_order(int x, int units, int ntiles, int chunk, int& unit, int& rank) {
+  const int per_chunk = chunk * ntiles;
+  const int c = x / per_chunk;
+  const int within = x - c * per_chunk;
+  const int n = min(chunk, units - c * chunk);  // heads in this (possibly last, shorter) chunk
+  rank = within / n;
+  unit = c * chunk + (within - rank * n);
 }
 
 // Query tiles [lo, hi] that see key tile j, and key tiles that query tile i sees.
@@ -238,11 +254,15 @@ enum : int {
   kDqFullV = 7,             // + stage (2)
   kDqEmptyV = 9,            // + stage (2)
   kDqS = 11,                // S and dP of the current key tile are in TMEM
-  kDqP = 12,                // dS written back (8 arrivals)
-  kDqAcc = 13,
-  kDqDrain = 14,
-  kDqDPFree = 15,           // the dS warps have loaded dP (8 arrivals)
+  kDqP = 12,                // dS of key tile t written back (8 arrivals), + t % 2 (2)
+  kDqAcc = 14,
+  kDqDrain = 15,
+  kDqDPFree = 16,           // the dS warps have loaded dP (8 arrivals)
 };
+// kDqP alternates between two barriers: the MMA warp issues dP(t + 1), which lets the dS
+// warps go on to key tile t + 1, before it waits for dS(t); on one barrier they could
+// complete the phases of t and t + 1 before that wait looks, and the wait would then see
+// the phase parity of t again and never return.
 constexpr int kDqTmemSlot = 192;
 constexpr int kDqAbort = 196;
 
@@ -259,7 +279,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (sbase - raw_u32);
-  const int j = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  // key tile j sees the query tiles j, j + 1, ... under a causal or window mask: rank j
+  int unit, j;
+  block_order(static_cast<int>(blockIdx.x), p.B * p.Hkv, p.ntiles, p.chunk_kv, unit, j);
+  const int kvh = unit % p.Hkv, b = unit / p.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int qlo, qhi;
   q_tiles_of_key_tile(p, j, qlo, qhi);
@@ -515,9 +538,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t sbase = (raw_u32 + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (sbase - raw_u32);
-  // with a causal or window mask the last query tiles see the most keys: launch them first
-  const int i = (p.mask_kind == ATTN_MASK_FULL) ? blockIdx.x : p.ntiles - 1 - blockIdx.x;
-  const int h = blockIdx.y, b = blockIdx.z;
+  // with a causal or window mask the last query tiles see the most keys: rank 0 is the last tile
+  int unit, rank;
+  block_order(static_cast<int>(blockIdx.x), p.B * p.Hq, p.ntiles, p.chunk_q, unit, rank);
+  const int i = (p.mask_kind == ATTN_MASK_FULL) ? rank : p.ntiles - 1 - rank;
+  const int h = unit % p.Hq, b = unit / p.Hq;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int klo, khi;
   k_tiles_of_q_tile(p, i, klo, khi);
@@ -539,7 +564,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(kDqEmptyV + s), 1);
     }
     mbar_init(bar(kDqS), 1);
-    mbar_init(bar(kDqP), kBwdSoftWarps);
+    for (int s = 0; s < 2; ++s) mbar_init(bar(kDqP + s), kBwdSoftWarps);
     mbar_init(bar(kDqAcc), 1);
     mbar_init(bar(kDqDrain), 1);
     mbar_init(bar(kDqDPFree), kBwdSoftWarps);
@@ -652,7 +677,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         issue_dp(t + 1);
       }
-      if (!wait(bar(kDqP), t & 1)) {
+      if (!wait(bar(kDqP + (t & 1)), (t >> 1) & 1)) {
         ok = false;
         break;
       }
@@ -687,10 +712,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool full_tile = (p.mask_kind == ATTN_MASK_FULL || (i > jt && (p.mask_kind == ATTN_MASK_CAUSAL ||
                                                                            (i * kT + kT - 1) - jt * kT < p.window))) &&
                              (i * kT + kT <= p.N) && (jt * kT + kT <= p.N);
-      // both chunks of dP first: once they are in registers the MMA warp may refill dP
-      uint32_t dpa[2][32];
+      // both chunks of dP and S at once: once dP is in registers the MMA warp may refill it
+      uint32_t dpa[2][32], sva[2][32];
       tmem_ld_32x32b_x32(lane_base + C::kColDP + 32u * (2 * ch), dpa[0]);
       tmem_ld_32x32b_x32(lane_base + C::kColDP + 32u * (2 * ch + 1), dpa[1]);
+      tmem_ld_32x32b_x32(lane_base + colS + 32u * (2 * ch), sva[0]);
+      tmem_ld_32x32b_x32(lane_base + colS + 32u * (2 * ch + 1), sva[1]);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -698,10 +725,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         const int c = 2 * ch + cc;  // 32-column chunk of the tile
-        uint32_t sv[32];
+        uint32_t* sv = sva[cc];
         const uint32_t* dpv = dpa[cc];
-        tmem_ld_32x32b_x32(lane_base + colS + 32u * c, sv);
-        tc_wait_ld();
         if (!full_tile) {
           // hidden (query, key) entries: a score of -inf makes P exactly 0 (scale_log2 > 0)
 #pragma unroll
@@ -710,19 +735,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!(qpos < p.N && kpos < p.N && bwd_visible(p, qpos, kpos))) sv[e] = __float_as_uint(-INFINITY);
           }
         }
+        // paired fp32 instructions, rounded as their scalar forms: P = 2^(s scale log2 e - LSE2),
+        // dS = P (dP - D)
+        const float2 sl2v = make_float2(sl2, sl2), nl2v = make_float2(-l2, -l2), ndr = make_float2(-dr, -dr);
         uint32_t dsk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const float p0 = exp2_approx(fmaf(__uint_as_float(sv[e]), sl2, -l2));
-          const float p1 = exp2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -l2));
-          dsk[e >> 1] = pack_bf16x2(p0 * (__uint_as_float(dpv[e]) - dr), p1 * (__uint_as_float(dpv[e + 1]) - dr));
+          const float2 x = ffma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2v, nl2v);
+          const float2 pr = make_float2(exp2_approx(x.x), exp2_approx(x.y));
+          const float2 ds = fmul2(pr, fadd2(make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])), ndr));
+          dsk[e >> 1] = pack_bf16x2(ds.x, ds.y);
         }
         tmem_st_32x32b_x16(lane_base + colS + 64u * ch + 16u * cc, dsk);  // dS as bf16 pairs, own half
       }
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kDqP));
+      if (lane == 0) mbar_arrive(bar(kDqP + (t & 1)));
     }
     // ------------------------------------------------------------ epilogue
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kDqAcc), 0, budget, abort_flag));
@@ -799,6 +828,18 @@ int launch_backward_t(const void* q, const void* k, const void* v, const void* o
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
   p.budget = wait_budget_cycles();
+  // Scheduling chunks of the dK/dV kernel: the K/V heads are split into as few equal chunks as
+  // keep the Q and dO tiles that a chunk's blocks read (its query heads' rows; under a window
+  // mask only the window's span of the sequence) within about 96 MB of L2. Its blocks differ
+  // most in size (key tile 0 of a causal mask reads every query tile), so the longest first
+  // pays; for the dQ kernel one head at a time (chunks of 1) measured as fast as any chunking.
+  const int span = (mask_kind == ATTN_MASK_SLIDING_WINDOW) ? std::min(N, window + kT) : N;
+  const double head_bytes = static_cast<double>(span) * D * 2, budget_bytes = 96.0 * 1024 * 1024;
+  const int units_kv = B * Hkv;
+  const double chunks = std::min(static_cast<double>(units_kv),
+                                 std::max(1.0, std::ceil(units_kv * 2.0 * p.group * head_bytes / budget_bytes)));
+  p.chunk_kv = std::max(1, static_cast<int>(std::ceil(units_kv / chunks)));
+  p.chunk_q = 1;
   const size_t rows = static_cast<size_t>(B) * Hq * p.npad;
   bwd_rowdot_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
@@ -806,9 +847,9 @@ int launch_backward_t(const void* q, const void* k, const void* v, const void* o
   if (cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dkdv) != cudaSuccess ||
       cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dq) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  bwd_dkdv_kernel<D><<<dim3(p.ntiles, Hkv, B), kBwdThreads, smem_dkdv, stream>>>(tq, tk, tv, tdo, p);
+  bwd_dkdv_kernel<D><<<B * Hkv * p.ntiles, kBwdThreads, smem_dkdv, stream>>>(tq, tk, tv, tdo, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  bwd_dq_kernel<D><<<dim3(p.ntiles, Hq, B), kBwdThreads, smem_dq, stream>>>(tq, tk, tv, tdo, p);
+  bwd_dq_kernel<D><<<B * Hq * p.ntiles, kBwdThreads, smem_dq, stream>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

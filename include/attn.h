@@ -281,6 +281,11 @@ ATTN_API size_t attn_prefill_backward_workspace_bytes(int B, int Hq, int N);
  *                bytes, 16-byte aligned
  *   status       device int32 or NULL (bounded-wait expiry: NaN outputs and
  *                ATTN_STATUS_BIT_TIMEOUT)
+ *
+ * Errors: ATTN_ERR_INVALID_ARG for NULL or misaligned tensors, non-positive
+ * sizes, Hq % Hkv != 0, a bad mask or scale; ATTN_ERR_UNSUPPORTED for d other
+ * than 64 or 128, B or Hq above 65535, or B * Hq * N of 2^31 or more;
+ * ATTN_ERR_WORKSPACE for a missing or short workspace.
  */
 ATTN_API int attn_prefill_backward(const void* q, const void* k, const void* v, const void* o, const void* d_o,
                                    const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
