@@ -25,7 +25,8 @@
 //                      tensor cores run the other's products.
 //   bwd_dq_kernel      one CTA per (batch, query head, 128-row query tile):
 //                      S = Q K^T and dP = dO V^T per key tile, dS (bf16) over
-//                      S, then dQ += dS K. S is double-buffered and dP is
+//                      S, then dQ += dS K. K and V stream through rings of
+//                      three and two stages; S is double-buffered and dP is
 //                      released as soon as the dS warps have loaded it, so
 //                      the next tile's scores are ready when they finish.
 // Each recomputes S once more than a single fused kernel would (seven

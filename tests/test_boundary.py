@@ -171,6 +171,14 @@ def _bwd(**kw):
     (dict(d=96), _lib.ATTN_ERR_UNSUPPORTED),
     (dict(ws=NULL), _lib.ATTN_ERR_WORKSPACE),
     (dict(wsb=100), _lib.ATTN_ERR_WORKSPACE),
+    (dict(B=0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(N=-1), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(mask=7), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(scale=0.0), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), _lib.ATTN_ERR_INVALID_ARG),
+    (dict(B=70000), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(Hq=70000, Hkv=2), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(B=1, Hq=4, N=1 << 29), _lib.ATTN_ERR_UNSUPPORTED),  # B * Hq * N = 2^31
 ])
 def test_backward_rejects_bad_arguments(kw, code):
     assert _bwd(**kw) == code
