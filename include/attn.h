@@ -140,6 +140,12 @@ ATTN_API int attn_prefill(const void* q, const void* k, const void* v, void* o, 
  * the pool is never dereferenced: that sequence's rows of o and lse are NaN
  * and ATTN_STATUS_BIT_DEVICE_CHECK is OR-ed into *status. With seq_lens[b] ==
  * Nq for every b and a contiguous block table this equals attn_prefill.
+ *
+ * Errors (nothing is launched): ATTN_ERR_INVALID_ARG for NULL or misaligned
+ * pointers, non-positive sizes, max_seq_len < Nq, Hq % Hkv != 0,
+ * max_blocks_per_seq * block_size < max_seq_len, a bad mask, window or scale;
+ * ATTN_ERR_UNSUPPORTED for d other than 64 or 128, another block_size, or
+ * B * Hq * Nq of 2^31 or more; ATTN_ERR_CUDA when a launch fails.
  */
 ATTN_API int attn_prefill_paged(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
                                 const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int d,
@@ -194,6 +200,14 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int m
  * A referenced block-table entry outside [0, num_blocks) or a seq_len outside
  * [1, max_seq_len] is never dereferenced: the affected rows of o and lse are
  * NaN and ATTN_STATUS_BIT_DEVICE_CHECK is OR-ed into *status.
+ *
+ * Errors (nothing is launched): ATTN_ERR_INVALID_ARG for NULL or misaligned
+ * pointers, non-positive sizes, Hq % Hkv != 0, max_blocks_per_seq *
+ * block_size < max_seq_len or a non-positive or non-finite scale;
+ * ATTN_ERR_UNSUPPORTED for d other than 64 or 128, block_size not a multiple
+ * of 16, B above 65535 or Hkv * ceil(Hq / Hkv / 16) above 65535;
+ * ATTN_ERR_WORKSPACE for a missing, misaligned or short workspace;
+ * ATTN_ERR_CUDA when the device query or the launch fails.
  */
 ATTN_API int attn_decode_paged(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
                       const int32_t* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int d,
@@ -243,6 +257,10 @@ ATTN_API size_t attn_decode_window_workspace_bytes(int B, int Hq, int Hkv, int d
  * cache may leave the entries of evicted middle blocks as -1. Out-of-range
  * entries that are read, and seq_lens outside [1, max_seq_len], are handled
  * as in attn_decode_paged.
+ *
+ * Errors: those of attn_decode_paged, plus ATTN_ERR_INVALID_ARG for window < 0,
+ * n_sink < 0, n_sink > max_seq_len, n_sink > 0 with window == 0, or a
+ * misaligned sinks pointer.
  */
 ATTN_API int attn_decode_paged_window(const void* q, const void* k_cache, const void* v_cache,
                                       const int32_t* block_table, const int32_t* seq_lens, const float* sinks, void* o,
@@ -329,6 +347,13 @@ ATTN_API size_t attn_mla_decode_workspace_bytes(int B, int H, int d_latent, int 
  *
  * Bad referenced table entries and seq_lens are handled as in
  * attn_decode_paged (NaN rows, ATTN_STATUS_BIT_DEVICE_CHECK).
+ *
+ * Errors (nothing is launched): ATTN_ERR_INVALID_ARG for NULL or misaligned
+ * pointers, non-positive sizes, max_blocks_per_seq * block_size < max_seq_len
+ * or a non-positive or non-finite scale; ATTN_ERR_UNSUPPORTED for other
+ * widths or block sizes, or B above 65535; ATTN_ERR_WORKSPACE for a missing,
+ * misaligned or short workspace; ATTN_ERR_CUDA when the device query or a
+ * launch fails.
  */
 ATTN_API int attn_mla_decode_paged(const void* q, const void* cache, const int32_t* block_table,
                                    const int32_t* seq_lens, void* o, float* lse, int B, int H, int d_latent,
@@ -347,6 +372,11 @@ ATTN_API int attn_mla_decode_paged(const void* q, const void* cache, const int32
  *   block_table, seq_lens as for attn_decode_paged (seq_lens[b] may be 0 here).
  * Invalid referenced entries: that token's row is NaN and the device-check
  * bit is set.
+ *
+ * Errors (nothing is launched): ATTN_ERR_INVALID_ARG for NULL or misaligned
+ * pointers, non-positive sizes or max_blocks_per_seq * block_size <
+ * max_seq_len; ATTN_ERR_UNSUPPORTED for d not a multiple of 8; ATTN_ERR_CUDA
+ * when the launch fails.
  */
 ATTN_API int attn_paged_gather(const void* cache, const int32_t* block_table, const int32_t* seq_lens, void* out, int B,
                       int Hkv, int d, int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len,
