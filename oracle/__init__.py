@@ -8,7 +8,7 @@ imports, calls or links anything here, and nothing here imports the product
 path: the two share no code.
 
 Every function cites the passage of the source pages it follows. All of them
-are pinned by ``tests/test_oracle_pins.py`` against values and identities the
+are pinned by ``tests/test_oracle_pins*.py`` against values and identities the
 pages and the mathematics fix; none is "parity unpinned".
 """
 
