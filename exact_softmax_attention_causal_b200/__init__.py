@@ -56,6 +56,24 @@ def _need(t: torch.Tensor, name: str, dtype, ndim: int) -> None:
         raise ValueError(f"{name} must be contiguous")
 
 
+def _need_out(t, name: str, dtype, shape) -> None:
+    """A caller-provided output must be a contiguous CUDA tensor of the exact
+    dtype and shape: the library writes shape-many elements at its address."""
+    _need(t, name, dtype, len(shape))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _need_buf(t, name: str) -> None:
+    """Workspace / status buffers: contiguous CUDA memory (any dtype)."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if name == "status" and (t.dtype != torch.int32 or t.numel() < 1):
+        raise TypeError("status must be an int32 CUDA tensor with at least one element")
+
+
 def prefill(q, k, v, mask: str = "causal", window: int = 0, scale: float | None = None, out=None, lse=None,
             status=None, stream=None, return_lse: bool = True):
     """O = softmax(scale * Q K^T + M) V for every query row; returns (O, LSE).
@@ -77,8 +95,12 @@ def prefill(q, k, v, mask: str = "causal", window: int = 0, scale: float | None 
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
+    _need_out(out, "out", torch.bfloat16, q.shape)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need_out(lse, "lse", torch.float32, (B, Hq, N))
+    _need_buf(status, "status")
     rc = _lib.lib().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d, MASKS[mask],
                                  int(window), float(scale), _ptr(status), _stream_handle(stream))
     _lib.check(rc, "attn_prefill")
@@ -112,8 +134,13 @@ def prefill_backward(q, k, v, o, lse, d_o, mask: str = "causal", window: int = 0
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    _need_out(dq, "dq", torch.bfloat16, q.shape)
+    _need_out(dk, "dk", torch.bfloat16, k.shape)
+    _need_out(dv, "dv", torch.bfloat16, v.shape)
     if workspace is None:
         workspace = torch.empty(prefill_backward_workspace_bytes(B, Hq, N), dtype=torch.uint8, device=q.device)
+    _need_buf(workspace, "workspace")
+    _need_buf(status, "status")
     rc = _lib.lib().attn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(d_o), _ptr(lse), _ptr(dq), _ptr(dk),
                                           _ptr(dv), B, Hq, Hkv, N, d, MASKS[mask], int(window), float(scale),
                                           _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
@@ -149,8 +176,12 @@ def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int, 
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
+    _need_out(out, "out", torch.bfloat16, q.shape)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need_out(lse, "lse", torch.float32, (B, Hq, Nq))
+    _need_buf(status, "status")
     rc = _lib.lib().attn_prefill_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
                                        _ptr(out), _ptr(lse), B, Hq, Hkv, Nq, d, num_blocks, block_size,
                                        block_table.shape[1], int(max_seq_len), MASKS[mask], int(window),
@@ -197,10 +228,15 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, max_seq_len: int, s
     if workspace is None:
         nbytes = decode_workspace_bytes(B, Hq, Hkv, d, max_seq_len, block_size)
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _need_buf(workspace, "workspace")
     if out is None:
         out = torch.empty_like(q)
+    _need_out(out, "out", torch.bfloat16, q.shape)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need_out(lse, "lse", torch.float32, (B, Hq))
+    _need_buf(status, "status")
     rc = _lib.lib().attn_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
                                       _ptr(out), _ptr(lse), B, Hq, Hkv, d, num_blocks, block_size,
                                       block_table.shape[1], int(max_seq_len), float(scale), _ptr(workspace),
@@ -246,10 +282,15 @@ def decode_paged_window(q, k_cache, v_cache, block_table, seq_lens, max_seq_len:
     if workspace is None:
         nbytes = decode_window_workspace_bytes(B, Hq, Hkv, d, max_seq_len, block_size, int(window), int(n_sink))
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _need_buf(workspace, "workspace")
     if out is None:
         out = torch.empty_like(q)
+    _need_out(out, "out", torch.bfloat16, q.shape)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need_out(lse, "lse", torch.float32, (B, Hq))
+    _need_buf(status, "status")
     rc = _lib.lib().attn_decode_paged_window(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
                                              _ptr(seq_lens), _ptr(sinks), _ptr(out), _ptr(lse), B, Hq, Hkv, d,
                                              num_blocks, block_size, block_table.shape[1], int(max_seq_len),
@@ -289,10 +330,15 @@ def mla_decode_paged(q, cache, block_table, seq_lens, max_seq_len: int, scale: f
     if workspace is None:
         workspace = torch.empty(mla_decode_workspace_bytes(B, H, max_seq_len, d_latent, d_rope), dtype=torch.uint8,
                                 device=q.device)
+    _need_buf(workspace, "workspace")
     if out is None:
         out = torch.empty((B, H, d_latent), dtype=torch.bfloat16, device=q.device)
+    _need_out(out, "out", torch.bfloat16, (B, H, d_latent))
     if lse is None and return_lse:
         lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need_out(lse, "lse", torch.float32, (B, H))
+    _need_buf(status, "status")
     rc = _lib.lib().attn_mla_decode_paged(_ptr(q), _ptr(cache), _ptr(block_table), _ptr(seq_lens), _ptr(out), _ptr(lse),
                                           B, H, d_latent, d_rope, num_blocks, block_size, block_table.shape[1],
                                           int(max_seq_len), float(scale), _ptr(workspace),
@@ -311,6 +357,8 @@ def paged_gather(cache, block_table, seq_lens, max_seq_len: int, out=None, statu
     B = block_table.shape[0]
     if out is None:
         out = torch.empty((B, Hkv, max_seq_len, d), dtype=cache.dtype, device=cache.device)
+    _need_out(out, "out", torch.bfloat16, (B, Hkv, max_seq_len, d))
+    _need_buf(status, "status")
     rc = _lib.lib().attn_paged_gather(_ptr(cache), _ptr(block_table), _ptr(seq_lens), _ptr(out), B, Hkv, d,
                                       num_blocks, block_size, block_table.shape[1], int(max_seq_len), _ptr(status),
                                       _stream_handle(stream))

@@ -401,7 +401,10 @@ ATTN_API int attn_paged_gather(const void* cache, const int32_t* block_table, co
  *     before anything is launched.
  *   - The first call on each device looks up that device's address of the
  *     array (a set-up step, done once per device with the device current);
- *     make that first call before any stream capture.
+ *     make that first call before any stream capture. The address is kept
+ *     for the life of the process: after cudaDeviceReset (or any teardown of
+ *     the device's primary context) it is stale, so do not call this entry
+ *     point on that device again in the same process.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind. Nothing in it has to start at zero: each call writes every
  *     partial it later reads. Calls whose kernels overlap on the GPU (two
