@@ -66,7 +66,7 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks and throttle reasons sampled every 25 ms while running."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -81,7 +81,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "25"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -162,6 +162,17 @@ def oracle_threads() -> int:
         pass
     return len(os.sched_getaffinity(0))
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 # ----------------------------------------------------------------------------
 # the fp64 CPU oracle, timed on the host cores (cpu_baseline and --impl reference)
 # ----------------------------------------------------------------------------
@@ -189,11 +200,48 @@ def oracle_prefill_heads(x, cfg, heads, budget_s=None):
     return per_head * done, time.perf_counter() - t0, done
 
 
+def oracle_config_rate(op, cfg, x, budget_s):
+    """The oracle on a bounded sample of one workload: evenly spaced query rows
+    of (batch, head) slices for a prefill (TFLOP/s over their visible pairs),
+    whole sequences' heads for a decode (GB/s of the K/V they read)."""
+    import oracle  # the oracle is only ever loaded by the baseline legs
+
+    t0 = time.perf_counter()
+    work, done = 0, []
+    if op == "prefill":
+        B, Hq, N, d = cfg["B"], cfg["Hq"], cfg["N"], cfg["d"]
+        kind = accounting.MASK_IDS[cfg["mask"]]
+        rows = list(range(0, N, max(1, N // 256)))
+        for i in range(B * Hq):
+            bh = (i * 37) % (B * Hq)
+            oracle.prefill_rows_ref(x.q, x.k, x.v, bh // Hq, bh % Hq, rows, kind, cfg["window"],
+                                    workloads.default_scale(d))
+            work += 4 * d * sum(accounting.row_visible_keys(N, i, cfg["mask"], cfg["window"]) for i in rows)
+            done.append(bh)
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        secs = time.perf_counter() - t0
+        return {"value": work / secs / 1e12, "unit": "TFLOP/s",
+                "sample": f"{len(rows)} evenly spaced rows of {len(done)} (batch, head) slices, {secs:.1f} s"}
+    Hq, Hkv, d = cfg["Hq"], cfg["Hkv"], cfg["d"]
+    for b in range(x.q.shape[0]):
+        oracle.decode_rows_ref(x.q, x.k_cache, x.v_cache, x.block_table, x.seq_lens, b, range(Hq),
+                               workloads.default_scale(d))
+        work += int(x.seq_lens[b]) * Hkv * d * 4
+        done.append(b)
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    secs = time.perf_counter() - t0
+    return {"value": work / secs / 1e9, "unit": "GB/s",
+            "sample": f"all {Hq} heads of {len(done)} sequence(s), {secs:.1f} s"}
+
+
 def cpu_baseline(x, cfg, budget_s):
     flops, secs, done = oracle_prefill_heads(x, cfg, heads=cfg["B"] * cfg["Hq"], budget_s=budget_s)
     return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+            "cpu_model": cpu_model(), "blas_threads": oracle_threads(),
             "sample": f"{done} of {cfg['B'] * cfg['Hq']} (batch, head) slices of the {cfg['name']} prefill, "
-                      f"all {cfg['N']} rows each, fp64 NumPy, {secs:.1f} s"}
+                      f"all {cfg['N']} rows each, fp64 NumPy (one process, BLAS-threaded matmuls), {secs:.1f} s"}
 
 
 def run_reference(args, cfg):
@@ -259,6 +307,8 @@ def run_ours(args, pcfg, dcfg):
                                        seq_lens=dcfg.get("seq_lens"), block_size=dcfg["block_size"], seed=seed)
     dq, kc, vc = xd.q.to(dev), xd.k_cache.to(dev), xd.v_cache.to(dev)
     bt, sl = xd.block_table.to(dev), xd.seq_lens.to(dev)
+    sl_dev = sl
+    xd_q_host, xd_bt_host, xd_sl_host = xd.q, xd.block_table, xd.seq_lens
     dout = torch.empty_like(dq)
     dlse = torch.empty((dB, dHq), dtype=torch.float32, device=dev)
     ws = torch.empty(attn.decode_workspace_bytes(dB, dHq, dHkv, dd, xd.max_seq_len, xd.block_size),
@@ -354,7 +404,59 @@ def run_ours(args, pcfg, dcfg):
     barrier()
     e2e_ms = e2e_ev[0].elapsed_time(e2e_ev[1])
 
-    p_ms, d_ms, region_ms, e2e_ms = sharding.max_over_ranks([p_ms, d_ms, region_ms, e2e_ms], device=dev)
+    # The decode half end to end: every step copies its new query tokens, block
+    # table and context lengths in from pinned host memory, decodes against the
+    # cache already resident in HBM, and copies O and LSE back out.
+    hdq, hbt, hsl = (t.pin_memory() for t in (xd_q_host, xd_bt_host, xd_sl_host))
+    dh2d = sum(t.numel() * t.element_size() for t in (hdq, hbt, hsl))
+    hdo = torch.empty(dout.shape, dtype=dout.dtype, pin_memory=True)
+    hdl = torch.empty(dlse.shape, dtype=dlse.dtype, pin_memory=True)
+    dd2h = sum(t.numel() * t.element_size() for t in (hdo, hdl))
+    dq2, bt2, sl2 = torch.empty_like(dq), torch.empty_like(bt), torch.empty_like(sl_dev)
+    barrier()
+    de2e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    de2e_ev[0].record(main)
+    for _ in range(args.steps):
+        dq2.copy_(hdq, non_blocking=True)
+        bt2.copy_(hbt, non_blocking=True)
+        sl2.copy_(hsl, non_blocking=True)
+        attn.decode_paged(dq2, kc, vc, bt2, sl2, dcfg_max_len(dcfg), out=dout, lse=dlse, workspace=ws)
+        hdo.copy_(dout, non_blocking=True)
+        hdl.copy_(dlse, non_blocking=True)
+    de2e_ev[1].record(main)
+    barrier()
+    de2e_ms = de2e_ev[0].elapsed_time(de2e_ev[1])
+
+    p_ms, d_ms, region_ms, e2e_ms, de2e_ms = sharding.max_over_ranks([p_ms, d_ms, region_ms, e2e_ms, de2e_ms],
+                                                                      device=dev)
+
+    # Every other configuration of the workload table, one entry point each,
+    # timed the same way (CUDA events around each launch, L2 flushed before it,
+    # max over ranks): the long-context causal and windowed prefills and the
+    # GQA dial (MHA / GQA-8 / MQA) prefills and single-sequence decodes.
+    del q, k, v, o, lse, dq, kc, vc, bt, dout, dlse, ws, bufs, dq2, bt2, sl2
+    torch.cuda.empty_cache()
+    peaks_all = measured_peaks()
+    configs = []
+    cfg_host = {}
+    with ClockSampler(local) as clk_cfg:
+        for op_name, wname in () if args.no_configs else CONFIG_SWEEP:
+            op = setup_op(op_name, wname, dev, seed, peaks_all, keep_host=(rank == 0 and world == 1))
+            ms = time_launches(op["launch"], args.config_steps, 3, flush, dist_on=world > 1)
+            (ms_max,) = sharding.max_over_ranks([ms], device=dev)
+            per_launch_s = ms / args.config_steps / 1e3
+            achieved = op["work"] / per_launch_s / op["scale_div"]
+            configs.append({
+                "workload": wname, "op": op_name, "unit": op["unit"],
+                "value": sharding.job_throughput(op["work"], world, args.config_steps, ms_max) / op["scale_div"],
+                "ms_per_launch": ms_max / args.config_steps, "work_per_launch": op["work"],
+                "roofline": {"bound": op["bound"], "achieved": achieved, "peak": op["peak"], "unit": op["unit"],
+                             "frac": achieved / op["peak"], "kernel": op["kernel"]},
+            })
+            if "host" in op["extra"]:
+                cfg_host[wname] = (op_name, op["cfg"], op["extra"]["host"])
+            del op
+            torch.cuda.empty_cache()
 
     result = None
     if rank == 0:
@@ -388,8 +490,11 @@ def run_ours(args, pcfg, dcfg):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "schedule": "per step: Q, K, V in from pinned host memory, prefill, O and LSE out; "
                                 "consecutive steps overlap on copy-in, compute and copy-out streams"},
-            "gpu_launches": 3 * K,
+            "gpu_launches": 2 * K,
+            "gpu_launches_note": "timed step region: one prefill and one decode kernel per step; the end-to-end "
+                                 "legs launch 2 * steps more and the configuration sweep config_steps per entry",
             "clocks": clk.summary(),
+            "clocks_configs": clk_cfg.summary(),
             "decode": {
                 "metric": "paged-decode KV GB/s", "value": sharding.job_throughput(kv_bytes, world, K, d_ms) / 1e9,
                 "unit": "GB/s", "workload": dcfg["name"], "kv_bytes_per_step": kv_bytes, "ms_per_step": d_ms / K,
@@ -397,12 +502,24 @@ def run_ours(args, pcfg, dcfg):
                              "frac": d_gbs_launch / peaks["hbm_gbs"],
                              "traffic": recorded_traffic("decode_split_kernel", "decode_sm100.cu", kv_bytes),
                              "peak_source": f"hbm_gbs {tag}",
-                             "kernel": "decode_split_kernel<128> + decode_merge_kernel<128>"},
+                             "kernel": "decode_split_kernel<128> (split-KV with the merge in the same launch)"},
+                "e2e": {"value": sharding.job_throughput(kv_bytes, world, K, de2e_ms) / 1e9, "unit": "GB/s",
+                        "h2d_bytes_per_step": dh2d, "d2h_bytes_per_step": dd2h,
+                        "schedule": "per step: new query tokens, block table and context lengths in from pinned "
+                                    "host memory, decode against the HBM-resident cache, O and LSE out"},
             },
             "region_ms": region_ms,
         }
+        result["configs"] = configs
         if world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(xp, pcfg, args.cpu_seconds)
+            # the oracle on a bounded sample of each configuration as well
+            for c in configs:
+                if c["workload"] in cfg_host:
+                    op_name, cfg, host = cfg_host[c["workload"]]
+                    c["cpu_baseline"] = dict(oracle_config_rate(op_name, cfg, host, args.cpu_seconds_per_config),
+                                             kind="oracle", cores=oracle_threads())
+                    c["gpu_over_cpu"] = c["value"] / c["cpu_baseline"]["value"]
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -411,26 +528,32 @@ def run_ours(args, pcfg, dcfg):
     return 0
 
 
-def run_single_op(args):
-    """Time one entry point on one named workload; one JSON line with its roofline.
+# The configurations timed beside the headline step: long-context prefill
+# (causal and sliding window, N = 32,768), the GQA dial of prefill (B = 2,
+# N = 8,192) and of single-sequence decode (131,072 cached tokens).
+CONFIG_SWEEP = (("prefill", "long_causal_n32768"), ("prefill", "long_window4096_n32768"),
+                ("prefill", "gqa_dial_prefill_mha"), ("prefill", "gqa_dial_prefill_gqa8"),
+                ("prefill", "gqa_dial_prefill_mqa"), ("decode", "gqa_dial_decode_mha"),
+                ("decode", "gqa_dial_decode_gqa8"), ("decode", "gqa_dial_decode_mqa"))
+
+LAUNCHES_PER_CALL = {"prefill": 1, "prefill_paged": 1, "prefill_backward": 3, "mla_decode": 2, "decode": 1,
+                     "decode_window": 1}
+
+
+def setup_op(op, name, dev, seed, peaks, keep_host=False):
+    """Inputs on the device and a launch() closure for one entry point on one
+    named workload, with its algorithmic work per launch and its roofline.
 
     prefill (TFLOP/s, tensor roofline), prefill_paged (TFLOP/s over the visible
     pairs of each chunk against its context), decode (KV GB/s, HBM roofline),
     decode_window (GB/s of the K/V bytes of the visible tokens only), mla_decode
     (GB/s of the latent cache, with its tensor-core rate reported beside it),
     prefill_backward (TFLOP/s counting 5 products per visible pair).
-    L2 is flushed before every timed launch; CUDA events on the launching stream.
     """
     import exact_softmax_attention_causal_b200 as attn
 
-    world, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    seed = sharding.rank_seed(args.seed, rank)
-    peaks = measured_peaks()
-    tag = "of measured" if peaks["source"] == "measured" else "of fallback"
-    name = args.workload
-    if args.op == "prefill":
+    extra = {}
+    if op == "prefill":
         cfg = workloads.PREFILL_WORKLOADS[name]
         x = workloads.prefill_inputs(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["N"], cfg["d"], seed)
         q, k, v = x.q.to(dev), x.k.to(dev), x.v.to(dev)
@@ -442,11 +565,13 @@ def run_single_op(args):
             attn.prefill(q, k, v, mask=cfg["mask"], window=cfg["window"], out=o, lse=lse)
         unit, bound, peak, scale_div = "TFLOP/s", "tensor", peaks["bf16_tflops"], 1e12
         metric = "prefill TFLOP/s (visible pairs)"
-    elif args.op == "prefill_paged":
+        kernel = f"prefill_fwd_kernel<{cfg['d']}>"
+    elif op == "prefill_paged":
         cfg = dict(workloads.PAGED_PREFILL_WORKLOADS[name])
-        mask, window = cfg.pop("mask"), cfg.pop("window")
-        B, Hq, Hkv, Nq, d = (cfg.pop(kk) for kk in ("B", "Hq", "Hkv", "Nq", "d"))
-        x = workloads.paged_prefill_inputs(B, Hq, Hkv, Nq, d, seed=seed, **cfg)
+        c = dict(cfg)
+        mask, window = c.pop("mask"), c.pop("window")
+        B, Hq, Hkv, Nq, d = (c.pop(kk) for kk in ("B", "Hq", "Hkv", "Nq", "d"))
+        x = workloads.paged_prefill_inputs(B, Hq, Hkv, Nq, d, seed=seed, **c)
         q, kc, vc = x.q.to(dev), x.k_cache.to(dev), x.v_cache.to(dev)
         bt, sl = x.block_table.to(dev), x.seq_lens.to(dev)
         o = torch.empty_like(q)
@@ -458,8 +583,8 @@ def run_single_op(args):
             attn.prefill_paged(q, kc, vc, bt, sl, msl, mask=mask, window=window, out=o, lse=lse)
         unit, bound, peak, scale_div = "TFLOP/s", "tensor", peaks["bf16_tflops"], 1e12
         metric = "chunked prefill TFLOP/s (visible pairs)"
-        cfg = dict(workloads.PAGED_PREFILL_WORKLOADS[name])
-    elif args.op == "decode_window":
+        kernel = f"prefill_fwd_kernel<{d}, paged>"
+    elif op == "decode_window":
         cfg = dict(workloads.WINDOW_DECODE_WORKLOADS[name])
         x = workloads.paged_decode_inputs(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"], len_range=cfg.get("len_range"),
                                           seq_lens=cfg.get("seq_lens"), block_size=cfg["block_size"], seed=seed,
@@ -480,7 +605,8 @@ def run_single_op(args):
                                      workspace=ws)
         unit, bound, peak, scale_div = "GB/s", "hbm", peaks["hbm_gbs"], 1e9
         metric = "windowed paged-decode KV GB/s (visible tokens)"
-    elif args.op == "prefill_backward":
+        kernel = f"decode_split_kernel<{cfg['d']}>"
+    elif op == "prefill_backward":
         cfg = workloads.PREFILL_WORKLOADS[name]
         x = workloads.prefill_inputs(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["N"], cfg["d"], seed)
         q, k, v = x.q.to(dev), x.k.to(dev), x.v.to(dev)
@@ -497,7 +623,8 @@ def run_single_op(args):
                                   workspace=ws)
         unit, bound, peak, scale_div = "TFLOP/s", "tensor", peaks["bf16_tflops"], 1e12
         metric = "attention backward TFLOP/s (5 products per visible pair)"
-    elif args.op == "mla_decode":
+        kernel = f"bwd_rowdot_kernel + bwd_dkdv_kernel<{cfg['d']}> + bwd_dq_kernel<{cfg['d']}>"
+    elif op == "mla_decode":
         cfg = dict(workloads.MLA_DECODE_WORKLOADS[name])
         x = workloads.mla_decode_inputs(cfg["B"], cfg["H"], cfg["d_latent"], cfg["d_rope"], len_range=cfg["len_range"],
                                         block_size=cfg["block_size"], seed=seed)
@@ -507,7 +634,8 @@ def run_single_op(args):
         ws = torch.empty(attn.mla_decode_workspace_bytes(cfg["B"], cfg["H"], x.max_seq_len), dtype=torch.uint8,
                          device=dev)
         work = accounting.mla_decode_bytes(x.seq_lens.tolist(), cfg["d_latent"], cfg["d_rope"])
-        mla_flops = accounting.mla_decode_flops(x.seq_lens.tolist(), cfg["H"], cfg["d_latent"], cfg["d_rope"])
+        extra["mla_flops"] = accounting.mla_decode_flops(x.seq_lens.tolist(), cfg["H"], cfg["d_latent"],
+                                                         cfg["d_rope"])
         msl = x.max_seq_len
         mla_scale = 1.0 / math.sqrt(cfg["d_head"] + cfg["d_rope"])
 
@@ -515,7 +643,8 @@ def run_single_op(args):
             attn.mla_decode_paged(q, cache, bt, sl, msl, mla_scale, out=o, lse=lse, workspace=ws)
         unit, bound, peak, scale_div = "GB/s", "hbm", peaks["hbm_gbs"], 1e9
         metric = "absorbed MLA decode latent-cache GB/s"
-    else:
+        kernel = "mla_split_kernel + decode_merge_kernel<512>"
+    elif op == "decode":
         cfg = dict(workloads.DECODE_WORKLOADS[name])
         x = workloads.paged_decode_inputs(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"], len_range=cfg.get("len_range"),
                                           seq_lens=cfg.get("seq_lens"), block_size=cfg["block_size"], seed=seed)
@@ -532,44 +661,74 @@ def run_single_op(args):
             attn.decode_paged(q, kc, vc, bt, sl, msl, out=o, lse=lse, workspace=ws)
         unit, bound, peak, scale_div = "GB/s", "hbm", peaks["hbm_gbs"], 1e9
         metric = "paged-decode KV GB/s"
+        kernel = f"decode_split_kernel<{cfg['d']}>"
+    else:
+        raise ValueError(op)
+    if keep_host:
+        extra["host"] = x
     del x
+    return dict(launch=launch, work=work, unit=unit, bound=bound, peak=peak, scale_div=scale_div, metric=metric,
+                cfg=cfg, kernel=kernel, extra=extra)
+
+
+def time_launches(launch, steps, warmup, flush, dist_on=False):
+    """CUDA-event time (ms, summed over `steps`) of launch(), each launch
+    preceded by an L2-flushing write outside the events."""
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for _ in range(warmup):
+        flush.fill_(1)
+        launch()
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for e0, e1 in events:
+        flush.fill_(1)
+        e0.record()
+        launch()
+        e1.record()
+    torch.cuda.synchronize()
+    return sum(e0.elapsed_time(e1) for e0, e1 in events)
+
+
+def run_single_op(args):
+    """Time one entry point on one named workload; one JSON line with its roofline.
+    L2 is flushed before every timed launch; CUDA events on the launching stream.
+    """
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    seed = sharding.rank_seed(args.seed, rank)
+    peaks = measured_peaks()
+    tag = "of measured" if peaks["source"] == "measured" else "of fallback"
+    name = args.workload
+    op = setup_op(args.op, name, dev, seed, peaks)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     with ClockSampler(local) as clk:
-        for _ in range(args.warmup):
-            flush.fill_(1)
-            launch()
-        torch.cuda.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
-        for e0, e1 in events:
-            flush.fill_(1)
-            e0.record()
-            launch()
-            e1.record()
-        torch.cuda.synchronize()
-    ms = sum(e0.elapsed_time(e1) for e0, e1 in events)
+        ms = time_launches(op["launch"], args.steps, args.warmup, flush, dist_on=world > 1)
     (ms_max,) = sharding.max_over_ranks([ms], device=dev)
-    achieved = work / (ms / args.steps / 1e3) / scale_div
+    achieved = op["work"] / (ms / args.steps / 1e3) / op["scale_div"]
     if rank == 0:
         line = {
-            "metric": metric, "value": sharding.job_throughput(work, world, args.steps, ms_max) / scale_div,
-            "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "metric": op["metric"],
+            "value": sharding.job_throughput(op["work"], world, args.steps, ms_max) / op["scale_div"],
+            "unit": op["unit"], "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic", "op": args.op,
-            "config": dict(workload=name, **{kk: vv for kk, vv in cfg.items()},
+            "config": dict(workload=name, **{kk: vv for kk, vv in op["cfg"].items()},
                            l2="flushed (256 MiB write) before every timed launch"),
-            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                         "traffic": None, "peak_source": tag},
-            "work_per_launch": work,
-            "gpu_launches": args.steps * {"prefill_backward": 3, "mla_decode": 2, "decode": 2,
-                                          "decode_window": 2}.get(args.op, 1),
+            "roofline": {"bound": op["bound"], "achieved": achieved, "peak": op["peak"], "unit": op["unit"],
+                         "frac": achieved / op["peak"], "traffic": None, "peak_source": tag,
+                         "kernel": op["kernel"]},
+            "work_per_launch": op["work"],
+            "gpu_launches": args.steps * LAUNCHES_PER_CALL[args.op],
             "clocks": clk.summary(),
         }
         if args.op == "mla_decode":  # the same launches against the tensor roofline, for context
-            tf = mla_flops / (ms / args.steps / 1e3) / 1e12
+            tf = op["extra"]["mla_flops"] / (ms / args.steps / 1e3) / 1e12
             line["tensor_context"] = {"achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                                      "frac": tf / peaks["bf16_tflops"], "flops_per_launch": mla_flops}
+                                      "frac": tf / peaks["bf16_tflops"],
+                                      "flops_per_launch": op["extra"]["mla_flops"]}
         print(json.dumps(line), flush=True)
     return 0
 
@@ -599,6 +758,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-heads", type=int, default=2, help="oracle (batch, head) slices per step")
+    ap.add_argument("--config-steps", type=int, default=20, help="timed launches per configuration of the sweep")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration sweep")
+    ap.add_argument("--cpu-seconds-per-config", type=float, default=3.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -26,6 +26,17 @@ def visible_pairs(n: int, mask: str, window: int = 0) -> int:
     raise ValueError(mask)
 
 
+def row_visible_keys(n: int, i: int, mask: str, window: int = 0) -> int:
+    """Keys visible to query row i of an n-row square prefill."""
+    if mask == "full":
+        return n
+    if mask == "causal":
+        return i + 1
+    if mask == "window":
+        return min(i + 1, int(window))
+    raise ValueError(mask)
+
+
 def prefill_flops(B: int, Hq: int, N: int, d: int, mask: str, window: int = 0) -> int:
     return 4 * B * Hq * d * visible_pairs(N, mask, window)
 

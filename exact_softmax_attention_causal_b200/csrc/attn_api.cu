@@ -84,8 +84,8 @@ int attn_prefill(const void* q, const void* k, const void* v, void* o, float* ls
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  // grid.y holds B, grid.z the query tiles; TMA coordinates are int32
-  if (B > 65535 || static_cast<long long>(B) * Hq * N > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
+  // TMA coordinates and the persistent kernel's item indices are int32
+  if (static_cast<long long>(B) * Hq * N > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
   if (mask_kind == ATTN_MASK_SLIDING_WINDOW && window >= N) mask_kind = ATTN_MASK_CAUSAL;
   return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, N, d, mask_kind, window, scale, status,
                         reinterpret_cast<cudaStream_t>(stream));
@@ -140,7 +140,7 @@ size_t decode_bytes(int B, int Hq, int Hkv, int d, int max_seq_len, int block_si
   if (current_sm_count(&sms) != ATTN_OK) return 0;
   DecodePlan plan;
   if (plan_decode(B, Hq, Hkv, decode_plan_length(max_seq_len, window, n_sink), sms, &plan) != ATTN_OK) return 0;
-  return decode_workspace_bytes(B, Hq, d, plan);
+  return decode_workspace_bytes(B, Hq, Hkv, d, plan);
 }
 
 int decode_common(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
@@ -171,7 +171,7 @@ int decode_common(const void* q, const void* k_cache, const void* v_cache, const
   DecodePlan plan;
   if (plan_decode(B, Hq, Hkv, decode_plan_length(max_seq_len, window, n_sink), sms, &plan) != ATTN_OK)
     return ATTN_ERR_INVALID_ARG;
-  if (!workspace || !aligned16(workspace) || workspace_bytes < decode_workspace_bytes(B, Hq, d, plan))
+  if (!workspace || !aligned16(workspace) || workspace_bytes < decode_workspace_bytes(B, Hq, Hkv, d, plan))
     return ATTN_ERR_WORKSPACE;
   const cudaError_t e = launch_decode(q, k_cache, v_cache, block_table, seq_lens, sinks, o, lse, B, Hq, Hkv, d,
                                       num_blocks, block_size, max_blocks_per_seq, max_seq_len, window, n_sink, scale,

@@ -16,8 +16,12 @@
 // group against them with mma.sync m16n8k16 (bf16 in, fp32 accumulate), and
 // keep FlashAttention's running (max, sum, output) per query head. The warps
 // combine in shared memory and write one normalised partial output and its
-// log-sum-exp per (sequence, head, chunk). The merge kernel combines the
-// chunks with the online softmax's rescaling.
+// log-sum-exp per (sequence, head, chunk). The CTA that finishes last among
+// the chunks of a (sequence, K/V head, head chunk) combines them with the
+// online softmax's rescaling and writes the output, in the same launch (a
+// ticket counter in the workspace tells each CTA whether it is the last).
+// Many chunks are combined in two levels: groups of chunks first, then the
+// groups.
 //
 // The kernel is HBM-bound: each K/V byte of a (sequence, K/V head) is read
 // once and shared by the whole query-head group.
@@ -36,6 +40,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -58,8 +64,12 @@ struct DecodeParams {
   const int32_t* seq_lens;
   float* o_part;    // [B, Hq, splits, D]
   float* lse_part;  // [B, Hq, splits]
-  // One split per sequence: the split kernel writes the final output itself
-  // (normalised, learned sink folded in) and no merge runs.
+  // Ticket counters, (1 + ngroups) per (sequence, K/V head, head chunk):
+  // [0] counts the merged groups, [1 + g] the finished chunks of group g.
+  unsigned long long* counters;
+  // Sequences whose visible sub-blocks fit one split are written directly by
+  // that split's CTA (normalised, learned sink folded in); the others by the
+  // CTA that merges their chunks.
   __nv_bfloat16* o;  // [B, Hq, D]
   float* lse;        // [B, Hq] or nullptr
   const float* sinks;
@@ -67,7 +77,9 @@ struct DecodeParams {
   int B, Hq, Hkv, group, hchunks;
   int num_blocks, block_size, max_blocks_per_seq, max_seq_len;
   int chunk, splits;
+  int group_slots, ngroups;  // chunks per first-level merge group; groups per row at most
   int window, n_sink;  // window 0: every cached token is visible (n_sink is then 0)
+  uint32_t token;      // this call's tag for the ticket counters (never 0)
   float scale_log2;  // scale * log2(e): scores live in the base-2 domain
 };
 
@@ -98,17 +110,31 @@ __device__ __forceinline__ void flag_status(int32_t* status, int bit) {
   if (status != nullptr) atomicOr(status, bit);
 }
 
-// Shared memory: Q tile [16][D] then, per warp, kStages x (K [16][D], V [16][D]).
+// Shared memory: Q tile [16][D], then per warp kStages x (K [16][D], V [16][D]),
+// then the split's block-table entries (one per listed sub-block), the merge's
+// staged log-sum-exps and two flags.
 // Rows are 16-byte-chunk swizzled: chunk c of row r lives at chunk c ^ (r & 7),
 // which makes every ldmatrix phase hit 8 distinct bank groups.
+// After the main loop the ring holds the warps' partial results and then the
+// partial outputs a merge reads: kMergeFloats floats, i.e. kMergeFloats / (rows * D)
+// chunks of `rows` query heads at a time (192 / rows, whatever D is).
 template <int D>
 struct DecSmem {
   static constexpr int kRowBytes = D * 2;
   static constexpr int kChunks = kRowBytes / 16;
   static constexpr int kTile = kSub * kRowBytes;
   static constexpr int kRing = kDecWarps * kStages * 2 * kTile;
-  static constexpr int kTotal = kTile + kRing + 64;
+  static constexpr int kMergeFloats = kRing / 4;
+  static constexpr int kMergeLse = kMergeFloats / D;  // staged log-sum-exps (chunks x rows) at most
+  static constexpr int kPhysOff = kTile + kRing;
+  static constexpr int kLseOff = kPhysOff + kDecodeMaxChunkSubs * 4;
+  static constexpr int kFlagOff = kLseOff + kMergeLse * 4;
+  static constexpr int kTotal = kFlagOff + 16;
 };
+static_assert(DecSmem<128>::kMergeLse == kDecodeMergeSlots && DecSmem<64>::kMergeLse == kDecodeMergeSlots,
+              "a merge staging holds kDecodeMergeSlots rows of D floats");
+static_assert(kDecodeCtasPerSm * (DecSmem<128>::kTotal + 1024) <= 228 * 1024,
+              "the split plan counts on two resident CTAs per SM at d = 128");
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk, int row_bytes) {
   return static_cast<uint32_t>(row * row_bytes + ((chunk ^ (row & 7)) << 4));
@@ -127,6 +153,143 @@ __device__ __forceinline__ float sink_fold(const float* sinks, int h, float lse_
   return lse_all;
 }
 
+// One ticket on a counter shared by `expected` CTAs of this launch; true for
+// the CTA that takes the last one. The counter's high 32 bits hold the tag of
+// the call that last counted on it: a different tag (another call, or memory
+// that was never a counter) counts as zero, so the workspace needs no
+// clearing. The last CTA puts the counter back to 0. A compare-and-swap fails
+// only when another CTA's ticket succeeded in between, and each of the other
+// expected - 1 CTAs takes exactly one, so the loop ends within `expected`
+// tries; its bound is a guard, on expiry the timeout bit is set.
+__device__ __forceinline__ bool take_last_ticket(unsigned long long* c, uint32_t token, int expected,
+                                                 int32_t* status) {
+  const unsigned long long tag = static_cast<unsigned long long>(token) << 32;
+  unsigned long long cur = atomicAdd(c, 0ull);
+  for (int i = 0; i < 2 * expected + 8; ++i) {
+    const unsigned long long want = ((cur >> 32) == token) ? cur + 1ull : (tag | 1ull);
+    const unsigned long long prev = atomicCAS(c, cur, want);
+    if (prev == cur) {
+      const bool last = static_cast<int>(want & 0xffffffffull) == expected;
+      if (last) atomicExch(c, 0ull);
+      return last;
+    }
+    cur = prev;
+  }
+  flag_status(status, ATTN_STATUS_BIT_TIMEOUT);
+  return false;
+}
+
+// Merge `count` partial results (slots first, first + stride, ...) of `rows`
+// query-head rows into one: lse = log sum_s exp(lse_s), O = sum_s
+// exp(lse_s - lse) O_s ("Inference attention" post, "FlashDecoding"). The
+// partials are staged in shared memory with cp.async (L2 only: they were
+// written by other CTAs of this launch), kMergeFloats / (rows * D) slots at a
+// time, and combined with the online softmax's rescaling between stagings.
+// With `to_output` the row is normalised, the learned sink folded in and O
+// (bf16) and LSE written; otherwise the merged partial goes back into slot
+// `first`. Called by all threads of the CTA.
+template <int D>
+__device__ void merge_partials(const DecodeParams& p, int b, int h0, int rows, int first, int count, int stride,
+                               bool to_output, float* stage, float* lse_s) {
+  constexpr int kMaxCpt = D / 8;
+  int tpr = D / 4;  // threads per row: a power of two, at least 8
+  while (tpr * rows > kDecThreads) tpr >>= 1;
+  const int cpt = D / tpr;  // columns per thread, a multiple of 4
+  const int r = threadIdx.x / tpr;
+  const int part = threadIdx.x % tpr;
+  const bool active = r < rows;
+  const int col0 = part * cpt;
+  const size_t rowg = static_cast<size_t>(b) * p.Hq + h0 + (active ? r : 0);
+  const int cap = DecSmem<D>::kMergeFloats / (rows * D);
+  constexpr int kQuads = D / 4;
+
+  float M = -INFINITY, L = 0.f;
+  bool nan_seen = false;
+  float acc[kMaxCpt];
+#pragma unroll
+  for (int e = 0; e < kMaxCpt; ++e) acc[e] = 0.f;
+
+  for (int c0 = 0; c0 < count; c0 += cap) {
+    const int n = min(cap, count - c0);
+    const int total = n * rows * kQuads;
+    for (int i = threadIdx.x; i < total; i += kDecThreads) {
+      const int sl = i / (rows * kQuads);
+      const int rem = i - sl * rows * kQuads;
+      const int rr = rem / kQuads, c4 = rem - rr * kQuads;
+      const size_t src_row = (static_cast<size_t>(b) * p.Hq + h0 + rr) * p.splits + first + (c0 + sl) * stride;
+      cp_async_16(smem_u32(stage + (sl * rows + rr) * D + c4 * 4), p.o_part + src_row * D + c4 * 4, 16u);
+    }
+    cp_async_commit();
+    for (int i = threadIdx.x; i < n * rows; i += kDecThreads) {
+      const int sl = i / rows, rr = i - sl * rows;
+      lse_s[i] = __ldcg(p.lse_part + (static_cast<size_t>(b) * p.Hq + h0 + rr) * p.splits + first +
+                        (c0 + sl) * stride);
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    if (active) {
+      float m_chunk = -INFINITY;
+      for (int sl = 0; sl < n; ++sl) {
+        const float x = lse_s[sl * rows + r];
+        nan_seen |= (x != x);
+        m_chunk = fmaxf(m_chunk, x);
+      }
+      const float m_new = fmaxf(M, m_chunk);
+      const float keep = (M == -INFINITY) ? 0.f : fast_exp2((M - m_new) * kLog2e);
+      L *= keep;
+#pragma unroll
+      for (int e = 0; e < kMaxCpt; ++e) acc[e] *= keep;
+      for (int sl = 0; sl < n; ++sl) {
+        const float x = lse_s[sl * rows + r];
+        const float w = (x == -INFINITY || x != x) ? 0.f : fast_exp2((x - m_new) * kLog2e);
+        L += w;
+        const float* src = stage + (sl * rows + r) * D + col0;
+#pragma unroll
+        for (int e = 0; e < kMaxCpt; e += 4) {
+          if (e < cpt) {
+            const float4 v = *reinterpret_cast<const float4*>(src + e);
+            acc[e] += w * v.x;
+            acc[e + 1] += w * v.y;
+            acc[e + 2] += w * v.z;
+            acc[e + 3] += w * v.w;
+          }
+        }
+      }
+      M = m_new;
+    }
+    __syncthreads();  // the staging area is refilled by the next round
+  }
+  if (!active) return;
+  float inv = 1.f / L;
+  const float lse_tok = M + __logf(L);
+  if (to_output) {
+    bool bad = nan_seen;
+    bool bad_sink = false;
+    const float lse_out = sink_fold(p.sinks, h0 + r, lse_tok, inv, bad_sink);
+    if (bad_sink && part == 0) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
+    bad |= bad_sink;
+    __nv_bfloat16* dst = p.o + rowg * D + col0;
+#pragma unroll
+    for (int e = 0; e < kMaxCpt; e += 2)
+      if (e < cpt)
+        *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(bad ? NAN : acc[e] * inv, bad ? NAN : acc[e + 1] * inv);
+    if (part == 0 && p.lse != nullptr) p.lse[rowg] = bad ? NAN : lse_out;
+  } else {
+    float* dst = p.o_part + (rowg * p.splits + first) * D + col0;
+#pragma unroll
+    for (int e = 0; e < kMaxCpt; e += 4)
+      if (e < cpt) {
+        float4 v;
+        v.x = nan_seen ? NAN : acc[e] * inv;
+        v.y = nan_seen ? NAN : acc[e + 1] * inv;
+        v.z = nan_seen ? NAN : acc[e + 2] * inv;
+        v.w = nan_seen ? NAN : acc[e + 3] * inv;
+        *reinterpret_cast<float4*>(dst + e) = v;
+      }
+    if (part == 0) p.lse_part[rowg * p.splits + first] = nan_seen ? NAN : lse_tok;
+  }
+}
+
 // WIN: the sequence is read through the visible-sub-block list (sliding window,
 // sink positions); without it every cached token is visible and the list
 // arithmetic folds away at compile time.
@@ -136,7 +299,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* q_s = smem;
   uint8_t* ring = smem + L::kTile;
-  int* cta_bad = reinterpret_cast<int*>(smem + L::kTile + L::kRing);
+  int* phys_s = reinterpret_cast<int*>(smem + L::kPhysOff);
+  float* lse_s = reinterpret_cast<float*>(smem + L::kLseOff);
+  int* cta_bad = reinterpret_cast<int*>(smem + L::kFlagOff);
+  int* last_flag = cta_bad + 1;
 
   const int split = blockIdx.x;
   const int kvh = blockIdx.y / p.hchunks;
@@ -144,13 +310,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   const int b = blockIdx.z;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int h0 = kvh * p.group + hc * 16;
+  const int rows = min(16, p.group - hc * 16);
 
   const int seq_len = p.seq_lens[b];
-  const bool direct = (p.splits == 1);
   if (seq_len < 1 || seq_len > p.max_seq_len) {
-    // the merge kernel flags this row; without a merge this CTA writes its NaN rows
-    if (direct) {
-      const int h0 = kvh * p.group + hc * 16, rows = min(16, p.group - hc * 16);
+    // the first split's CTA writes the NaN rows of this head chunk
+    if (split == 0) {
       for (int i = threadIdx.x; i < rows * D; i += kDecThreads)
         p.o[(static_cast<size_t>(b) * p.Hq + h0 + i / D) * D + i % D] = __float2bfloat16_rn(NAN);
       if (threadIdx.x < rows && p.lse != nullptr) p.lse[static_cast<size_t>(b) * p.Hq + h0 + threadIdx.x] = NAN;
@@ -159,13 +325,20 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
     return;
   }
   const VisibleList vis(seq_len, WIN ? p.window : 0, WIN ? p.n_sink : 0);
-  const int u0 = split * (p.chunk / kSub);  // this split's listed sub-blocks [u0, u0 + nsub)
-  if (u0 >= vis.nsb) return;  // split past the end of the list: the merge never reads it
-  const int nsub = min(p.chunk / kSub, vis.nsb - u0);
-  const int h0 = kvh * p.group + hc * 16;
-  const int rows = min(16, p.group - hc * 16);
+  const int per_split = p.chunk / kSub;
+  const int u0 = split * per_split;  // this split's listed sub-blocks [u0, u0 + nsub)
+  if (u0 >= vis.nsb) return;  // split past the end of the list: nothing to read, no ticket to take
+  const int nsub = min(per_split, vis.nsb - u0);
+  const int ns = (vis.nsb + per_split - 1) / per_split;  // splits that hold sub-blocks of this sequence
+  const bool direct = (ns == 1);
 
   if (threadIdx.x == 0) *cta_bad = 0;
+  // The split's block-table entries, all requested at once (one per listed
+  // sub-block), so that no cache copy waits on a table read later.
+  for (int i = threadIdx.x; i < nsub; i += kDecThreads) {
+    const int lblk = vis.token0(u0 + i) / p.block_size;
+    phys_s[i] = __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks_per_seq + lblk);
+  }
   // Q rows of this head chunk -> swizzled shared tile; padding rows are zero.
   for (int i = threadIdx.x; i < 16 * L::kChunks; i += kDecThreads) {
     const int r = i / L::kChunks, c = i % L::kChunks;
@@ -176,28 +349,17 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   }
   __syncthreads();
 
-  // A fragments of Q for every 16-wide k step (rows = query heads).
-  uint32_t qf[D / 16][4];
-  {
-    const uint32_t qb = smem_u32(q_s);
-    const int r = lane & 15;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const int c = kk * 2 + (lane >> 4);
-      ldmatrix_x4(qb + swz(r, c, L::kRowBytes), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
-    }
-  }
-
   // Per-warp streaming over sub-blocks warp, warp + 4, ...
   uint8_t* my_ring = ring + warp * kStages * 2 * L::kTile;
   const int n_my = (nsub > warp) ? (nsub - warp + kDecWarps - 1) / kDecWarps : 0;
   bool bad = false;
 
   auto issue = [&](int j, int stage) {
-    const int t = vis.token0(u0 + warp + j * kDecWarps);  // first token of the sub-block
+    const int i = warp + j * kDecWarps;  // sub-block of this split
+    const int t = vis.token0(u0 + i);    // its first token
     const int lblk = t / p.block_size;
     const int off = t - lblk * p.block_size;  // multiple of 16, off + 15 < block_size
-    const int phys = __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks_per_seq + lblk);
+    const int phys = phys_s[i];
     const bool ok = (phys >= 0) && (phys < p.num_blocks);
     bad |= !ok;
     const uint32_t kdst = smem_u32(my_ring + stage * 2 * L::kTile);
@@ -213,6 +375,24 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
     }
   };
 
+#pragma unroll
+  for (int j = 0; j < kStages - 1; ++j) {
+    if (j < n_my) issue(j, j);
+    cp_async_commit();
+  }
+
+  // A fragments of Q for every 16-wide k step (rows = query heads).
+  uint32_t qf[D / 16][4];
+  {
+    const uint32_t qb = smem_u32(q_s);
+    const int r = lane & 15;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int c = kk * 2 + (lane >> 4);
+      ldmatrix_x4(qb + swz(r, c, L::kRowBytes), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+    }
+  }
+
   const float neg_inf = -INFINITY;
   float m_run[2] = {neg_inf, neg_inf};  // rows g and g + 8 of this lane (base-2 domain)
   float l_run[2] = {0.f, 0.f};          // per-lane partial sums; reduced over the quad at the end
@@ -222,11 +402,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
 
   const int g = lane >> 2, tq = lane & 3;
 
-#pragma unroll
-  for (int j = 0; j < kStages - 1; ++j) {
-    if (j < n_my) issue(j, j);
-    cp_async_commit();
-  }
   for (int j = 0; j < n_my; ++j) {
     const int jn = j + kStages - 1;
     if (jn < n_my) issue(jn, jn % kStages);
@@ -396,6 +571,40 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
       }
     }
   }
+  if (direct) return;
+
+  // Split-KV merge in this launch. The chunks of the sequence are merged in
+  // groups of group_slots; the CTA finishing a group last merges it (into the
+  // group's first slot, or straight into the output when there is one group),
+  // and the CTA finishing the last group merges the groups. Partial results
+  // are published with a device-scope fence before the ticket and read after
+  // one (through L2), so the merging CTA sees every other CTA's stores.
+  unsigned long long* counters =
+      p.counters + (static_cast<size_t>(b) * gridDim.y + blockIdx.y) * (1 + p.ngroups);
+  const int G = p.group_slots;
+  const int grp = split / G;
+  const int gfirst = grp * G;
+  const int gcount = min(G, ns - gfirst);
+  const int ngroups = (ns + G - 1) / G;
+  float* stage = reinterpret_cast<float*>(ring);
+  __threadfence();
+  __syncthreads();  // the combine area is read above; the merge refills it
+  if (threadIdx.x == 0) *last_flag = take_last_ticket(counters + 1 + grp, p.token, gcount, p.status) ? 1 : 0;
+  __syncthreads();
+  if (*last_flag == 0) return;
+  __threadfence();
+  if (ngroups == 1) {
+    merge_partials<D>(p, b, h0, rows, 0, ns, 1, true, stage, lse_s);
+    return;
+  }
+  merge_partials<D>(p, b, h0, rows, gfirst, gcount, 1, false, stage, lse_s);
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) *last_flag = take_last_ticket(counters, p.token, ngroups, p.status) ? 1 : 0;
+  __syncthreads();
+  if (*last_flag == 0) return;
+  __threadfence();
+  merge_partials<D>(p, b, h0, rows, 0, ngroups, G, true, stage, lse_s);
 }
 
 struct MergeParams {
@@ -591,16 +800,19 @@ template <int D>
 cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
                             const int32_t* seq_lens, const float* sinks, void* o, float* lse, int B, int Hq, int Hkv,
                             int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, int window,
-                            int n_sink, float scale, void* workspace, const DecodePlan& plan, int32_t* status,
-                            cudaStream_t stream) {
+                            int n_sink, float scale, void* workspace, const DecodePlan& plan, uint32_t token,
+                            int32_t* status, cudaStream_t stream) {
   DecodeParams p;
+  const DecodeWorkspace ws = decode_workspace_layout(B, Hq, Hkv, D, plan);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
   p.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
   p.block_table = block_table;
   p.seq_lens = seq_lens;
-  p.o_part = static_cast<float*>(workspace);
-  p.lse_part = p.o_part + static_cast<size_t>(B) * Hq * plan.splits * D;
+  p.o_part = reinterpret_cast<float*>(base + ws.o_part_offset);
+  p.lse_part = reinterpret_cast<float*>(base + ws.lse_part_offset);
+  p.counters = reinterpret_cast<unsigned long long*>(base + ws.counters_offset);
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.sinks = sinks;
@@ -616,8 +828,11 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   p.max_seq_len = max_seq_len;
   p.chunk = plan.chunk;
   p.splits = plan.splits;
+  p.group_slots = plan.group_slots;
+  p.ngroups = plan.ngroups;
   p.window = window;
   p.n_sink = n_sink;
+  p.token = token;
   p.scale_log2 = scale * kLog2e;
 
   const int smem = DecSmem<D>::kTotal;
@@ -626,11 +841,7 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   if (e != cudaSuccess) return e;
   dim3 grid(plan.splits, Hkv * plan.hchunks, B);
   kernel<<<grid, kDecThreads, smem, stream>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || plan.splits == 1) return e;  // one split: the split kernel wrote the output
-
-  return launch_decode_merge(p.o_part, p.lse_part, seq_lens, sinks, o, lse, B, Hq, D, plan.splits, plan.chunk,
-                             max_seq_len, window, n_sink, status, stream);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -672,9 +883,19 @@ cudaError_t launch_decode_merge(const float* o_part, const float* lse_part, cons
   return cudaGetLastError();
 }
 
-size_t decode_workspace_bytes(int B, int Hq, int d, const DecodePlan& plan) {
+DecodeWorkspace decode_workspace_layout(int B, int Hq, int Hkv, int d, const DecodePlan& plan) {
+  DecodeWorkspace w;
   const size_t rows = static_cast<size_t>(B) * Hq * plan.splits;
-  return rows * d * sizeof(float) + rows * sizeof(float);
+  w.o_part_offset = 0;
+  w.lse_part_offset = rows * d * sizeof(float);
+  w.counters_offset = (w.lse_part_offset + rows * sizeof(float) + 15) / 16 * 16;
+  const size_t units = static_cast<size_t>(B) * Hkv * plan.hchunks;
+  w.bytes = w.counters_offset + units * (1 + plan.ngroups) * sizeof(unsigned long long);
+  return w;
+}
+
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, const DecodePlan& plan) {
+  return decode_workspace_layout(B, Hq, Hkv, d, plan).bytes;
 }
 
 int decode_plan_length(int max_seq_len, int window, int n_sink) {
@@ -690,18 +911,40 @@ int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan
     return ATTN_ERR_INVALID_ARG;
   const int group = Hq / Hkv;
   const int hchunks = (group + 15) / 16;
-  const long long units = static_cast<long long>(B) * Hkv * hchunks;
-  // CTAs: at least one per SM. More, shorter splits were measured slower on
-  // single long sequences (per-CTA latency and merge work outweigh the fill).
-  const long long target = 1LL * num_sms;
-  int chunk = 2048;
-  while (chunk > 256 && units * ((max_seq_len + chunk - 1) / chunk) < target) chunk >>= 1;
+  const int rows = group < 16 ? group : 16;
+  const long long units = static_cast<long long>(B) * Hkv * hchunks;  // (sequence, K/V head, head chunk)
+  const long long subs = (static_cast<long long>(max_seq_len) + 15) / 16;
+  const long long slots = static_cast<long long>(kDecodeCtasPerSm) * num_sms;  // CTAs resident at once
+  const long long cap = kDecodeMergeSlots / rows;  // partials one merge stages at a time
+  long long splits;
+  if (units >= slots) {
+    // Enough (sequence, head) units to fill the GPU: 2048-token splits, so
+    // that long sequences of a batch are cut and short ones take one split.
+    splits = (subs + 127) / 128;
+  } else {
+    // Few units (a single long sequence, a small batch): whole waves of
+    // resident CTAs, each split at most kDecodeMaxChunkSubs sub-blocks; with
+    // one wave, at most cap^2 splits so that a two-level merge stages each
+    // level once.
+    const long long waves = (units * subs + slots * kDecodeMaxChunkSubs - 1) / (slots * kDecodeMaxChunkSubs);
+    splits = waves * slots / units;
+    if (waves == 1 && splits > cap * cap) splits = cap * cap;
+    const long long min_chunk_subs = 16;  // at least 256 tokens (4 sub-blocks per warp)
+    splits = std::min(splits, (subs + min_chunk_subs - 1) / min_chunk_subs);
+    splits = std::max(splits, (subs + kDecodeMaxChunkSubs - 1) / kDecodeMaxChunkSubs);
+    splits = std::max(splits, 1LL);
+  }
   // spread the 16-token sub-blocks evenly over the splits (no near-empty last split)
-  const int subs = (max_seq_len + 15) / 16;
-  const int nominal_splits = (max_seq_len + chunk - 1) / chunk;
-  out->chunk = 16 * ((subs + nominal_splits - 1) / nominal_splits);
-  out->splits = (max_seq_len + out->chunk - 1) / out->chunk;
+  const long long chunk_subs = (subs + splits - 1) / splits;
+  out->chunk = static_cast<int>(16 * chunk_subs);
+  out->splits = static_cast<int>((subs + chunk_subs - 1) / chunk_subs);
   out->hchunks = hchunks;
+  // first-level merge groups: all splits in one group when one staging holds
+  // them, else near-equal groups of at most cap splits
+  const long long s = out->splits;
+  const long long nstage = (s + cap - 1) / cap;
+  out->group_slots = static_cast<int>((s + nstage - 1) / nstage);
+  out->ngroups = static_cast<int>((s + out->group_slots - 1) / out->group_slots);
   return ATTN_OK;
 }
 
@@ -710,13 +953,18 @@ cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cach
                           int d, int num_blocks, int block_size, int max_blocks_per_seq, int max_seq_len, int window,
                           int n_sink, float scale, void* workspace, const DecodePlan& plan, int32_t* status,
                           cudaStream_t stream) {
+  // A fresh tag per call for the ticket counters (never 0, the value a finished
+  // call leaves behind).
+  static std::atomic<uint32_t> next_token{0x9e3779b9u};
+  uint32_t token = next_token.fetch_add(1u, std::memory_order_relaxed);
+  if (token == 0u) token = next_token.fetch_add(1u, std::memory_order_relaxed);
   if (d == 128)
     return launch_decode_t<128>(q, k_cache, v_cache, block_table, seq_lens, sinks, o, lse, B, Hq, Hkv, num_blocks,
                                 block_size, max_blocks_per_seq, max_seq_len, window, n_sink, scale, workspace, plan,
-                                status, stream);
+                                token, status, stream);
   return launch_decode_t<64>(q, k_cache, v_cache, block_table, seq_lens, sinks, o, lse, B, Hq, Hkv, num_blocks,
                              block_size, max_blocks_per_seq, max_seq_len, window, n_sink, scale, workspace, plan,
-                             status, stream);
+                             token, status, stream);
 }
 
 cudaError_t launch_paged_gather(const void* cache, const int32_t* block_table, const int32_t* seq_lens, void* out,

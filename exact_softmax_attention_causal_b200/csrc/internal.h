@@ -25,16 +25,31 @@ constexpr long long kDrainBudgetCycles = 4000000000LL;
 void* tensor_map_encode_fn();
 
 struct DecodePlan {
-  int chunk;       // tokens per split (multiple of 16, at most 2048)
-  int splits;      // ceil(planning length / chunk)
-  int hchunks;     // query-head chunks of <= 16 per K/V head
+  int chunk;        // tokens per split (multiple of 16, at most 16 * kDecodeMaxChunkSubs)
+  int splits;       // ceil(planning length / chunk)
+  int hchunks;      // query-head chunks of <= 16 per K/V head
+  int group_slots;  // splits per first-level merge group
+  int ngroups;      // ceil(splits / group_slots)
 };
+// Split plan constants: resident decode CTAs per SM (two fit in shared memory
+// at d = 128), the most 16-token sub-blocks per split, and the partials one
+// merge staging holds for one query-head row (divided by the rows merged).
+constexpr int kDecodeCtasPerSm = 2;
+constexpr int kDecodeMaxChunkSubs = 256;
+constexpr int kDecodeMergeSlots = 192;
 
 int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan* out);
 // Length the split plan is made for: max_seq_len without a window, else the
 // most tokens a windowed query's visible sub-block list can span.
 int decode_plan_length(int max_seq_len, int window, int n_sink);
-size_t decode_workspace_bytes(int B, int Hq, int d, const DecodePlan& plan);
+// Workspace: partial outputs [B, Hq, splits, d] fp32, partial LSEs
+// [B, Hq, splits] fp32, then (16-byte aligned) the merge's ticket counters,
+// 1 + ngroups uint64 per (sequence, K/V head, head chunk).
+struct DecodeWorkspace {
+  size_t o_part_offset, lse_part_offset, counters_offset, bytes;
+};
+DecodeWorkspace decode_workspace_layout(int B, int Hq, int Hkv, int d, const DecodePlan& plan);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, const DecodePlan& plan);
 
 // Kernel launchers (defined next to their kernels). Return cudaError_t.
 // window 0 = every cached token visible (n_sink must then be 0); sinks may be nullptr.

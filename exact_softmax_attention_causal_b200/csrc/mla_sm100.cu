@@ -16,28 +16,37 @@
 // the paged decode's merge kernel (online-softmax rescaling, "Inference
 // attention" post, "FlashDecoding"). The 64 heads' 512-wide fp32 outputs fill
 // 256 of the 512 TMEM columns, so the CTA works on the transposed problem:
-//   S^T [128 tokens x 64 heads]  = K_tile [128 x 576] . Q^T          (M = tokens)
-//   O^T [512 latent x 64 heads] += V_tile^T [512 x 128] . P^T        (4 MMAs of M = 128)
-// K_tile arrives as nine 64-column chunks (128-byte swizzle); its first eight
-// chunks are V_tile, read a second time as an MN-major A operand. P^T is
-// written by the softmax into the ninth chunk's slot once the score MMAs have
-// read it. The softmax runs over the 128 TMEM lanes of each score column
-// (tokens), so its maxima and sums are reduced across lanes: shuffles inside a
-// warp, shared memory across the four warps of a column half.
+//   S^T [64 tokens x 64 heads]   = K_tile [64 x 576] . Q^T          (M = 64 tokens)
+//   O^T [512 latent x 64 heads] += V_tile^T [512 x 64] . P^T        (4 MMAs of M = 128)
+// A tile is 64 cached rows in nine 64-column chunks (128-byte swizzle); its
+// first eight chunks are V_tile, read a second time as an MN-major A operand.
+// Two tiles are in flight: the shared memory holds the resident Q^T (72 KB)
+// and two 72 KB tile slots, so the next tile streams in while the current one
+// is scored, exponentiated and multiplied. P^T is written by the softmax into
+// the ninth chunk's slot once the score MMAs have read it. An M = 64 score
+// tile lives in TMEM lanes 0-15 of each 32-lane sub-partition (token
+// 16 q + i in lane 32 q + i). The softmax runs over the token lanes of each
+// score column, so its maxima and sums are reduced across lanes: shuffles
+// inside a warp, shared memory across the four warps of a column half.
 //
 // Roles (320 threads):
-//   warps 0-7  softmax: warp w reads TMEM lanes 32 (w % 4) .. + 31 (tokens of
-//              the score tile, latent rows of each output block) and head
+//   warps 0-7  softmax: warp w reads TMEM lanes 32 (w % 4) .. + 31 (16 tokens
+//              of the score tile, latent rows of each output block) and head
 //              columns 32 (w / 4) .. + 31. Lazy rescaling as in the prefill:
 //              the max a column's exponentials use moves only when the tile
 //              max exceeds it by more than 8 (base 2).
 //   warp 8     TMA producer: Q^T once (nine 8 KB chunks), then for every tile
-//              the nine 16 KB chunks of 128 cached rows, one box per pool
-//              block, lane e issuing block e's boxes (block-table entries
-//              fetched a tile ahead, one per lane). Rows past the
-//              sequence come in as zeros (one-row boxes for the partly filled
-//              last block, out-of-range block index for whole blocks).
-//   warp 9     MMA issuer; allocates and frees TMEM.
+//              the nine 8 KB chunks of its 64 cached rows into the tile's
+//              slot, one box per pool block (64-row boxes inside blocks of
+//              128), lane e issuing block e's boxes (block-table entries
+//              fetched a tile ahead, one per lane). Rows past the split come
+//              in as zeros (one-row boxes for a partly filled block,
+//              out-of-range block index for whole blocks).
+//   warp 9     MMA issuer; allocates and frees TMEM. It issues each tile's
+//              score MMAs as soon as the tile has landed and a score buffer
+//              is free, and each tile's output MMAs as soon as its P^T is
+//              written, whichever is ready first, so the tensor core works
+//              on the next tile's scores while the softmax runs.
 // All pipeline waits are bounded; on expiry the CTA records
 // ATTN_STATUS_BIT_TIMEOUT, writes NaN partials, drains and exits.
 
@@ -59,8 +68,9 @@ constexpr int kDc = 512;             // latent width d_c (the value width)
 constexpr int kDr = 64;              // positional-key width d_h^R
 constexpr int kRow = kDc + kDr;      // cached row width
 constexpr int kChunks = kRow / 64;   // 64-column chunks of a row (128-byte swizzle)
-constexpr int kTok = 128;            // tokens per tile = TMEM lanes
+constexpr int kTok = 64;             // tokens per tile (the score MMA's M)
 constexpr int kNH = 64;              // heads per CTA = MMA N
+constexpr int kSlots = 2;            // tiles in flight
 constexpr int kPSlot = kChunks - 1;  // the positional chunk's slot holds P^T after the score MMAs
 constexpr int kMlaThreads = 320;
 constexpr int kMlaTmaWarp = 8;
@@ -68,10 +78,11 @@ constexpr int kMlaMmaWarp = 9;
 constexpr float kMlaRescaleThreshold = 8.0f;
 
 constexpr int kQChunkBytes = kNH * 128;   // 64 heads x 64 columns
-constexpr int kKChunkBytes = kTok * 128;  // 128 tokens x 64 columns
+constexpr int kKChunkBytes = kTok * 128;  // 64 tokens x 64 columns
+constexpr int kTileBytes = kChunks * kKChunkBytes;
 constexpr int kQOff = 0;
 constexpr int kKOff = kQOff + kChunks * kQChunkBytes;
-constexpr int kRedOff = kKOff + kChunks * kKChunkBytes;  // cross-warp reductions: [2 halves][4 warps][32]
+constexpr int kRedOff = kKOff + kSlots * kTileBytes;  // cross-warp reductions: [2 halves][4 warps][32]
 constexpr int kRedBytes = 2 * 4 * 32 * 4;
 constexpr int kMOff = kRedOff + kRedBytes;  // running max per head column: [2 halves][32]
 constexpr int kBarOff = kMOff + 2 * 32 * 4;
@@ -86,14 +97,14 @@ constexpr uint32_t kTmemCols = 512;
 
 enum : int {
   kMbQFull = 0,
-  kMbKFull = 1,    // + chunk (9)
-  kMbKEmpty = 10,  // + chunk (9)
-  kMbSFull = 19,   // + buffer (2)
-  kMbSFree = 21,   // + buffer (2), one arrival per softmax warp
-  kMbPFull = 23,   // one arrival per softmax warp
-  kMbOReady = 24,  // the tile's output MMAs completed
-  kMbDrain = 25,
-  kMbCount = 26,
+  kMbKFull = 1,    // + slot (2): the tile's nine chunks landed
+  kMbKEmpty = 3,   // + slot (2): the tile's output MMAs have read it
+  kMbSFull = 5,    // + buffer (2)
+  kMbSFree = 7,    // + buffer (2), one arrival per softmax warp
+  kMbPFull = 9,    // + slot (2), one arrival per softmax warp
+  kMbOReady = 11,  // the tile's output MMAs completed
+  kMbDrain = 12,
+  kMbCount = 13,
 };
 constexpr int kMlaTmemSlot = 224;
 constexpr int kMlaAbort = 228;
@@ -172,15 +183,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kMbQFull), 1);
-    for (int j = 0; j < kChunks; ++j) {
-      mbar_init(bar(kMbKFull + j), 1);
-      mbar_init(bar(kMbKEmpty + j), 1);
-    }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(bar(kMbKFull + s), 1);
+      mbar_init(bar(kMbKEmpty + s), 1);
       mbar_init(bar(kMbSFull + s), 1);
       mbar_init(bar(kMbSFree + s), 8);
+      mbar_init(bar(kMbPFull + s), 8);
     }
-    mbar_init(bar(kMbPFull), 8);
     mbar_init(bar(kMbOReady), 1);
     mbar_init(bar(kMbDrain), 1);
     *abort_flag = 0;
@@ -199,11 +208,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 
   if (warp == kMlaTmaWarp) {
     // ------------------------------------------------------------ TMA producer
-    // Lane 0 waits on the slots and arms their barriers; lane e then issues the
-    // boxes of the tile's e-th pool block, so the (up to 8) copies of a chunk go
-    // out from different threads at once.
+    // Lane 0 waits for the tile's slot and arms its barrier; lane e then issues
+    // the boxes of the tile's e-th pool block (or, for 128-token blocks, the
+    // tile's 64-row half of its block), so a tile's copies go out from several
+    // threads at once.
     const int bs = p.block_size;
-    const int boxes = kTok / bs;  // pool blocks per tile (block_size divides 128)
+    const int box_rows = bs < kTok ? bs : kTok;
+    const int boxes = kTok / box_rows;
     const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -217,61 +228,54 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // out-of-range index num_blocks (TMA fills zeros); a bad referenced entry
     // also marks the CTA's output as invalid.
     auto fetch = [&](int tile) -> int {
-      const int key = t0 + tile * kTok + lane * bs;
+      const int key = t0 + tile * kTok + lane * box_rows;
       return (lane < boxes && key < t1) ? __ldg(table + key / bs) : p.num_blocks;
     };
     int ent = fetch(0);
-    int issued = 0;  // lane 0: tiles whose copies were issued for every chunk
-    int last_j = -1;  // lane 0: chunks of the tile being issued when a wait gave up
+    int issued = 0;  // tiles whose copies were all issued
     bool ok = true;
     for (int i = 0; i < ntiles && ok; ++i) {
+      const int slot = i % kSlots;
       const int ent_next = (i + 1 < ntiles) ? fetch(i + 1) : p.num_blocks;
-      const int tok0 = t0 + i * kTok;
-      const int key = tok0 + lane * bs;
+      const int key = t0 + i * kTok + lane * box_rows;
       int phys = ent;
       if (lane < boxes && key < t1 && (phys < 0 || phys >= p.num_blocks)) {
         *bad_flag = 1;
         phys = p.num_blocks;
       }
       if (key >= t1) phys = p.num_blocks;
-      for (int j = 0; j < kChunks; ++j) {
-        bool armed = true;
-        if (lane == 0) {
-          armed = (i == 0) || mbar_wait_bounded(bar(kMbKEmpty + j), (i - 1) & 1, budget, abort_flag);
-          if (armed) {
-            mbar_arrive_expect_tx(bar(kMbKFull + j), kKChunkBytes);
-            last_j = j;
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, armed, 0);
-        if (!ok) break;
-        if (lane < boxes) {
-          const uint32_t dst = sbase + kKOff + j * kKChunkBytes + lane * bs * 128;
-          if (key + bs <= t1 || phys == p.num_blocks) {
-            tma_load_3d(dst, &tm_c, bar(kMbKFull + j), 64 * j, 0, phys);
-          } else {
-            const int valid = t1 - key;  // 1 .. bs - 1 rows hold tokens of this split
-            for (int r = 0; r < bs; ++r)
-              tma_load_3d(dst + r * 128, &tm_crow, bar(kMbKFull + j), 64 * j, r, r < valid ? phys : p.num_blocks);
-          }
+      bool armed = true;
+      if (lane == 0) {
+        armed = (i < kSlots) ||
+                mbar_wait_bounded(bar(kMbKEmpty + slot), ((i - kSlots) / kSlots) & 1, budget, abort_flag);
+        if (armed) mbar_arrive_expect_tx(bar(kMbKFull + slot), kTileBytes);
+      }
+      ok = __shfl_sync(0xffffffffu, armed, 0);
+      if (!ok) break;
+      if (lane < boxes) {
+        const int row0 = key % bs;  // first row of the box inside its block
+        const uint32_t dst0 = sbase + kKOff + slot * kTileBytes + lane * box_rows * 128;
+        if (key + box_rows <= t1 || phys == p.num_blocks) {
+          for (int j = 0; j < kChunks; ++j)
+            tma_load_3d(dst0 + j * kKChunkBytes, &tm_c, bar(kMbKFull + slot), 64 * j, row0, phys);
+        } else {
+          const int valid = t1 - key;  // 1 .. box_rows - 1 rows hold tokens of this split
+          for (int j = 0; j < kChunks; ++j)
+            for (int r = 0; r < box_rows; ++r)
+              tma_load_3d(dst0 + j * kKChunkBytes + r * 128, &tm_crow, bar(kMbKFull + slot), 64 * j, row0 + r,
+                          r < valid ? phys : p.num_blocks);
         }
       }
-      if (ok) {
-        issued = i + 1;
-        last_j = -1;
-      }
+      issued = i + 1;
       ent = ent_next;
     }
     if (lane == 0) {
       if (!ok) mla_abort(abort_flag, p.status);
-      // Drain: Q and the newest copy of every chunk slot landed before the CTA may exit
-      // (chunks 0 .. last_j of an interrupted tile belong to tile `issued`).
+      // Drain: Q and the newest copy of every slot landed before the CTA may exit.
       volatile int never = 0;
       mbar_wait_bounded(bar(kMbQFull), 0, kDrainBudgetCycles, &never);
-      for (int j = 0; j < kChunks; ++j) {
-        const int n = (j <= last_j) ? issued + 1 : issued;
-        if (n > 0) mbar_wait_bounded(bar(kMbKFull + j), (n - 1) & 1, kDrainBudgetCycles, &never);
-      }
+      for (int i = (issued > kSlots ? issued - kSlots : 0); i < issued; ++i)
+        mbar_wait_bounded(bar(kMbKFull + i % kSlots), (i / kSlots) & 1, kDrainBudgetCycles, &never);
     }
   } else if (warp == kMlaMmaWarp) {
     if (lane == 0) {
@@ -279,50 +283,64 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       const uint64_t dq = desc_sw128(sbase + kQOff, 16, 1024);
       const uint64_t dk = desc_sw128(sbase + kKOff, 16, 1024);
       // V^T block m: chunks 2m and 2m + 1 (64 latent columns each) as one MN-major
-      // operand; P^T in the positional slot, MN-major, one 64-head group.
+      // operand; P^T in the positional chunk's place, MN-major, one 64-head group.
       const uint64_t dv = desc_sw128(sbase + kKOff, kKChunkBytes, 1024);
       const uint64_t dp = desc_sw128(sbase + kKOff + kPSlot * kKChunkBytes, kKChunkBytes, 1024);
+      constexpr uint64_t kTileUnits = kTileBytes >> 4;
       bool ok = mbar_wait_bounded(bar(kMbQFull), 0, budget, abort_flag);
-      for (int i = 0; i < ntiles && ok; ++i) {
-        const int sb = i & 1;
-        if (i >= 2 && !mbar_wait_bounded(bar(kMbSFree + sb), ((i - 2) >> 1) & 1, budget, abort_flag)) {
-          ok = false;
-          break;
-        }
-        // S^T = K . Q^T over the nine chunks, 4 steps of 16 columns each
-        for (int j = 0; j < kChunks && ok; ++j) {
-          if (!mbar_wait_bounded(bar(kMbKFull + j), i & 1, budget, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+      // Tile j's scores need its slot loaded and score buffer j % 2 released by
+      // the softmax of tile j - 2; its output MMAs need its P^T. Each is issued
+      // as soon as it is ready. Every barrier tested here is at most one phase
+      // ahead of the phase tested (the next phase needs work issued after this
+      // test), so the parity tests are unambiguous.
+      int ns = 0, npv = 0;
+      long long idle_since = clock64();
+      while (ok && npv < ntiles) {
+        bool progressed = false;
+        if (ns < ntiles && ns < npv + kSlots) {
+          const int sl = ns % kSlots;
+          if (mbar_try_wait(bar(kMbKFull + sl), (ns / kSlots) & 1) &&
+              (ns < kSlots || mbar_try_wait(bar(kMbSFree + sl), ((ns - kSlots) / kSlots) & 1))) {
+            tc_fence_after();
+            // S^T = K . Q^T over the nine chunks, 4 steps of 16 columns each
+            for (int j = 0; j < kChunks; ++j) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t a = dk + static_cast<uint64_t>((j * kKChunkBytes + kk * 32) >> 4);
-            const uint64_t bq = dq + static_cast<uint64_t>((j * kQChunkBytes + kk * 32) >> 4);
-            tc_mma_ss(tmem + kColS + 64u * sb, a, bq, kIdescScore, (j | kk) != 0 ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t a = dk + sl * kTileUnits + static_cast<uint64_t>((j * kKChunkBytes + kk * 32) >> 4);
+                const uint64_t bq = dq + static_cast<uint64_t>((j * kQChunkBytes + kk * 32) >> 4);
+                tc_mma_ss(tmem + kColS + 64u * sl, a, bq, kIdescScore, (j | kk) != 0 ? 1u : 0u);
+              }
+            }
+            tc_commit(bar(kMbSFull + sl));
+            ++ns;
+            progressed = true;
           }
         }
-        if (!ok) break;
-        tc_commit(bar(kMbSFull + sb));
-        // O^T += V^T . P^T once the softmax wrote P^T (and rescaled O^T if needed)
-        if (!mbar_wait_bounded(bar(kMbPFull), i & 1, budget, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        for (int m = 0; m < 4; ++m) {
+        if (!progressed && npv < ns) {
+          const int sl = npv % kSlots;
+          if (mbar_try_wait(bar(kMbPFull + sl), (npv / kSlots) & 1)) {
+            tc_fence_after();
+            // O^T += V^T . P^T (the softmax rescaled O^T first where its max moved)
+            for (int m = 0; m < 4; ++m) {
 #pragma unroll
-          for (int kk = 0; kk < kTok / 16; ++kk) {
-            const uint64_t a = dv + static_cast<uint64_t>((2 * m * kKChunkBytes + kk * 2048) >> 4);
-            const uint64_t bp = dp + static_cast<uint64_t>((kk * 2048) >> 4);
-            tc_mma_ss(tmem + kColO + 64u * m, a, bp, kIdescOut, (i > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < kTok / 16; ++kk) {
+                const uint64_t a =
+                    dv + sl * kTileUnits + static_cast<uint64_t>((2 * m * kKChunkBytes + kk * 2048) >> 4);
+                const uint64_t bp = dp + sl * kTileUnits + static_cast<uint64_t>((kk * 2048) >> 4);
+                tc_mma_ss(tmem + kColO + 64u * m, a, bp, kIdescOut, (npv > 0 || kk > 0) ? 1u : 0u);
+              }
+            }
+            tc_commit(bar(kMbKEmpty + sl));
+            tc_commit(bar(kMbOReady));
+            ++npv;
+            progressed = true;
           }
-          tc_commit(bar(kMbKEmpty + 2 * m));
-          tc_commit(bar(kMbKEmpty + 2 * m + 1));
         }
-        tc_commit(bar(kMbKEmpty + kPSlot));
-        tc_commit(bar(kMbOReady));
+        if (progressed) {
+          idle_since = clock64();
+        } else if (*abort_flag || clock64() - idle_since > budget) {
+          ok = false;
+        }
       }
       if (!ok) mla_abort(abort_flag, p.status);
       tc_commit(bar(kMbDrain));
@@ -333,11 +351,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // ------------------------------------------------------------ softmax warps 0-7
     const int sp = warp & 3;    // TMEM sub-partition: lanes 32 sp .. 32 sp + 31
     const int hh = warp >> 2;   // head columns 32 hh .. 32 hh + 31
-    const int r = sp * 32 + lane;  // token row of a score tile / latent row of an output block
+    const int r = sp * 32 + lane;      // latent row of an output block
+    const int tok = sp * 16 + lane;    // token of a score tile held by this lane (lanes 0-15)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(sp * 32) << 16);
     float* red = reinterpret_cast<float*>(smem + kRedOff) + hh * 4 * 32;  // [4 warps][32]
     float* msm = reinterpret_cast<float*>(smem + kMOff) + hh * 32;        // running max per head column
-    uint8_t* pslot = smem + kKOff + kPSlot * kKChunkBytes;
     const float sl2 = p.scale_log2;
     if (sp == 0) msm[lane] = -INFINITY;
     float l_part[32];  // this thread's share (its token rows) of every column's sum
@@ -350,10 +368,12 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // work), so no warp can be left waiting at a barrier the others skipped.
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
-      const int sb = i & 1;
+      const int sb = i % kSlots;
       const uint32_t col_s = lane_base + kColS + 64u * sb + 32u * hh;
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kMbSFull + sb), (i >> 1) & 1, budget, abort_flag));
-      const bool valid = ok && (t0 + i * kTok + r) < t1;
+      if (ok)
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kMbSFull + sb), (i / kSlots) & 1, budget, abort_flag));
+      // lanes 16-31 of the sub-partition hold no score of an M = 64 tile
+      const bool valid = ok && lane < 16 && (t0 + i * kTok + tok) < t1;
       float wmax = -INFINITY;
       if (ok) {
         tc_fence_after();
@@ -363,7 +383,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         float v[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) v[c] = valid ? __uint_as_float(raw[c]) * sl2 : -INFINITY;
-        wmax = warp_reduce_scatter32<true>(v, lane);  // lane c: column c over this warp's 32 tokens
+        wmax = warp_reduce_scatter32<true>(v, lane);  // lane c: column c over this warp's 16 tokens
       }
       // tile max of every head column across the 4 warps; running max update
       red[sp * 32 + lane] = wmax;
@@ -399,8 +419,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         }
       }
       // probabilities from a second read of the scores (fewer live registers);
-      // P^T row r (token), head columns 32 hh .. + 31 -> 64 bytes of the
-      // 128-byte swizzled row: 16-byte chunk q lands at chunk q ^ (r & 7)
+      // P^T row tok (lanes 0-15), head columns 32 hh .. + 31 -> 64 bytes of the
+      // 128-byte swizzled row: 16-byte chunk q lands at chunk q ^ (tok & 7)
       uint32_t raw[32];
       tmem_ld_32x32b_x32(col_s, raw);
       tc_wait_ld();
@@ -418,23 +438,26 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         l_part[c + 1] += p1;
         pk[c >> 1] = pack_bf16x2(p0, p1);
       }
+      if (lane < 16) {
+        uint8_t* pslot = smem + kKOff + sb * kTileBytes + kPSlot * kKChunkBytes;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int chunk = hh * 4 + q;
-        *reinterpret_cast<uint4*>(pslot + r * 128 + ((chunk ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        for (int q = 0; q < 4; ++q) {
+          const int chunk = hh * 4 + q;
+          *reinterpret_cast<uint4*>(pslot + tok * 128 + ((chunk ^ (tok & 7)) << 4)) =
+              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kMbPFull));
+      if (lane == 0) mbar_arrive(bar(kMbPFull + sb));
     }
     // ------------------------------------------------------------ epilogue
     if (ok)
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kMbOReady), (ntiles - 1) & 1, budget, abort_flag));
     if (!ok) mla_abort(abort_flag, p.status);
     tc_fence_after();
-    // column sums of the probabilities over all 128 token rows
+    // column sums of the probabilities over all 64 token rows
     const float wsum = warp_reduce_scatter32<false>(l_part, lane);
     red[sp * 32 + lane] = wsum;
     named_sync(1 + hh, 128);
@@ -511,7 +534,8 @@ int launch_mla_decode(const void* q, const void* cache, const int32_t* block_tab
                       int max_seq_len, float scale, void* workspace, const MlaPlan& plan, int32_t* status,
                       cudaStream_t stream) {
   CUtensorMap tq, tc, tcr;
-  if (!encode_rank3(&tq, q, kRow, H, B, kNH) || !encode_rank3(&tc, cache, kRow, block_size, num_blocks, block_size) ||
+  const int box_rows = block_size < kTok ? block_size : kTok;  // 64-row boxes inside 128-token blocks
+  if (!encode_rank3(&tq, q, kRow, H, B, kNH) || !encode_rank3(&tc, cache, kRow, block_size, num_blocks, box_rows) ||
       !encode_rank3(&tcr, cache, kRow, block_size, num_blocks, 1))
     return ATTN_ERR_CUDA;
   MlaParams p;

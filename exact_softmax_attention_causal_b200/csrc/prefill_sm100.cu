@@ -197,6 +197,27 @@ __device__ __forceinline__ ItemGeom item_geom(const PrefillParams& p, const Work
   return ItemGeom{nk, pos0, lo, hi - lo + 1, bad};
 }
 
+// Key tiles each query tile of an item needs, relative to the item's first
+// key tile: tile A (x = 0) uses [0, a1), tile B (x = 1) uses [b0, T). Tile A's
+// rows end one key tile earlier under a causal or window mask, and tile B's
+// window starts up to one tile later, so each skips the tile only the other
+// needs. A always uses the first key tile and B the last, and together they
+// cover all T.
+struct TileRanges {
+  int a1, b0;
+};
+__device__ __forceinline__ TileRanges tile_ranges(const PrefillParams& p, const WorkItem& wi, const ItemGeom& gm) {
+  int a1 = gm.T, b0 = 0;
+  if (p.mask_kind != ATTN_MASK_FULL) {
+    const int hi_a = min((gm.nk - 1) / kBN, (gm.pos0 + wi.q0 + kBM - 1) / kBN);
+    a1 = hi_a - gm.lo + 1;
+  }
+  if (p.mask_kind == ATTN_MASK_SLIDING_WINDOW) b0 = max(0, gm.pos0 + wi.q0 + kBM - p.window + 1) / kBN - gm.lo;
+  // a tile B wholly past the last row still runs the last key tile (its rows are
+  // never stored), so that both tiles finish every item
+  return TileRanges{a1, min(b0, gm.T - 1)};
+}
+
 // True when every (row, key) pair of a 128 x 128 tile is visible: rows at
 // positions [qpos0, qpos0 + 128), keys [k0, k0 + 128) of nk.
 __device__ __forceinline__ bool tile_is_full(const PrefillParams& p, int qpos0, int k0, int nk) {
@@ -209,30 +230,6 @@ __device__ __forceinline__ bool tile_is_full(const PrefillParams& p, int qpos0, 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int32_t* status) {
   *abort_flag = 1;
   if (status != nullptr) atomicOr(status, ATTN_STATUS_BIT_TIMEOUT);
-}
-
-// 2^x for a pair of x on the FMA pipes instead of the special-function unit:
-// x = n + f with n = round(x) (added to the exponent field) and f in
-// [-1/2, 1/2]; 2^f by a degree-4 polynomial whose maximum relative error on
-// that interval is minimised (Remez exchange, fitted by fit_exp2_poly.py next
-// to this file: 2.7e-6 in float32). x is clamped to >= -126 so the result
-// stays a positive number below 2^-125 where the true value is smaller.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
-  x.x = fmaxf(x.x, -126.0f);
-  x.y = fmaxf(x.y, -126.0f);
-  const float2 t = fadd2(x, make_float2(kRound, kRound));
-  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
-  const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);
-  float2 p = ffma2(make_float2(0.009570102207362652f, 0.009570102207362652f), f,
-                   make_float2(0.05591785907745361f, 0.05591785907745361f));
-  p = ffma2(p, f, make_float2(0.240247443318367f, 0.240247443318367f));
-  p = ffma2(p, f, make_float2(0.6931217908859253f, 0.6931217908859253f));
-  p = ffma2(p, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
-  // the low mantissa bits of t hold n; shifting by 23 moves n into the exponent
-  const uint32_t r0 = __float_as_uint(p.x) + (__float_as_uint(t.x) << 23);
-  const uint32_t r1 = __float_as_uint(p.y) + (__float_as_uint(t.y) << 23);
-  return make_float2(__uint_as_float(r0), __uint_as_float(r1));
 }
 
 // One MMA step of S = Q K^T: descriptors are the operand bases plus a fixed
@@ -271,9 +268,6 @@ __device__ __forceinline__ void mma_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_
   if constexpr (KK + 1 < END) mma_pv<D, KK + 1, END>(d_tmem, p_tmem, dv, first);
 }
 
-// Column pairs (of every 8) whose exponentials run on the FMA pipes: bit e set
-// = pair e uses exp2_poly2, the others use the special-function unit.
-constexpr uint32_t kPolyPairs = 0x00;
 // Scale-and-shift and the running sums with paired fp32 instructions.
 constexpr bool kPairedFma = true;
 
@@ -510,9 +504,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc_commit(bar(kBarSFull + x));
       };
       // O_x (+)= P_x V for keys [64 half, 64 half + 64) of global key tile g; P_x sits in
-      // the first 64 score columns (16 keys = 8 columns per MMA step); `first` starts O_x
-      auto pv_half = [&](int x, int g, int half, bool first) -> bool {
-        if (!mbar_wait_bounded(bar((half ? kBarPHi : kBarPLo) + x), g & 1, budget, abort_flag)) return false;
+      // the first 64 score columns (16 keys = 8 columns per MMA step); `first` starts O_x.
+      // c is tile x's count of score tiles so far (the parity of its S and P barriers).
+      auto pv_half = [&](int x, int g, int c, int half, bool first) -> bool {
+        if (!mbar_wait_bounded(bar((half ? kBarPHi : kBarPLo) + x), c & 1, budget, abort_flag)) return false;
         tc_fence_after();
         const uint64_t dv = dv0 + static_cast<uint64_t>(g % C::kVStages) * kTileUnits;
         if (half == 0)
@@ -522,12 +517,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         return true;
       };
       int g = 0, it = 0;
+      int cnt[kTilesPerCta] = {0, 0};  // score tiles computed per query tile
       bool ok = true;
       for (int round = 0; ok; ++round) {
         const int w = item_index(round, cta, G);
         if (w >= p.num_items) break;
         const WorkItem wi = item_at(p, w, order, use_order);
-        const int T = item_geom<PAGED>(p, wi).T;
+        const ItemGeom gm = item_geom<PAGED>(p, wi);
+        const int T = gm.T;
+        const TileRanges tr = tile_ranges(p, wi, gm);
         if (!mbar_wait_bounded(bar(kBarQFull), it & 1, budget, abort_flag) ||
             !mbar_wait_bounded(bar(kBarKFull + g % C::kKStages), (g / C::kKStages) & 1, budget, abort_flag)) {
           ok = false;
@@ -535,37 +533,46 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         tc_fence_after();
         issue_s(0, g);
-        issue_s(1, g);
+        if (tr.b0 == 0) issue_s(1, g);
         tc_commit(bar(kBarKEmpty + g % C::kKStages));
         if (T == 1) tc_commit(bar(kBarQEmpty));
         for (int j = 0; j < T; ++j) {
           const int gj = g + j, gn = gj + 1;
           const int s = gj % C::kVStages;  // V stage of key tile j
-          // tile A: P.V of key tile j (as each half of P lands), then the scores of tile
-          // j + 1 (in issue order, so the new scores overwrite P only after P.V read it)
-          if (!mbar_wait_bounded(bar(kBarVFull + s), (gj / C::kVStages) & 1, budget, abort_flag) ||
-              !pv_half(0, gj, 0, j == 0) || !pv_half(0, gj, 1, j == 0)) {
+          if (!mbar_wait_bounded(bar(kBarVFull + s), (gj / C::kVStages) & 1, budget, abort_flag)) {
             ok = false;
             break;
           }
-          if (j == T - 1) tc_commit(bar(kBarOFinal + 0));
+          // tile A: P.V of key tile j (as each half of P lands), then the scores of tile
+          // j + 1 (in issue order, so the new scores overwrite P only after P.V read it)
+          if (j < tr.a1) {
+            if (!pv_half(0, gj, cnt[0], 0, j == 0) || !pv_half(0, gj, cnt[0], 1, j == 0)) {
+              ok = false;
+              break;
+            }
+            ++cnt[0];
+            if (j == tr.a1 - 1) tc_commit(bar(kBarOFinal + 0));
+          }
           if (j + 1 < T) {
             if (!mbar_wait_bounded(bar(kBarKFull + gn % C::kKStages), (gn / C::kKStages) & 1, budget, abort_flag)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            issue_s(0, gn);
+            if (j + 1 < tr.a1) issue_s(0, gn);
           }
           // tile B
-          if (!pv_half(1, gj, 0, j == 0) || !pv_half(1, gj, 1, j == 0)) {
-            ok = false;
-            break;
+          if (j >= tr.b0) {
+            if (!pv_half(1, gj, cnt[1], 0, j == tr.b0) || !pv_half(1, gj, cnt[1], 1, j == tr.b0)) {
+              ok = false;
+              break;
+            }
+            ++cnt[1];
+            if (j == T - 1) tc_commit(bar(kBarOFinal + 1));
           }
-          if (j == T - 1) tc_commit(bar(kBarOFinal + 1));
           tc_commit(bar(kBarVEmpty + s));
           if (j + 1 < T) {
-            issue_s(1, gn);
+            if (j + 1 >= tr.b0) issue_s(1, gn);
             tc_commit(bar(kBarKEmpty + gn % C::kKStages));
             if (j + 2 == T) tc_commit(bar(kBarQEmpty));  // that was the item's last read of Q
           }
@@ -589,7 +596,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t colO = lane_base + C::col_o(x);
     const float sl2 = p.scale_log2;
     auto rescale_rows = [](uint32_t col, float f) { rescale_row_t<D>(col, f); };
-    int g = 0, it = 0;
+    int cnt = 0, it = 0;  // this tile's score tiles so far, items so far
     bool ok = true;
     for (int round = 0;; ++round) {
       const int w = item_index(round, cta, G);
@@ -619,10 +626,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       float m_used = -INFINITY;         // max the exponentials are taken against (base 2)
       float l_sum = 0.f;                // running sum of 2^(x - m_used), fp32
-      for (int j = 0; j < T && ok; ++j) {
-        const int gj = g + j;
+      const TileRanges tr = tile_ranges(p, wi, gm);
+      const int j_end = x == 0 ? tr.a1 : T;
+      for (int j = x == 0 ? 0 : tr.b0; j < j_end && ok; ++j, ++cnt) {
         const int k0 = (kt_lo + j) * kBN;
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBarSFull + x), gj & 1, budget, abort_flag));
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBarSFull + x), cnt & 1, budget, abort_flag));
         if (!ok) break;
         tc_fence_after();
         uint32_t raw[kBN];
@@ -683,12 +691,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               xv.y = fmaf(sv[c + 1], sl2, neg_m);
             }
             float2 pv;
-            if ((kPolyPairs >> (e & 7)) & 1) {
-              pv = exp2_poly2(xv);
-            } else {
-              pv.x = fast_exp2(xv.x);
-              pv.y = fast_exp2(xv.y);
-            }
+            pv.x = fast_exp2(xv.x);
+            pv.y = fast_exp2(xv.y);
             float2& acc = (e & 3) == 0 ? acc0 : (e & 3) == 1 ? acc1 : (e & 3) == 2 ? acc2 : acc3;
             if (kPairedFma) {
               acc = fadd2(acc, pv);
@@ -759,7 +763,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // The next item's first P.V overwrites O: its P is announced only after
       // these loads completed (tcgen05.wait::ld above, fence before the arrive).
       tc_fence_before();
-      g += T;
       ++it;
     }
     if (lane == 0) bulk_wait_all();  // output stores complete before the CTA exits

@@ -157,15 +157,19 @@ ATTN_API int attn_prefill_paged(const void* q, const void* k_cache, const void* 
  * GPU needed). Long sequences are cut into chunks of *chunk_tokens tokens
  * (a multiple of 16); each (sequence, K/V head, chunk) is one unit of work
  * ("Inference attention" post, "FlashDecoding": split keys along the
- * sequence so that small batches fill the GPU). num_sms is the device's SM
- * count. Returns ATTN_OK or ATTN_ERR_INVALID_ARG.
+ * sequence so that small batches fill the GPU). With at least two (sequence,
+ * K/V head, 16-head chunk) units per SM the chunks are 2048 tokens; with fewer
+ * (a single long sequence, a small batch) the chunk count fills whole waves
+ * of two resident CTAs per SM, each chunk at most 4096 tokens. num_sms is the
+ * device's SM count. Returns ATTN_OK or ATTN_ERR_INVALID_ARG.
  */
 ATTN_API int attn_decode_plan(int B, int Hq, int Hkv, int max_seq_len, int num_sms, int* chunk_tokens, int* num_splits);
 
 /*
  * attn_decode_workspace_bytes - bytes of device workspace attn_decode_paged
  * needs for these sizes on the current device (partial outputs fp32
- * [B, Hq, splits, d] plus partial log-sum-exp fp32 [B, Hq, splits]).
+ * [B, Hq, splits, d], partial log-sum-exp fp32 [B, Hq, splits], then the
+ * split merge's ticket counters, a few uint64 per (sequence, K/V head)).
  * Returns 0 for invalid sizes.
  */
 ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int max_seq_len, int block_size);
@@ -180,7 +184,8 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int m
  * block block_table[b][t / block_size]. The query attends to all seq_lens[b]
  * cached tokens, its own K/V already appended ("USAAIO Lesson 90", part 2), so
  * no mask applies. Split partials are merged with the online softmax's
- * rescaling ("Inference attention" post, "FlashDecoding").
+ * rescaling ("Inference attention" post, "FlashDecoding"), inside the same
+ * single launch: the last CTA to finish a sequence's splits merges them.
  *
  *   q            [B, Hq, d] bf16                            read
  *   k_cache,
@@ -194,7 +199,11 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int m
  *   block_size   a multiple of 16 (the pages' default is 16)
  *   max_seq_len  <= max_blocks_per_seq * block_size
  *   workspace    device scratch of at least attn_decode_workspace_bytes(...)
- *                bytes, 16-byte aligned; contents on entry are irrelevant.
+ *                bytes, 16-byte aligned; contents on entry are irrelevant
+ *                (the merge's counters carry a 32-bit tag that changes with
+ *                every call; a counter without this call's tag counts as
+ *                zero). Calls whose kernels overlap on the GPU must not share
+ *                a workspace.
  *   status       device int32 or NULL.
  *
  * A referenced block-table entry outside [0, num_blocks) or a seq_len outside
@@ -407,8 +416,10 @@ ATTN_API int attn_paged_gather(const void* cache, const int32_t* block_table, co
  *     point on that device again in the same process.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind. Nothing in it has to start at zero: each call writes every
- *     partial it later reads. Calls whose kernels overlap on the GPU (two
- *     streams, or two host threads) race on the array: serialise them.
+ *     partial it later reads, and the merge's ticket counters carry a tag
+ *     that changes with every call (the array is zero when the library
+ *     loads). Calls whose kernels overlap on the GPU (two streams, or two
+ *     host threads) race on the array: serialise them.
  * Outputs, errors and device checks are exactly those of attn_decode_paged.
  */
 #define ATTN_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20) /* 32 MiB */

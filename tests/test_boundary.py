@@ -231,7 +231,7 @@ def _plan(B, Hq, Hkv, L, sms=148):
 def test_decode_plan_covers_the_sequence(B, Hq, Hkv, L):
     rc, chunk, splits = _plan(B, Hq, Hkv, L)
     assert rc == _lib.ATTN_OK
-    assert chunk % 16 == 0 and 16 <= chunk <= 2048
+    assert chunk % 16 == 0 and 16 <= chunk <= 4096
     assert splits == -(-L // chunk)
     # the 16-token sub-blocks are spread evenly: no split holds less than a sub-block less than another
     subs = -(-L // 16)
@@ -242,9 +242,11 @@ def test_decode_plan_covers_the_sequence(B, Hq, Hkv, L):
 
 
 def test_decode_plan_examples():
-    assert _plan(64, 32, 8, 32768)[1:] == (2048, 16)
-    assert _plan(1, 32, 1, 131072)[1:] == (1024, 128)  # 2 head chunks x 128 splits
-    assert _plan(1, 32, 8, 131072)[1:] == (2048, 64)
+    assert _plan(64, 32, 8, 32768)[1:] == (2048, 16)  # enough (sequence, head) units: 2048-token splits
+    # few units: whole waves of two resident CTAs per SM (296 on 148 SMs)
+    assert _plan(1, 32, 8, 131072)[1:] == (3552, 37)   # 8 units x 37 splits = 296 CTAs, one wave
+    assert _plan(1, 32, 32, 131072)[1:] == (3552, 37)  # 32 units x 37 splits = 4 waves
+    assert _plan(1, 32, 1, 131072)[1:] == (912, 144)   # 2 head chunks x 144 splits (12 x 12 two-level merge)
     assert _plan(64, 32, 8, 4128)[1:] == (1376, 3)  # a 4096 window + 4 sinks: 258 sub-blocks in 3 even splits
     assert _plan(0, 32, 1, 131072)[0] == _lib.ATTN_ERR_INVALID_ARG
     assert _plan(1, 32, 3, 100)[0] == _lib.ATTN_ERR_INVALID_ARG

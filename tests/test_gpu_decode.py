@@ -182,3 +182,45 @@ def test_full_size_sampled(name):
     seqs = sorted(set([0, B - 1] + rng.integers(0, B, 3).tolist()))
     heads = sorted(set([0, Hq - 1] + rng.integers(0, Hq, 4).tolist()))
     _check(x, heads=heads, seqs=seqs, poison=False, what=name)
+
+
+# --------------------------------------------------------------------------
+# the in-launch split merge: ticket counters in a reused, never-cleared
+# workspace; two-level merges; a result that does not depend on which CTA
+# finished last
+# --------------------------------------------------------------------------
+def test_two_level_merge_single_sequence():
+    """16 query heads on one K/V head: 139 splits merged as 12 groups (the
+    last one partial), then the groups."""
+    x = workloads.paged_decode_inputs(1, 16, 1, 128, seq_lens=[40000], block_size=16, seed=21)
+    _check(x, poison=False, what="two-level merge")
+
+
+def test_workspace_reused_with_garbage_and_other_plans():
+    """The workspace is never cleared by the caller: random bytes, then the
+    leftovers of a call with another plan, must not change any result, and
+    repeated calls are bit-identical."""
+    xa = workloads.paged_decode_inputs(2, 16, 4, 128, seq_lens=[30000, 7000], block_size=16, seed=22)
+    xb = workloads.paged_decode_inputs(3, 32, 1, 64, seq_lens=[9000, 100, 25000], block_size=16, seed=23)
+    from exact_softmax_attention_causal_b200 import decode_workspace_bytes
+
+    nbytes = max(decode_workspace_bytes(2, 16, 4, 128, xa.max_seq_len, 16),
+                 decode_workspace_bytes(3, 32, 1, 64, xb.max_seq_len, 16))
+    gen = torch.Generator("cpu").manual_seed(24)
+    ws = torch.randint(0, 256, (nbytes,), generator=gen, dtype=torch.uint8).cuda()
+    a, b = _to_cuda(xa), _to_cuda(xb)
+    outs = []
+    for x, t in ((xa, a), (xb, b), (xa, a), (xb, b)):
+        o, lse = decode_paged(*t, x.max_seq_len, workspace=ws[: decode_workspace_bytes(
+            t[0].shape[0], t[0].shape[1], t[1].shape[2], t[0].shape[2], x.max_seq_len, 16)])
+        outs.append((o.clone(), lse.clone()))
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0][0], outs[2][0]) and torch.equal(outs[0][1], outs[2][1])
+    assert torch.equal(outs[1][0], outs[3][0]) and torch.equal(outs[1][1], outs[3][1])
+    for x, (o, lse) in ((xa, outs[0]), (xb, outs[1])):
+        d = x.q.shape[-1]
+        for bi in range(x.q.shape[0]):
+            heads = [0, x.q.shape[1] - 1]
+            o_ref, l_ref = oracle.decode_rows_ref(x.q, x.k_cache, x.v_cache, x.block_table, x.seq_lens, bi, heads,
+                                                  1.0 / math.sqrt(d))
+            assert_parity(o[bi, heads].cpu(), o_ref, lse[bi, heads].cpu(), l_ref, what=f"reused workspace b={bi}")

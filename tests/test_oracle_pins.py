@@ -516,3 +516,11 @@ def test_chunked_prefill_equals_full_forward(kind, w):
 def test_prefix_visible_pairs_closed_form(n_k, n_q, mask, w):
     kind = accounting.MASK_IDS[mask]
     assert accounting.prefix_visible_pairs(n_k, n_q, mask, w) == int(oracle.allowed_mask(n_q, n_k, kind, w).sum())
+
+
+@pytest.mark.parametrize("n,mask,w", [(9, "full", 0), (9, "causal", 0), (9, "window", 4), (9, "window", 20)])
+def test_row_visible_keys_sum_to_visible_pairs(n, mask, w):
+    kind = accounting.MASK_IDS[mask]
+    counts = oracle.allowed_mask(n, n, kind, w).sum(axis=1).tolist()
+    assert counts == [accounting.row_visible_keys(n, i, mask, w) for i in range(n)]
+    assert sum(counts) == accounting.visible_pairs(n, mask, w)
