@@ -201,7 +201,7 @@ __device__ void merge_partials(const DecodeParams& p, int b, int h0, int rows, i
   const int col0 = part * cpt;
   const size_t rowg = static_cast<size_t>(b) * p.Hq + h0 + (active ? r : 0);
   const int cap = DecSmem<D>::kMergeFloats / (rows * D);
-  constexpr int kQuads = D / 4;
+  constexpr int kQuads = D / 4;  // 16-byte pieces of one row
 
   float M = -INFINITY, L = 0.f;
   bool nan_seen = false;
@@ -209,17 +209,20 @@ __device__ void merge_partials(const DecodeParams& p, int b, int h0, int rows, i
 #pragma unroll
   for (int e = 0; e < kMaxCpt; ++e) acc[e] = 0.f;
 
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int c0 = 0; c0 < count; c0 += cap) {
     const int n = min(cap, count - c0);
-    const int total = n * rows * kQuads;
-    for (int i = threadIdx.x; i < total; i += kDecThreads) {
-      const int sl = i / (rows * kQuads);
-      const int rem = i - sl * rows * kQuads;
-      const int rr = rem / kQuads, c4 = rem - rr * kQuads;
+    // one warp per (slot, row): the row's D floats are contiguous in the workspace
+    for (int pi = warp; pi < n * rows; pi += kDecWarps) {
+      const int sl = pi / rows, rr = pi - sl * rows;
       const size_t src_row = (static_cast<size_t>(b) * p.Hq + h0 + rr) * p.splits + first + (c0 + sl) * stride;
-      cp_async_16(smem_u32(stage + (sl * rows + rr) * D + c4 * 4), p.o_part + src_row * D + c4 * 4, 16u);
+      const float* src = p.o_part + src_row * D;
+      const uint32_t dst = smem_u32(stage + pi * D);
+#pragma unroll
+      for (int c4 = lane; c4 < kQuads; c4 += 32) cp_async_16(dst + c4 * 16, src + c4 * 4, 16u);
     }
     cp_async_commit();
+    // the log-sum-exps: independent loads, one or two per thread, all in flight together
     for (int i = threadIdx.x; i < n * rows; i += kDecThreads) {
       const int sl = i / rows, rr = i - sl * rows;
       lse_s[i] = __ldcg(p.lse_part + (static_cast<size_t>(b) * p.Hq + h0 + rr) * p.splits + first +
@@ -587,23 +590,33 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   const int gcount = min(G, ns - gfirst);
   const int ngroups = (ns + G - 1) / G;
   float* stage = reinterpret_cast<float*>(ring);
-  __threadfence();
-  __syncthreads();  // the combine area is read above; the merge refills it
-  if (threadIdx.x == 0) *last_flag = take_last_ticket(counters + 1 + grp, p.token, gcount, p.status) ? 1 : 0;
+  // Publish, then count: the barrier orders every thread's partial stores
+  // before thread 0's device-scope release fence and ticket; the thread that
+  // takes the last ticket fences again (acquire) before the barrier that
+  // releases the CTA into the merge.
+  __syncthreads();  // also: the combine area was read above; the merge refills it
+  if (threadIdx.x == 0) {
+    fence_acq_rel_gpu();
+    const bool last = take_last_ticket(counters + 1 + grp, p.token, gcount, p.status);
+    if (last) fence_acq_rel_gpu();
+    *last_flag = last ? 1 : 0;
+  }
   __syncthreads();
   if (*last_flag == 0) return;
-  __threadfence();
   if (ngroups == 1) {
     merge_partials<D>(p, b, h0, rows, 0, ns, 1, true, stage, lse_s);
     return;
   }
   merge_partials<D>(p, b, h0, rows, gfirst, gcount, 1, false, stage, lse_s);
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) *last_flag = take_last_ticket(counters, p.token, ngroups, p.status) ? 1 : 0;
+  if (threadIdx.x == 0) {
+    fence_acq_rel_gpu();
+    const bool last = take_last_ticket(counters, p.token, ngroups, p.status);
+    if (last) fence_acq_rel_gpu();
+    *last_flag = last ? 1 : 0;
+  }
   __syncthreads();
   if (*last_flag == 0) return;
-  __threadfence();
   merge_partials<D>(p, b, h0, rows, 0, ngroups, G, true, stage, lse_s);
 }
 

@@ -37,6 +37,11 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Device-scope acquire-release fence: orders this thread's (and, through a
+// preceding bar.sync, its CTA's) earlier memory accesses before its later ones
+// for every other thread of the GPU.
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;\n" ::: "memory"); }
+
 // ----------------------------------------------------------------------------
 // cp.async (16-byte, L2-only, with zero fill when src_bytes == 0)
 // ----------------------------------------------------------------------------
