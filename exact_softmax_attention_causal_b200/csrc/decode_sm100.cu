@@ -78,6 +78,7 @@ struct DecodeParams {
   int num_blocks, block_size, max_blocks_per_seq, max_seq_len;
   int chunk, splits;
   int group_slots, ngroups;  // chunks per first-level merge group; groups per row at most
+  int merge_in_launch;       // 1: the last CTA merges; 0: every CTA leaves its partial to a merge kernel
   int window, n_sink;  // window 0: every cached token is visible (n_sink is then 0)
   uint32_t token;      // this call's tag for the ticket counters (never 0)
   float scale_log2;  // scale * log2(e): scores live in the base-2 domain
@@ -333,7 +334,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   if (u0 >= vis.nsb) return;  // split past the end of the list: nothing to read, no ticket to take
   const int nsub = min(per_split, vis.nsb - u0);
   const int ns = (vis.nsb + per_split - 1) / per_split;  // splits that hold sub-blocks of this sequence
-  const bool direct = (ns == 1);
+  // one split: this CTA writes the output itself (only when no merge kernel
+  // follows, which would otherwise merge this row's single partial)
+  const bool direct = (ns == 1) && p.merge_in_launch;
 
   if (threadIdx.x == 0) *cta_bad = 0;
   // The split's block-table entries, all requested at once (one per listed
@@ -574,7 +577,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
       }
     }
   }
-  if (direct) return;
+  if (direct || !p.merge_in_launch) return;
 
   // Split-KV merge in this launch. The chunks of the sequence are merged in
   // groups of group_slots; the CTA finishing a group last merges it (into the
@@ -843,6 +846,10 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   p.splits = plan.splits;
   p.group_slots = plan.group_slots;
   p.ngroups = plan.ngroups;
+  // One merge level: the last CTA of a (sequence, head) merges in this launch.
+  // More partials than one staging holds: a separate merge kernel spreads the
+  // rows over the whole GPU, which costs less than two in-launch levels.
+  p.merge_in_launch = plan.ngroups == 1 ? 1 : 0;
   p.window = window;
   p.n_sink = n_sink;
   p.token = token;
@@ -854,7 +861,10 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   if (e != cudaSuccess) return e;
   dim3 grid(plan.splits, Hkv * plan.hchunks, B);
   kernel<<<grid, kDecThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.merge_in_launch) return e;
+  return launch_decode_merge(p.o_part, p.lse_part, seq_lens, sinks, o, lse, B, Hq, D, plan.splits, plan.chunk,
+                             max_seq_len, window, n_sink, status, stream);
 }
 
 }  // namespace
