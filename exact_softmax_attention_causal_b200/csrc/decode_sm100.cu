@@ -946,12 +946,9 @@ int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan
     splits = (subs + 127) / 128;
   } else {
     // Few units (a single long sequence, a small batch): whole waves of
-    // resident CTAs, each split at most kDecodeMaxChunkSubs sub-blocks; with
-    // one wave, at most cap^2 splits so that a two-level merge stages each
-    // level once.
+    // resident CTAs, each split at most kDecodeMaxChunkSubs sub-blocks.
     const long long waves = (units * subs + slots * kDecodeMaxChunkSubs - 1) / (slots * kDecodeMaxChunkSubs);
     splits = waves * slots / units;
-    if (waves == 1 && splits > cap * cap) splits = cap * cap;
     const long long min_chunk_subs = 16;  // at least 256 tokens (4 sub-blocks per warp)
     splits = std::min(splits, (subs + min_chunk_subs - 1) / min_chunk_subs);
     splits = std::max(splits, (subs + kDecodeMaxChunkSubs - 1) / kDecodeMaxChunkSubs);

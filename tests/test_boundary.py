@@ -246,7 +246,7 @@ def test_decode_plan_examples():
     # few units: whole waves of two resident CTAs per SM (296 on 148 SMs)
     assert _plan(1, 32, 8, 131072)[1:] == (3552, 37)   # 8 units x 37 splits = 296 CTAs, one wave
     assert _plan(1, 32, 32, 131072)[1:] == (3552, 37)  # 32 units x 37 splits = 4 waves
-    assert _plan(1, 32, 1, 131072)[1:] == (912, 144)   # 2 head chunks x 144 splits (12 x 12 two-level merge)
+    assert _plan(1, 32, 1, 131072)[1:] == (896, 147)   # 2 head chunks x 147 splits: one wave
     assert _plan(64, 32, 8, 4128)[1:] == (1376, 3)  # a 4096 window + 4 sinks: 258 sub-blocks in 3 even splits
     assert _plan(0, 32, 1, 131072)[0] == _lib.ATTN_ERR_INVALID_ARG
     assert _plan(1, 32, 3, 100)[0] == _lib.ATTN_ERR_INVALID_ARG
