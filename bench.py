@@ -6,7 +6,10 @@ N=4096, d=128) followed by one paged decode step of 64 sequences (context
 uniform in [1024, 32768], Hq=32, Hkv=8, d=128, 16-token blocks). The headline
 `value` is the prefill's TFLOP/s (causal FLOPs: only visible pairs count);
 the decode's KV GB/s sits under "decode". Inputs are resident in HBM before
-the timed region; L2 is flushed (a 256 MiB write) before every timed kernel.
+the timed region. Before every timed prefill L2 is flushed (a 256 MiB write);
+a decode whose cache is more than twice the L2 size is timed without a flush
+(its inputs are larger than L2: nothing it reads can still be there), since the
+flush's dirty lines would otherwise be written back inside its timed region.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -326,7 +329,8 @@ def config_block(cfg, n_gpus):
     return {"workload": cfg["name"], "B": cfg["B"], "Hq": cfg["Hq"], "Hkv": cfg["Hkv"], "N": cfg["N"],
             "d": cfg["d"], "mask": cfg["mask"], "window": cfg["window"], "global_batch": cfg["B"] * n_gpus,
             "seq_len": cfg["N"], "parallelism": f"independent batch per GPU x{n_gpus}",
-            "l2": "flushed (256 MiB write) before every timed kernel"}
+            "l2": "prefill: flushed (256 MiB write) before every timed launch; decode: inputs larger than L2 "
+                  "(a cache of more than twice the L2 size, timed without a flush)"}
 
 # ----------------------------------------------------------------------------
 # the CUDA path
@@ -364,6 +368,7 @@ def run_ours(args, pcfg, dcfg):
                      dtype=torch.uint8, device=dev)
     kv_bytes = accounting.decode_kv_bytes(xd.seq_lens.tolist(), dHkv, dd)
     del xd
+    decode_flush = needs_flush(kv_bytes, dev)
 
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
@@ -374,7 +379,8 @@ def run_ours(args, pcfg, dcfg):
         attn.prefill(q, k, v, mask=pcfg["mask"], window=pcfg["window"], out=o, lse=lse)
         if ev:
             ev[1].record()
-        flush.fill_(2)
+        if decode_flush:
+            flush.fill_(2)
         if ev:
             ev[2].record()
         attn.decode_paged(dq, kc, vc, bt, sl, dcfg_max_len(dcfg), out=dout, lse=dlse, workspace=ws)
@@ -491,14 +497,14 @@ def run_ours(args, pcfg, dcfg):
     with ClockSampler(local) as clk_cfg:
         for op_name, wname in () if args.no_configs else CONFIG_SWEEP:
             op = setup_op(op_name, wname, dev, seed, peaks_all, keep_host=(rank == 0 and world == 1))
-            ms = time_launches(op["launch"], args.config_steps, 3, flush, dist_on=world > 1)
+            ms = time_launches(op["launch"], args.config_steps, 3, flush, dist_on=world > 1, do_flush=op["flush"])
             (ms_max,) = sharding.max_over_ranks([ms], device=dev)
             per_launch_s = ms / args.config_steps / 1e3
             achieved = op["work"] / per_launch_s / op["scale_div"]
             configs.append({
                 "workload": wname, "op": op_name, "unit": op["unit"],
                 "value": sharding.job_throughput(op["work"], world, args.config_steps, ms_max) / op["scale_div"],
-                "ms_per_launch": ms_max / args.config_steps, "work_per_launch": op["work"],
+                "ms_per_launch": ms_max / args.config_steps, "work_per_launch": op["work"], "l2": op["l2"],
                 "roofline": {"bound": op["bound"], "achieved": achieved, "peak": op["peak"], "unit": op["unit"],
                              "frac": achieved / op["peak"], "kernel": op["kernel"]},
             })
@@ -547,6 +553,8 @@ def run_ours(args, pcfg, dcfg):
             "decode": {
                 "metric": "paged-decode KV GB/s", "value": sharding.job_throughput(kv_bytes, world, K, d_ms) / 1e9,
                 "unit": "GB/s", "workload": dcfg["name"], "kv_bytes_per_step": kv_bytes, "ms_per_step": d_ms / K,
+                "l2": ("flushed (256 MiB write) before every timed launch" if decode_flush else
+                       f"inputs larger than L2 ({kv_bytes / 1e6:.0f} MB of K/V per launch): timed without a flush"),
                 "roofline": {"bound": "hbm", "achieved": d_gbs_launch, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                              "frac": d_gbs_launch / peaks["hbm_gbs"],
                              "traffic": recorded_traffic("decode_split_kernel", "decode_sm100.cu", kv_bytes),
@@ -716,23 +724,37 @@ def setup_op(op, name, dev, seed, peaks, keep_host=False):
     if keep_host:
         extra["host"] = x
     del x
+    # HBM-bound entry points stream `work` bytes; prefill-type launches are always flushed
+    flush_needed = True if bound == "tensor" else needs_flush(work, dev)
+    l2 = ("flushed (256 MiB write) before every timed launch" if flush_needed else
+          f"inputs larger than L2 ({work / 1e6:.0f} MB streamed per launch, more than twice the L2 size): "
+          "timed without a flush")
     return dict(launch=launch, work=work, unit=unit, bound=bound, peak=peak, scale_div=scale_div, metric=metric,
-                cfg=cfg, kernel=kernel, extra=extra)
+                cfg=cfg, kernel=kernel, extra=extra, flush=flush_needed, l2=l2)
 
 
-def time_launches(launch, steps, warmup, flush, dist_on=False):
+def needs_flush(stream_bytes, dev):
+    """An HBM-bound launch that streams more than twice the L2 capacity starts
+    cold anyway (a streamed working set that large leaves nothing reusable in
+    L2), so it is timed without a flush; anything smaller is flushed."""
+    return stream_bytes < 2 * torch.cuda.get_device_properties(dev).L2_cache_size
+
+
+def time_launches(launch, steps, warmup, flush, dist_on=False, do_flush=True):
     """CUDA-event time (ms, summed over `steps`) of launch(), each launch
-    preceded by an L2-flushing write outside the events."""
+    preceded (when do_flush) by an L2-flushing write outside the events."""
     events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for _ in range(warmup):
-        flush.fill_(1)
+        if do_flush:
+            flush.fill_(1)
         launch()
     torch.cuda.synchronize()
     if dist_on:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     for e0, e1 in events:
-        flush.fill_(1)
+        if do_flush:
+            flush.fill_(1)
         e0.record()
         launch()
         e1.record()
@@ -754,7 +776,7 @@ def run_single_op(args):
     op = setup_op(args.op, name, dev, seed, peaks)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     with ClockSampler(local) as clk:
-        ms = time_launches(op["launch"], args.steps, args.warmup, flush, dist_on=world > 1)
+        ms = time_launches(op["launch"], args.steps, args.warmup, flush, dist_on=world > 1, do_flush=op["flush"])
     (ms_max,) = sharding.max_over_ranks([ms], device=dev)
     achieved = op["work"] / (ms / args.steps / 1e3) / op["scale_div"]
     if rank == 0:
@@ -765,7 +787,7 @@ def run_single_op(args):
             "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic", "op": args.op,
             "config": dict(workload=name, **{kk: vv for kk, vv in op["cfg"].items()},
-                           l2="flushed (256 MiB write) before every timed launch"),
+                           l2=op["l2"]),
             "roofline": {"bound": op["bound"], "achieved": achieved, "peak": op["peak"], "unit": op["unit"],
                          "frac": achieved / op["peak"], "traffic": None, "peak_source": tag,
                          "kernel": op["kernel"]},
