@@ -79,6 +79,7 @@ struct DecodeParams {
   int chunk, splits;
   int group_slots, ngroups;  // chunks per first-level merge group; groups per row at most
   int merge_in_launch;       // 1: the last CTA merges; 0: every CTA leaves its partial to a merge kernel
+  int early_dependents;      // 1: let the merge kernel's CTAs launch now (they wait for this grid to finish)
   int window, n_sink;  // window 0: every cached token is visible (n_sink is then 0)
   uint32_t token;      // this call's tag for the ticket counters (never 0)
   float scale_log2;  // scale * log2(e): scores live in the base-2 domain
@@ -109,6 +110,22 @@ struct VisibleList {
 
 __device__ __forceinline__ void flag_status(int32_t* status, int bit) {
   if (status != nullptr) atomicOr(status, bit);
+}
+
+// Warp reduce-scatter of 32 columns: on entry lane l holds v[c] for its own
+// row; on exit the returned value on lane l is the sum of column l over the 32 lanes.
+__device__ __forceinline__ float warp_reduce_scatter_sum32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int k = 0; k < o; ++k) {
+      const float keep = upper ? v[k + o] : v[k];
+      const float send = upper ? v[k] : v[k + o];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return v[0];
 }
 
 // Shared memory: Q tile [16][D], then per warp kStages x (K [16][D], V [16][D]),
@@ -308,6 +325,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   int* cta_bad = reinterpret_cast<int*>(smem + L::kFlagOff);
   int* last_flag = cta_bad + 1;
 
+  // One wave followed by the merge kernel: its CTAs may take the SMs' spare
+  // room now and wait there for this grid, instead of being launched after it.
+  if (p.early_dependents) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   const int split = blockIdx.x;
   const int kvh = blockIdx.y / p.hchunks;
   const int hc = blockIdx.y % p.hchunks;
@@ -649,6 +669,7 @@ constexpr int kMergeUnroll = 4;
 // own columns of the partial outputs.
 template <int D, int COLS>
 __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const MergeParams p) {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");  // the split grid has finished and its stores are visible
   constexpr int PER = COLS / 32;  // columns per lane
   __shared__ float s_max[kMergeWarps];
   __shared__ int s_nan[kMergeWarps];
@@ -773,6 +794,121 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
   }
 }
 
+// Rows with many splits: one CTA of kMergeWarps warps per (sequence, query
+// head, 32 columns). Every thread takes one split of a round of 256: its
+// log-sum-exp and its 32 columns of the partial output are all requested at
+// once, so a round costs one memory round trip. The round's maximum comes
+// from a block reduction; each warp then sums its splits' weighted columns
+// with a reduce-scatter (lane c ends with column c), and the warps' sums are
+// added in shared memory onto the running result, rescaled between rounds
+// as in the online softmax.
+template <int D>
+__global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_wide_kernel(const MergeParams p) {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");  // the split grid has finished and its stores are visible
+  constexpr int kRound = kMergeWarps * 32;
+  __shared__ float s_max[kMergeWarps];
+  __shared__ int s_nan[kMergeWarps];
+  __shared__ float s_w[kMergeWarps];
+  __shared__ float s_acc[kMergeWarps][32];
+  const size_t row = blockIdx.x;  // b * Hq + h
+  const int c0 = static_cast<int>(blockIdx.y) * 32;
+  const bool lead = (blockIdx.y == 0);  // writes the row's LSE and status bits
+  const int b = static_cast<int>(row / p.Hq);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seq_len = p.seq_lens[b];
+  __nv_bfloat16* orow = p.o + row * D + c0;
+  if (seq_len < 1 || seq_len > p.max_seq_len) {
+    if (threadIdx.x == 0 && lead) {
+      flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
+      if (p.lse) p.lse[row] = NAN;
+    }
+    if (warp == 0) orow[lane] = __float2bfloat16_rn(NAN);
+    return;
+  }
+  const int per_split = p.chunk / kSub;
+  const int ns = (VisibleList(seq_len, p.window, p.n_sink).nsb + per_split - 1) / per_split;
+  const float* lrow = p.lse_part + row * p.splits;
+  const float* obase = p.o_part + row * p.splits * D + c0;
+  float M_run = -INFINITY, L_run = 0.f, acc_run = 0.f;  // acc_run: column `lane` (warp 0)
+  bool any_nan = false;
+  for (int s0 = 0; s0 < ns; s0 += kRound) {
+    const int s = s0 + static_cast<int>(threadIdx.x);
+    const bool valid = s < ns;
+    float v[32];
+    float x = -INFINITY;
+    if (valid) {
+      x = __ldcg(lrow + s);
+      const float4* src = reinterpret_cast<const float4*>(obase + static_cast<size_t>(s) * D);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 t = __ldcg(src + q);
+        v[4 * q] = t.x;
+        v[4 * q + 1] = t.y;
+        v[4 * q + 2] = t.z;
+        v[4 * q + 3] = t.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = 0.f;
+    }
+    // the round's maximum and NaN flag over all threads
+    const bool is_nan = (x != x);
+    float m = is_nan ? -INFINITY : x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const bool warp_nan = __any_sync(0xffffffffu, is_nan);
+    if (lane == 0) {
+      s_max[warp] = m;
+      s_nan[warp] = warp_nan ? 1 : 0;
+    }
+    __syncthreads();
+    float m_round = s_max[0];
+    int nan_round = s_nan[0];
+#pragma unroll
+    for (int w = 1; w < kMergeWarps; ++w) {
+      m_round = fmaxf(m_round, s_max[w]);
+      nan_round |= s_nan[w];
+    }
+    any_nan |= (nan_round != 0);
+    const float m_new = fmaxf(M_run, m_round);
+    // this split's weight against the running maximum; empty or NaN splits weigh 0
+    const float wgt = (x == -INFINITY || is_nan) ? 0.f : fast_exp2((x - m_new) * kLog2e);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) v[e] *= wgt;
+    const float col = warp_reduce_scatter_sum32(v, lane);  // column `lane` of this warp's splits
+    float wsum = wgt;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+    s_acc[warp][lane] = col;
+    if (lane == 0) s_w[warp] = wsum;
+    __syncthreads();
+    if (warp == 0) {
+      const float keep = (M_run == -INFINITY) ? 0.f : fast_exp2((M_run - m_new) * kLog2e);
+      float csum = 0.f, wtot = 0.f;
+#pragma unroll
+      for (int w = 0; w < kMergeWarps; ++w) {
+        csum += s_acc[w][lane];
+        wtot += s_w[w];
+      }
+      acc_run = acc_run * keep + csum;
+      L_run = L_run * keep + wtot;
+    }
+    M_run = m_new;
+    __syncthreads();  // s_max / s_acc are rewritten by the next round
+  }
+  if (warp == 0) {
+    float inv = 1.f / L_run;
+    bool bad_sink = false;
+    const float lse_out = sink_fold(p.sinks, static_cast<int>(row % p.Hq), M_run + __logf(L_run), inv, bad_sink);
+    if (bad_sink) {
+      any_nan = true;
+      if (lane == 0 && lead) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
+    }
+    orow[lane] = __float2bfloat16_rn(any_nan ? NAN : acc_run * inv);
+    if (lane == 0 && lead && p.lse) p.lse[row] = any_nan ? NAN : lse_out;
+  }
+}
+
 // Gather: out[b][h][t][:] = cache[block_table[b][t / bs]][t % bs][h][:] for
 // t < seq_lens[b], zero for the rest of [0, max_seq_len). One thread per
 // 16-byte chunk; consecutive threads walk (head, chunk) of one token, which
@@ -850,6 +986,12 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   // More partials than one staging holds: a separate merge kernel spreads the
   // rows over the whole GPU, which costs less than two in-launch levels.
   p.merge_in_launch = plan.ngroups == 1 ? 1 : 0;
+  const long long ctas = static_cast<long long>(plan.splits) * Hkv * plan.hchunks * B;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                 cudaSuccess)
+    return cudaErrorUnknown;
+  p.early_dependents = (!p.merge_in_launch && ctas <= static_cast<long long>(kDecodeCtasPerSm) * sms) ? 1 : 0;
   p.window = window;
   p.n_sink = n_sink;
   p.token = token;
@@ -864,14 +1006,15 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   e = cudaGetLastError();
   if (e != cudaSuccess || p.merge_in_launch) return e;
   return launch_decode_merge(p.o_part, p.lse_part, seq_lens, sinks, o, lse, B, Hq, D, plan.splits, plan.chunk,
-                             max_seq_len, window, n_sink, status, stream);
+                             max_seq_len, window, n_sink, status, stream, p.early_dependents != 0);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_merge(const float* o_part, const float* lse_part, const int32_t* seq_lens,
                                 const float* sinks, void* o, float* lse, int B, int Hq, int d, int splits, int chunk,
-                                int max_seq_len, int window, int n_sink, int32_t* status, cudaStream_t stream) {
+                                int max_seq_len, int window, int n_sink, int32_t* status, cudaStream_t stream,
+                                bool after_split_grid) {
   MergeParams m;
   m.o_part = o_part;
   m.lse_part = lse_part;
@@ -889,17 +1032,34 @@ cudaError_t launch_decode_merge(const float* o_part, const float* lse_part, cons
   m.n_sink = n_sink;
   // rows with many splits: 32 columns per CTA, so a single long sequence still
   // spreads its merge over many SMs
+  // rows with many splits: 32 columns per CTA, one split per thread per round
   const bool wide = splits >= 32;
   const unsigned rows = static_cast<unsigned>(B) * static_cast<unsigned>(Hq);
   const dim3 grid(rows, wide ? static_cast<unsigned>(d / 32) : 1u);
+  if (after_split_grid && wide && (d == 128 || d == 64)) {
+    // programmatic dependent launch: the split grid let these CTAs launch early;
+    // each waits (griddepcontrol.wait) until the split grid has completed
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kMergeWarps * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return d == 128 ? cudaLaunchKernelEx(&cfg, decode_merge_wide_kernel<128>, m)
+                    : cudaLaunchKernelEx(&cfg, decode_merge_wide_kernel<64>, m);
+  }
   if (d == 128)
-    wide ? decode_merge_kernel<128, 32><<<grid, kMergeWarps * 32, 0, stream>>>(m)
+    wide ? decode_merge_wide_kernel<128><<<grid, kMergeWarps * 32, 0, stream>>>(m)
          : decode_merge_kernel<128, 128><<<grid, kMergeWarps * 32, 0, stream>>>(m);
   else if (d == 64)
-    wide ? decode_merge_kernel<64, 32><<<grid, kMergeWarps * 32, 0, stream>>>(m)
+    wide ? decode_merge_wide_kernel<64><<<grid, kMergeWarps * 32, 0, stream>>>(m)
          : decode_merge_kernel<64, 64><<<grid, kMergeWarps * 32, 0, stream>>>(m);
   else if (d == 512)
-    wide ? decode_merge_kernel<512, 32><<<grid, kMergeWarps * 32, 0, stream>>>(m)
+    wide ? decode_merge_wide_kernel<512><<<grid, kMergeWarps * 32, 0, stream>>>(m)
          : decode_merge_kernel<512, 512><<<grid, kMergeWarps * 32, 0, stream>>>(m);
   else
     return cudaErrorInvalidValue;

@@ -80,9 +80,12 @@ int launch_mla_decode(const void* q, const void* cache, const int32_t* block_tab
                       int max_seq_len, float scale, void* workspace, const MlaPlan& plan, int32_t* status,
                       cudaStream_t stream);
 // The split-merge kernel of the paged decode, for head widths 64, 128 and 512.
+// after_split_grid: launched right after a decode split grid that let its
+// dependents launch early (programmatic dependent launch).
 cudaError_t launch_decode_merge(const float* o_part, const float* lse_part, const int32_t* seq_lens,
                                 const float* sinks, void* o, float* lse, int B, int Hq, int d, int splits, int chunk,
-                                int max_seq_len, int window, int n_sink, int32_t* status, cudaStream_t stream);
+                                int max_seq_len, int window, int n_sink, int32_t* status, cudaStream_t stream,
+                                bool after_split_grid = false);
 
 // Backward pass (backward_sm100.cu): workspace = D = rowsum(dO * O), fp32 [B, Hq, N].
 size_t backward_workspace_bytes(int B, int Hq, int N);

@@ -290,7 +290,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       bool ok = mbar_wait_bounded(bar(kMbQFull), 0, budget, abort_flag);
       // Tile j's scores need its slot loaded and score buffer j % 2 released by
       // the softmax of tile j - 2; its output MMAs need its P^T. Each is issued
-      // as soon as it is ready. Every barrier tested here is at most one phase
+      // as soon as it is ready: the barriers are polled with test_wait, which
+      // never suspends, so waiting on one never hides that another completed. Every barrier tested here is at most one phase
       // ahead of the phase tested (the next phase needs work issued after this
       // test), so the parity tests are unambiguous.
       int ns = 0, npv = 0;
@@ -299,8 +300,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         bool progressed = false;
         if (ns < ntiles && ns < npv + kSlots) {
           const int sl = ns % kSlots;
-          if (mbar_try_wait(bar(kMbKFull + sl), (ns / kSlots) & 1) &&
-              (ns < kSlots || mbar_try_wait(bar(kMbSFree + sl), ((ns - kSlots) / kSlots) & 1))) {
+          if (mbar_test_wait(bar(kMbKFull + sl), (ns / kSlots) & 1) &&
+              (ns < kSlots || mbar_test_wait(bar(kMbSFree + sl), ((ns - kSlots) / kSlots) & 1))) {
             tc_fence_after();
             // S^T = K . Q^T over the nine chunks, 4 steps of 16 columns each
             for (int j = 0; j < kChunks; ++j) {
@@ -318,7 +319,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         }
         if (!progressed && npv < ns) {
           const int sl = npv % kSlots;
-          if (mbar_try_wait(bar(kMbPFull + sl), (npv / kSlots) & 1)) {
+          if (mbar_test_wait(bar(kMbPFull + sl), (npv / kSlots) & 1)) {
             tc_fence_after();
             // O^T += V^T . P^T (the softmax rescaled O^T first where its max moved)
             for (int m = 0; m < 4; ++m) {
