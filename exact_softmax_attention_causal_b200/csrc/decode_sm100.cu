@@ -654,21 +654,18 @@ struct MergeParams {
   int B, Hq, splits, chunk, max_seq_len, window, n_sink;
 };
 
-// One CTA of 8 warps per (sequence, query head): lse = log sum_s exp(lse_s),
-// O = sum_s exp(lse_s - lse) O_s over the chunks that hold tokens. Warp w
-// takes chunks w, w + 8, ... four at a time (their loads are all in flight
-// before the first is used) and the warps combine their partial sums in
-// shared memory, so a single long sequence with hundreds of chunks still
-// merges in parallel. A learned sink logit joins the normaliser last (it
-// carries no value).
+// Rows with fewer than 32 splits: one CTA of 8 warps per (sequence, query
+// head): lse = log sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s over the
+// chunks that hold tokens. Warp w takes chunks w, w + 8, ... four at a time
+// (their loads are all in flight before the first is used) and the warps
+// combine their partial sums in shared memory. A learned sink logit joins the
+// normaliser last (it carries no value).
 constexpr int kMergeWarps = 8;
 constexpr int kMergeUnroll = 4;
 
-// COLS < D: the row's columns are shared out over D / COLS CTAs (blockIdx.y),
-// for rows with many splits; each reads every split's log-sum-exp and its
-// own columns of the partial outputs.
-template <int D, int COLS>
+template <int D>
 __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const MergeParams p) {
+  constexpr int COLS = D;
   asm volatile("griddepcontrol.wait;\n" ::: "memory");  // the split grid has finished and its stores are visible
   constexpr int PER = COLS / 32;  // columns per lane
   __shared__ float s_max[kMergeWarps];
@@ -676,14 +673,12 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
   __shared__ float s_sum[kMergeWarps];
   __shared__ float s_acc[kMergeWarps][COLS];
   const size_t row = blockIdx.x;  // b * Hq + h
-  const int c0 = static_cast<int>(blockIdx.y) * COLS;
-  const bool lead = (blockIdx.y == 0);  // writes the row's LSE and status bits
   const int b = static_cast<int>(row / p.Hq);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int seq_len = p.seq_lens[b];
-  __nv_bfloat16* orow = p.o + row * D + c0 + lane * PER;
+  __nv_bfloat16* orow = p.o + row * D + lane * PER;
   if (seq_len < 1 || seq_len > p.max_seq_len) {
-    if (threadIdx.x == 0 && lead) {
+    if (threadIdx.x == 0) {
       flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
       if (p.lse) p.lse[row] = NAN;
     }
@@ -723,7 +718,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  const float* obase = p.o_part + row * p.splits * D + c0 + lane * PER;
+  const float* obase = p.o_part + row * p.splits * D + lane * PER;
   for (int base = warp; base < ns; base += kMergeUnroll * kMergeWarps) {
     float ls[kMergeUnroll];
     float v[kMergeUnroll][PER];
@@ -772,7 +767,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
     const float lse_out = sink_fold(p.sinks, static_cast<int>(row % p.Hq), M + __logf(total), inv, bad_sink);
     if (bad_sink) {
       any_nan = 1;
-      if (lane == 0 && lead) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
+      if (lane == 0) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
     }
     float out[PER];
 #pragma unroll
@@ -790,7 +785,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
 #pragma unroll
       for (int e = 0; e < PER; ++e) orow[e] = __float2bfloat16_rn(out[e]);
     }
-    if (lane == 0 && lead && p.lse) p.lse[row] = any_nan ? NAN : lse_out;
+    if (lane == 0 && p.lse) p.lse[row] = any_nan ? NAN : lse_out;
   }
 }
 
@@ -1054,13 +1049,13 @@ cudaError_t launch_decode_merge(const float* o_part, const float* lse_part, cons
   }
   if (d == 128)
     wide ? decode_merge_wide_kernel<128><<<grid, kMergeWarps * 32, 0, stream>>>(m)
-         : decode_merge_kernel<128, 128><<<grid, kMergeWarps * 32, 0, stream>>>(m);
+         : decode_merge_kernel<128><<<grid, kMergeWarps * 32, 0, stream>>>(m);
   else if (d == 64)
     wide ? decode_merge_wide_kernel<64><<<grid, kMergeWarps * 32, 0, stream>>>(m)
-         : decode_merge_kernel<64, 64><<<grid, kMergeWarps * 32, 0, stream>>>(m);
+         : decode_merge_kernel<64><<<grid, kMergeWarps * 32, 0, stream>>>(m);
   else if (d == 512)
     wide ? decode_merge_wide_kernel<512><<<grid, kMergeWarps * 32, 0, stream>>>(m)
-         : decode_merge_kernel<512, 512><<<grid, kMergeWarps * 32, 0, stream>>>(m);
+         : decode_merge_kernel<512><<<grid, kMergeWarps * 32, 0, stream>>>(m);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();
