@@ -6,10 +6,13 @@ N=4096, d=128) followed by one paged decode step of 64 sequences (context
 uniform in [1024, 32768], Hq=32, Hkv=8, d=128, 16-token blocks). The headline
 `value` is the prefill's TFLOP/s (causal FLOPs: only visible pairs count);
 the decode's KV GB/s sits under "decode". Inputs are resident in HBM before
-the timed region. Before every timed prefill L2 is flushed (a 256 MiB write);
-a decode whose cache is more than twice the L2 size is timed without a flush
-(its inputs are larger than L2: nothing it reads can still be there), since the
-flush's dirty lines would otherwise be written back inside its timed region.
+the timed region. Before every timed prefill L2 is flushed (a 256 MiB write).
+An HBM-bound launch is flushed by a 256 MiB write followed by a 256 MiB read
+of another buffer, which leaves L2 holding clean lines of neither the
+workload nor the write (a write flush alone leaves dirty lines that would be
+written back inside the timed region); a decode whose cache is more than twice
+the L2 size is timed without a flush (its inputs are larger than L2: nothing it
+reads can still be there).
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -370,17 +373,17 @@ def run_ours(args, pcfg, dcfg):
     del xd
     decode_flush = needs_flush(kv_bytes, dev)
 
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     def step(ev=None):
-        flush.fill_(1)
+        flush("write")
         if ev:
             ev[0].record()
         attn.prefill(q, k, v, mask=pcfg["mask"], window=pcfg["window"], out=o, lse=lse)
         if ev:
             ev[1].record()
         if decode_flush:
-            flush.fill_(2)
+            flush("clean")
         if ev:
             ev[2].record()
         attn.decode_paged(dq, kc, vc, bt, sl, dcfg_max_len(dcfg), out=dout, lse=dlse, workspace=ws)
@@ -497,7 +500,7 @@ def run_ours(args, pcfg, dcfg):
     with ClockSampler(local) as clk_cfg:
         for op_name, wname in () if args.no_configs else CONFIG_SWEEP:
             op = setup_op(op_name, wname, dev, seed, peaks_all, keep_host=(rank == 0 and world == 1))
-            ms = time_launches(op["launch"], args.config_steps, 3, flush, dist_on=world > 1, do_flush=op["flush"])
+            ms = time_launches(op["launch"], args.config_steps, 3, flush, dist_on=world > 1, kind=op["flush"])
             (ms_max,) = sharding.max_over_ranks([ms], device=dev)
             per_launch_s = ms / args.config_steps / 1e3
             achieved = op["work"] / per_launch_s / op["scale_div"]
@@ -553,7 +556,7 @@ def run_ours(args, pcfg, dcfg):
             "decode": {
                 "metric": "paged-decode KV GB/s", "value": sharding.job_throughput(kv_bytes, world, K, d_ms) / 1e9,
                 "unit": "GB/s", "workload": dcfg["name"], "kv_bytes_per_step": kv_bytes, "ms_per_step": d_ms / K,
-                "l2": ("flushed (256 MiB write) before every timed launch" if decode_flush else
+                "l2": (FLUSH_NOTE["clean"] if decode_flush else
                        f"inputs larger than L2 ({kv_bytes / 1e6:.0f} MB of K/V per launch): timed without a flush"),
                 "roofline": {"bound": "hbm", "achieved": d_gbs_launch, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                              "frac": d_gbs_launch / peaks["hbm_gbs"],
@@ -725,12 +728,12 @@ def setup_op(op, name, dev, seed, peaks, keep_host=False):
         extra["host"] = x
     del x
     # HBM-bound entry points stream `work` bytes; prefill-type launches are always flushed
-    flush_needed = True if bound == "tensor" else needs_flush(work, dev)
-    l2 = ("flushed (256 MiB write) before every timed launch" if flush_needed else
+    kind = "write" if bound == "tensor" else ("clean" if needs_flush(work, dev) else None)
+    l2 = (FLUSH_NOTE[kind] if kind else
           f"inputs larger than L2 ({work / 1e6:.0f} MB streamed per launch, more than twice the L2 size): "
           "timed without a flush")
     return dict(launch=launch, work=work, unit=unit, bound=bound, peak=peak, scale_div=scale_div, metric=metric,
-                cfg=cfg, kernel=kernel, extra=extra, flush=flush_needed, l2=l2)
+                cfg=cfg, kernel=kernel, extra=extra, flush=kind, l2=l2)
 
 
 def needs_flush(stream_bytes, dev):
@@ -740,21 +743,46 @@ def needs_flush(stream_bytes, dev):
     return stream_bytes < 2 * torch.cuda.get_device_properties(dev).L2_cache_size
 
 
-def time_launches(launch, steps, warmup, flush, dist_on=False, do_flush=True):
+FLUSH_NOTE = {
+    "write": "flushed (256 MiB write) before every timed launch",
+    "clean": "flushed (256 MiB write, then a 256 MiB read of another buffer: no dirty line left) before every "
+             "timed launch",
+}
+
+
+class L2Flush:
+    """Evicts the workload from L2 between timed launches. "write": fill a
+    256 MiB buffer. "clean": the same write, then a read of another 256 MiB
+    buffer, so that L2 ends up holding clean lines only and the timed kernel
+    pays for no write-back of the flush's own lines."""
+
+    def __init__(self, dev):
+        self.wbuf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.rbuf = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+        self.acc = torch.empty((), dtype=torch.int64, device=dev)
+
+    def __call__(self, kind):
+        if kind is None:
+            return
+        self.wbuf.fill_(1)
+        if kind == "clean":
+            torch.sum(self.rbuf, dim=0, out=self.acc)
+
+
+def time_launches(launch, steps, warmup, flush, dist_on=False, kind="write"):
     """CUDA-event time (ms, summed over `steps`) of launch(), each launch
-    preceded (when do_flush) by an L2-flushing write outside the events."""
+    preceded by an L2 flush of the given kind (None: no flush) outside the
+    events."""
     events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for _ in range(warmup):
-        if do_flush:
-            flush.fill_(1)
+        flush(kind)
         launch()
     torch.cuda.synchronize()
     if dist_on:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     for e0, e1 in events:
-        if do_flush:
-            flush.fill_(1)
+        flush(kind)
         e0.record()
         launch()
         e1.record()
@@ -774,9 +802,9 @@ def run_single_op(args):
     tag = "of measured" if peaks["source"] == "measured" else "of fallback"
     name = args.workload
     op = setup_op(args.op, name, dev, seed, peaks)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     with ClockSampler(local) as clk:
-        ms = time_launches(op["launch"], args.steps, args.warmup, flush, dist_on=world > 1, do_flush=op["flush"])
+        ms = time_launches(op["launch"], args.steps, args.warmup, flush, dist_on=world > 1, kind=op["flush"])
     (ms_max,) = sharding.max_over_ranks([ms], device=dev)
     achieved = op["work"] / (ms / args.steps / 1e3) / op["scale_div"]
     if rank == 0:

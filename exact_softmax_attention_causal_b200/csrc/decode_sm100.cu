@@ -14,9 +14,12 @@
 // K and V through a private 3-stage cp.async ring in shared memory (16-byte
 // loads of whole 256-byte head rows), score the <= 16 query heads of the
 // group against them with mma.sync m16n8k16 (bf16 in, fp32 accumulate), and
-// keep FlashAttention's running (max, sum, output) per query head. The warps
-// combine in shared memory and write one normalised partial output and its
-// log-sum-exp per (sequence, head, chunk). The CTA that finishes last among
+// keep FlashAttention's running (max, sum, output) per query head. With 17 to
+// 32 query heads per K/V head (MQA) a CTA takes 32 heads with 8 warps: each
+// pair of warps streams the sub-blocks through one shared 6-stage ring and
+// scores 16 heads per warp, so the tiles are read once for all the heads.
+// The warps combine in shared memory and write one normalised partial output
+// and its log-sum-exp per (sequence, head, chunk). The CTA that finishes last among
 // the chunks of a (sequence, K/V head, head chunk) combines them with the
 // online softmax's rescaling and writes the output, in the same launch (a
 // ticket counter in the workspace tells each CTA whether it is the last).
@@ -51,10 +54,33 @@
 namespace attn {
 namespace {
 
-constexpr int kDecWarps = 4;
-constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kStages = 3;  // per-warp ring depth
+constexpr int kGroups = 4;  // token groups of a split CTA: group t streams sub-blocks t, t + 4, ...
 constexpr int kSub = 16;    // tokens per sub-block
+// Lazy rescaling (FlashAttention-4): a row's running maximum, and with it the
+// rescaling of its output accumulator, is only moved when a new score exceeds
+// it by more than this many factors of 2; until then the probabilities are
+// taken against the stale maximum (at most 2^8, exact in the final
+// normalisation, which divides by a sum taken against the same maximum).
+constexpr float kDecRescaleLog2 = 8.0f;
+// Run-time work split (one-wave plans without a window, 16 heads per CTA):
+// the sequence's sub-blocks form grains of kDecGrainSubs; every warp starts
+// with two fixed grains and then takes the next free one from a counter, so
+// that warps on SMs that stream faster take more of the sequence.
+constexpr int kDecGrainSubs = 2;
+
+// A split CTA covers HC chunks of 16 query heads of one K/V head. HC = 1: one
+// warp per token group, each with a private 3-stage ring (two CTAs per SM).
+// HC = 2 (17 to 32 query heads per K/V head, e.g. MQA): a pair of warps per
+// token group shares one 6-stage ring, each warp scoring its own 16 heads
+// against the same K/V tiles, so every tile crosses into the SM once for all
+// 32 heads (one CTA of 8 warps per SM).
+template <int HC>
+struct DecShape {
+  static constexpr int kWarps = kGroups * HC;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kStages = HC == 1 ? 3 : 6;
+  static constexpr int kRows = 16 * HC;  // query-head rows of a CTA
+};
 
 struct DecodeParams {
   const __nv_bfloat16* q;
@@ -64,8 +90,9 @@ struct DecodeParams {
   const int32_t* seq_lens;
   float* o_part;    // [B, Hq, splits, D]
   float* lse_part;  // [B, Hq, splits]
-  // Ticket counters, (1 + ngroups) per (sequence, K/V head, head chunk):
-  // [0] counts the merged groups, [1 + g] the finished chunks of group g.
+  // Counters, (2 + ngroups) per (sequence, K/V head, head chunk): [0] counts
+  // the merged groups, [1 + g] the finished chunks of group g, [1 + ngroups]
+  // hands out grains (DYN kernels).
   unsigned long long* counters;
   // Sequences whose visible sub-blocks fit one split are written directly by
   // that split's CTA (normalised, learned sink folded in); the others by the
@@ -81,7 +108,8 @@ struct DecodeParams {
   int merge_in_launch;       // 1: the last CTA merges; 0: every CTA leaves its partial to a merge kernel
   int early_dependents;      // 1: let the merge kernel's CTAs launch now (they wait for this grid to finish)
   int window, n_sink;  // window 0: every cached token is visible (n_sink is then 0)
-  uint32_t token;      // this call's tag for the ticket counters (never 0)
+  int dyn;             // 1: grains of kDecGrainSubs sub-blocks handed out at run time (DYN kernels)
+  uint32_t token;      // this call's tag for the ticket and grain counters (never 0)
   float scale_log2;  // scale * log2(e): scores live in the base-2 domain
 };
 
@@ -128,31 +156,34 @@ __device__ __forceinline__ float warp_reduce_scatter_sum32(float (&v)[32], int l
   return v[0];
 }
 
-// Shared memory: Q tile [16][D], then per warp kStages x (K [16][D], V [16][D]),
-// then the split's block-table entries (one per listed sub-block), the merge's
-// staged log-sum-exps and two flags.
+// Shared memory: Q tile [16 * HC][D], then per token group kStages x (K [16][D],
+// V [16][D]), then the split's block-table entries (one per listed sub-block),
+// the merge's staged log-sum-exps and two flags.
 // Rows are 16-byte-chunk swizzled: chunk c of row r lives at chunk c ^ (r & 7),
 // which makes every ldmatrix phase hit 8 distinct bank groups.
 // After the main loop the ring holds the warps' partial results and then the
 // partial outputs a merge reads: kMergeFloats floats, i.e. kMergeFloats / (rows * D)
 // chunks of `rows` query heads at a time (192 / rows, whatever D is).
-template <int D>
+template <int D, int HC>
 struct DecSmem {
+  using S = DecShape<HC>;
   static constexpr int kRowBytes = D * 2;
   static constexpr int kChunks = kRowBytes / 16;
   static constexpr int kTile = kSub * kRowBytes;
-  static constexpr int kRing = kDecWarps * kStages * 2 * kTile;
-  static constexpr int kMergeFloats = kRing / 4;
-  static constexpr int kMergeLse = kMergeFloats / D;  // staged log-sum-exps (chunks x rows) at most
-  static constexpr int kPhysOff = kTile + kRing;
+  static constexpr int kQBytes = S::kRows * kRowBytes;
+  static constexpr int kRing = kGroups * S::kStages * 2 * kTile;
+  static constexpr int kMergeFloats = kDecodeMergeSlots * D;
+  static constexpr int kCombineFloats = kGroups * S::kRows * (2 + D);  // per token group: m, l, O rows
+  static constexpr int kPhysOff = kQBytes + kRing;
   static constexpr int kLseOff = kPhysOff + kDecodeMaxChunkSubs * 4;
-  static constexpr int kFlagOff = kLseOff + kMergeLse * 4;
+  static constexpr int kFlagOff = kLseOff + kDecodeMergeSlots * 4;
   static constexpr int kTotal = kFlagOff + 16;
+  static_assert(kMergeFloats * 4 <= kRing && kCombineFloats * 4 <= kRing,
+                "the ring holds the combine area and one merge staging");
 };
-static_assert(DecSmem<128>::kMergeLse == kDecodeMergeSlots && DecSmem<64>::kMergeLse == kDecodeMergeSlots,
-              "a merge staging holds kDecodeMergeSlots rows of D floats");
-static_assert(kDecodeCtasPerSm * (DecSmem<128>::kTotal + 1024) <= 228 * 1024,
+static_assert(kDecodeCtasPerSm * (DecSmem<128, 1>::kTotal + 1024) <= 228 * 1024,
               "the split plan counts on two resident CTAs per SM at d = 128");
+static_assert(DecSmem<128, 2>::kTotal <= 227 * 1024, "a paired CTA fits one SM at d = 128");
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk, int row_bytes) {
   return static_cast<uint32_t>(row * row_bytes + ((chunk ^ (row & 7)) << 4));
@@ -161,36 +192,41 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk, int row_bytes) {
 // Final output of one row from its unnormalised sum (already divided by the
 // token sum: `inv`) and the tokens' log-sum-exp; folds a learned sink logit
 // into the normaliser. Returns the natural-log LSE written for the row.
-__device__ __forceinline__ float sink_fold(const float* sinks, int h, float lse_tok, float& scale_out, bool& bad) {
-  if (sinks == nullptr) return lse_tok;
-  const float sk = sinks[h];
+__device__ __forceinline__ float sink_fold_value(float sk, float lse_tok, float& scale_out, bool& bad) {
   if (!(fabsf(sk) <= 3.0e38f)) bad = true;  // NaN or infinite sink logit
   const float hi = fmaxf(lse_tok, sk), lo = fminf(lse_tok, sk);
   const float lse_all = hi + log1pf(__expf(lo - hi));
   scale_out *= __expf(lse_tok - lse_all);
   return lse_all;
 }
+__device__ __forceinline__ float sink_fold(const float* sinks, int h, float lse_tok, float& scale_out, bool& bad) {
+  return sinks == nullptr ? lse_tok : sink_fold_value(sinks[h], lse_tok, scale_out, bad);
+}
 
-// One ticket on a counter shared by `expected` CTAs of this launch; true for
-// the CTA that takes the last one. The counter's high 32 bits hold the tag of
-// the call that last counted on it: a different tag (another call, or memory
-// that was never a counter) counts as zero, so the workspace needs no
-// clearing. The last CTA puts the counter back to 0. A compare-and-swap fails
-// only when another CTA's ticket succeeded in between, and each of the other
-// expected - 1 CTAs takes exactly one, so the loop ends within `expected`
-// tries; its bound is a guard, on expiry the timeout bit is set.
-__device__ __forceinline__ bool take_last_ticket(unsigned long long* c, uint32_t token, int expected,
-                                                 int32_t* status) {
+// One ticket on a counter this call has claimed (claim_counter), shared by
+// `expected` CTAs of this launch: true for the CTA that takes the last one.
+// A single atomic add, whatever the number of CTAs finishing at once.
+__device__ __forceinline__ bool take_ticket(unsigned long long* c, int expected) {
+  const unsigned long long old = atomicAdd(c, 1ull);
+  return static_cast<int>(old & 0xffffffffull) + 1 == expected;
+}
+
+// Makes a workspace counter this call's before the CTA counts on it. The
+// counter's high 32 bits hold the tag of the call that last claimed it: a
+// different tag (another call, or memory that was never a counter) is
+// replaced by (tag, 0), so the workspace needs no clearing, and once any CTA
+// of this call has claimed it the others leave it as it is (their counts are
+// never lost). A compare-and-swap fails only when another CTA of this call
+// claimed or counted in between, after which the tag is this call's, so the
+// loop ends within two tries; its bound is a guard, on expiry the timeout bit
+// is set and the CTA does not count on the counter.
+__device__ __forceinline__ bool claim_counter(unsigned long long* c, uint32_t token, int32_t* status) {
   const unsigned long long tag = static_cast<unsigned long long>(token) << 32;
   unsigned long long cur = atomicAdd(c, 0ull);
-  for (int i = 0; i < 2 * expected + 8; ++i) {
-    const unsigned long long want = ((cur >> 32) == token) ? cur + 1ull : (tag | 1ull);
-    const unsigned long long prev = atomicCAS(c, cur, want);
-    if (prev == cur) {
-      const bool last = static_cast<int>(want & 0xffffffffull) == expected;
-      if (last) atomicExch(c, 0ull);
-      return last;
-    }
+  for (int i = 0; i < 64; ++i) {
+    if ((cur >> 32) == token) return true;
+    const unsigned long long prev = atomicCAS(c, cur, tag);
+    if (prev == cur) return true;
     cur = prev;
   }
   flag_status(status, ATTN_STATUS_BIT_TIMEOUT);
@@ -205,20 +241,20 @@ __device__ __forceinline__ bool take_last_ticket(unsigned long long* c, uint32_t
 // time, and combined with the online softmax's rescaling between stagings.
 // With `to_output` the row is normalised, the learned sink folded in and O
 // (bf16) and LSE written; otherwise the merged partial goes back into slot
-// `first`. Called by all threads of the CTA.
-template <int D>
+// `first`. Called by all NT threads of the CTA.
+template <int D, int NT>
 __device__ void merge_partials(const DecodeParams& p, int b, int h0, int rows, int first, int count, int stride,
                                bool to_output, float* stage, float* lse_s) {
   constexpr int kMaxCpt = D / 8;
   int tpr = D / 4;  // threads per row: a power of two, at least 8
-  while (tpr * rows > kDecThreads) tpr >>= 1;
+  while (tpr * rows > NT) tpr >>= 1;
   const int cpt = D / tpr;  // columns per thread, a multiple of 4
   const int r = threadIdx.x / tpr;
   const int part = threadIdx.x % tpr;
   const bool active = r < rows;
   const int col0 = part * cpt;
   const size_t rowg = static_cast<size_t>(b) * p.Hq + h0 + (active ? r : 0);
-  const int cap = DecSmem<D>::kMergeFloats / (rows * D);
+  const int cap = kDecodeMergeSlots / rows;
   constexpr int kQuads = D / 4;  // 16-byte pieces of one row
 
   float M = -INFINITY, L = 0.f;
@@ -231,7 +267,7 @@ __device__ void merge_partials(const DecodeParams& p, int b, int h0, int rows, i
   for (int c0 = 0; c0 < count; c0 += cap) {
     const int n = min(cap, count - c0);
     // one warp per (slot, row): the row's D floats are contiguous in the workspace
-    for (int pi = warp; pi < n * rows; pi += kDecWarps) {
+    for (int pi = warp; pi < n * rows; pi += NT / 32) {
       const int sl = pi / rows, rr = pi - sl * rows;
       const size_t src_row = (static_cast<size_t>(b) * p.Hq + h0 + rr) * p.splits + first + (c0 + sl) * stride;
       const float* src = p.o_part + src_row * D;
@@ -241,7 +277,7 @@ __device__ void merge_partials(const DecodeParams& p, int b, int h0, int rows, i
     }
     cp_async_commit();
     // the log-sum-exps: independent loads, one or two per thread, all in flight together
-    for (int i = threadIdx.x; i < n * rows; i += kDecThreads) {
+    for (int i = threadIdx.x; i < n * rows; i += NT) {
       const int sl = i / rows, rr = i - sl * rows;
       lse_s[i] = __ldcg(p.lse_part + (static_cast<size_t>(b) * p.Hq + h0 + rr) * p.splits + first +
                         (c0 + sl) * stride);
@@ -313,17 +349,26 @@ __device__ void merge_partials(const DecodeParams& p, int b, int h0, int rows, i
 
 // WIN: the sequence is read through the visible-sub-block list (sliding window,
 // sink positions); without it every cached token is visible and the list
-// arithmetic folds away at compile time.
-template <int D, bool WIN>
-__global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeParams p) {
-  using L = DecSmem<D>;
+// arithmetic folds away at compile time. HC: 16-head chunks per CTA (DecShape).
+// DYN: the split's sub-blocks are handed out as grains at run time (HC = 1,
+// no window); every CTA of a (sequence, K/V head) then writes a partial.
+template <int D, bool WIN, int HC, bool DYN>
+__global__ void __launch_bounds__(DecShape<HC>::kThreads) decode_split_kernel(const DecodeParams p) {
+  static_assert(!DYN || (HC == 1 && !WIN), "run-time grains: 16 heads per CTA, no window");
+  using L = DecSmem<D, HC>;
+  using Sh = DecShape<HC>;
+  constexpr int NT = Sh::kThreads;
+  constexpr int kStages = Sh::kStages;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* q_s = smem;
-  uint8_t* ring = smem + L::kTile;
+  uint8_t* ring = smem + L::kQBytes;
   int* phys_s = reinterpret_cast<int*>(smem + L::kPhysOff);
   float* lse_s = reinterpret_cast<float*>(smem + L::kLseOff);
   int* cta_bad = reinterpret_cast<int*>(smem + L::kFlagOff);
   int* last_flag = cta_bad + 1;
+  int* grain_ok = cta_bad + 2;
+  int* tickets_ok = cta_bad + 3;
+  int* dtok = reinterpret_cast<int*>(smem + L::kPhysOff);  // DYN: first token per (warp, stage), -1: no tile
 
   // One wave followed by the merge kernel: its CTAs may take the SMs' spare
   // room now and wait there for this grid, instead of being launched after it.
@@ -334,14 +379,71 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   const int b = blockIdx.z;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int h0 = kvh * p.group + hc * 16;
-  const int rows = min(16, p.group - hc * 16);
+  const int h0 = kvh * p.group + hc * Sh::kRows;
+  const int rows = min(Sh::kRows, p.group - hc * Sh::kRows);
+  // the learned sink logit of the row this thread finishes (row tid / 8 of the
+  // combine below), requested now so that its latency hides behind the split
+  const float sink_pre =
+      (p.sinks != nullptr && static_cast<int>(threadIdx.x >> 3) < rows) ? __ldg(p.sinks + h0 + (threadIdx.x >> 3)) : 0.f;
+
+  // Requests that do not depend on the sequence length go out with its read:
+  // the Q rows and, without a window, the split's block-table entries (its
+  // sub-blocks are then positions 16 u0 .. in order; entries past the
+  // sequence are read but never used, and stay inside the table's row).
+  const int per_split = p.chunk / kSub;
+  const int u0 = split * per_split;  // this split's listed sub-blocks [u0, u0 + nsub)
+  constexpr int kQPer = (Sh::kRows * L::kChunks + NT - 1) / NT;
+  uint4 qv[kQPer];
+#pragma unroll
+  for (int k = 0; k < kQPer; ++k) {
+    const int i = threadIdx.x + k * NT;
+    const int r = i / L::kChunks, c = i % L::kChunks;
+    qv[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (i < Sh::kRows * L::kChunks && r < rows)
+      qv[k] = *reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.Hq + h0 + r) * D + c * 8);
+  }
+  constexpr int kTabPer = (kDecodeMaxChunkSubs + NT - 1) / NT;
+  int tab[kTabPer];
+  // DYN: the block-table entries of this warp's two fixed grains, lane l < kDecGrainSubs
+  // holding sub-block l of grain g_cur (ph_a) and of grain g_nxt (ph_b).
+  const int n_fixed = p.splits * Sh::kWarps;  // fixed grains per round: one per warp of the sequence's CTAs
+  int g_cur = split * Sh::kWarps + warp;
+  int g_nxt = g_cur + n_fixed;
+  int ph_a = -1, ph_b = -1;
+  unsigned long long* grain_ctr = nullptr;
+  if constexpr (DYN) {
+    const int subs_max = (p.max_seq_len + kSub - 1) / kSub;
+    const int32_t* trow = p.block_table + static_cast<size_t>(b) * p.max_blocks_per_seq;
+    const int ua = g_cur * kDecGrainSubs + lane, ub = g_nxt * kDecGrainSubs + lane;
+    if (lane < kDecGrainSubs && ua < subs_max) ph_a = __ldg(trow + ua * kSub / p.block_size);
+    if (lane < kDecGrainSubs && ub < subs_max) ph_b = __ldg(trow + ub * kSub / p.block_size);
+    grain_ctr = p.counters + (static_cast<size_t>(b) * gridDim.y + blockIdx.y) * (2 + p.ngroups) + 1 + p.ngroups;
+    if (threadIdx.x == 64) *grain_ok = claim_counter(grain_ctr, p.token, p.status) ? 1 : 0;
+  } else if constexpr (!WIN) {
+    const int subs_max = (p.max_seq_len + kSub - 1) / kSub;
+#pragma unroll
+    for (int k = 0; k < kTabPer; ++k) {
+      const int i = threadIdx.x + k * NT;
+      tab[k] = (i < per_split && u0 + i < subs_max)
+                   ? __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks_per_seq + (u0 + i) * kSub / p.block_size)
+                   : -1;
+    }
+  }
+
+  // The in-launch merge's ticket counters (this split's group, and the
+  // groups' counter when there are several), claimed by two other warps while
+  // the loads above are in flight.
+  unsigned long long* counters = p.counters + (static_cast<size_t>(b) * gridDim.y + blockIdx.y) * (2 + p.ngroups);
+  if (p.merge_in_launch) {
+    if (threadIdx.x == 0) *last_flag = claim_counter(counters + 1 + split / p.group_slots, p.token, p.status) ? 1 : 0;
+    if (threadIdx.x == 32) *tickets_ok = (p.ngroups == 1 || claim_counter(counters, p.token, p.status)) ? 1 : 0;
+  }
 
   const int seq_len = p.seq_lens[b];
   if (seq_len < 1 || seq_len > p.max_seq_len) {
     // the first split's CTA writes the NaN rows of this head chunk
     if (split == 0) {
-      for (int i = threadIdx.x; i < rows * D; i += kDecThreads)
+      for (int i = threadIdx.x; i < rows * D; i += NT)
         p.o[(static_cast<size_t>(b) * p.Hq + h0 + i / D) * D + i % D] = __float2bfloat16_rn(NAN);
       if (threadIdx.x < rows && p.lse != nullptr) p.lse[static_cast<size_t>(b) * p.Hq + h0 + threadIdx.x] = NAN;
       if (threadIdx.x == 0) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
@@ -349,53 +451,123 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
     return;
   }
   const VisibleList vis(seq_len, WIN ? p.window : 0, WIN ? p.n_sink : 0);
-  const int per_split = p.chunk / kSub;
-  const int u0 = split * per_split;  // this split's listed sub-blocks [u0, u0 + nsub)
-  if (u0 >= vis.nsb) return;  // split past the end of the list: nothing to read, no ticket to take
-  const int nsub = min(per_split, vis.nsb - u0);
-  const int ns = (vis.nsb + per_split - 1) / per_split;  // splits that hold sub-blocks of this sequence
+  // split past the end of the list: nothing to read, no ticket to take (with
+  // DYN every CTA may receive grains and writes a partial, empty or not)
+  if (!DYN && u0 >= vis.nsb) return;
+  const int nsub = DYN ? 0 : min(per_split, vis.nsb - u0);
+  // partials of this sequence: the splits that hold its sub-blocks, or every split with DYN
+  const int ns = DYN ? p.splits : (vis.nsb + per_split - 1) / per_split;
+  const int n_grains = (vis.nsb + kDecGrainSubs - 1) / kDecGrainSubs;
   // one split: this CTA writes the output itself (only when no merge kernel
   // follows, which would otherwise merge this row's single partial)
   const bool direct = (ns == 1) && p.merge_in_launch;
 
   if (threadIdx.x == 0) *cta_bad = 0;
-  // The split's block-table entries, all requested at once (one per listed
-  // sub-block), so that no cache copy waits on a table read later.
-  for (int i = threadIdx.x; i < nsub; i += kDecThreads) {
-    const int lblk = vis.token0(u0 + i) / p.block_size;
-    phys_s[i] = __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks_per_seq + lblk);
+  // The split's block-table entries, one per listed sub-block, in shared
+  // memory before any cache copy is issued (with a window they depend on the
+  // sequence length and are requested now, all at once).
+  if constexpr (DYN) {
+  } else if constexpr (!WIN) {
+#pragma unroll
+    for (int k = 0; k < kTabPer; ++k) {
+      const int i = threadIdx.x + k * NT;
+      if (i < nsub) phys_s[i] = tab[k];
+    }
+  } else {
+    for (int i = threadIdx.x; i < nsub; i += NT) {
+      const int lblk = vis.token0(u0 + i) / p.block_size;
+      phys_s[i] = __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks_per_seq + lblk);
+    }
   }
   // Q rows of this head chunk -> swizzled shared tile; padding rows are zero.
-  for (int i = threadIdx.x; i < 16 * L::kChunks; i += kDecThreads) {
-    const int r = i / L::kChunks, c = i % L::kChunks;
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (r < rows)
-      val = *reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.Hq + h0 + r) * D + c * 8);
-    *reinterpret_cast<uint4*>(q_s + swz(r, c, L::kRowBytes)) = val;
+#pragma unroll
+  for (int k = 0; k < kQPer; ++k) {
+    const int i = threadIdx.x + k * NT;
+    if (i < Sh::kRows * L::kChunks)
+      *reinterpret_cast<uint4*>(q_s + swz(i / L::kChunks, i % L::kChunks, L::kRowBytes)) = qv[k];
   }
   __syncthreads();
 
-  // Per-warp streaming over sub-blocks warp, warp + 4, ...
-  uint8_t* my_ring = ring + warp * kStages * 2 * L::kTile;
-  const int n_my = (nsub > warp) ? (nsub - warp + kDecWarps - 1) / kDecWarps : 0;
+  // Token group tg streams sub-blocks tg, tg + 4, ... through its ring; with
+  // HC = 2 its two warps (hw = 0, 1) each copy half of every tile and score
+  // query-head rows 16 hw .. 16 hw + 15 of the CTA against all of it.
+  const int tg = warp / HC;
+  const int hw = warp % HC;
+  uint8_t* my_ring = ring + tg * kStages * 2 * L::kTile;
+  const int n_my = (nsub > tg) ? (nsub - tg + kGroups - 1) / kGroups : 0;
   bool bad = false;
 
+  // Tile copies: the 32 * HC lanes of a token group copy 16-byte chunk c_l of
+  // rows r_l, r_l + kRowStep, ... of each 16-row K and V tile.
+  constexpr int kRowStep = 32 * HC / L::kChunks;
+  constexpr int kCopies = kSub / kRowStep;
+  static_assert(kRowStep * L::kChunks == 32 * HC && kCopies * kRowStep == kSub, "lanes tile the sub-block");
+  const int r_l = (hw * 32 + lane) / L::kChunks, c_l = (hw * 32 + lane) % L::kChunks;
+  const size_t row_elems = static_cast<size_t>(p.Hkv) * D;  // pool elements from one token to the next
+  const size_t lane_src = static_cast<size_t>(r_l) * row_elems + static_cast<size_t>(kvh) * D + c_l * 8;
+
   auto issue = [&](int j, int stage) {
-    const int i = warp + j * kDecWarps;  // sub-block of this split
+    const int i = tg + j * kGroups;  // sub-block of this split
     const int t = vis.token0(u0 + i);    // its first token
     const int lblk = t / p.block_size;
     const int off = t - lblk * p.block_size;  // multiple of 16, off + 15 < block_size
     const int phys = phys_s[i];
     const bool ok = (phys >= 0) && (phys < p.num_blocks);
     bad |= !ok;
+    const size_t base = ok ? (static_cast<size_t>(phys) * p.block_size + off) * row_elems + lane_src : 0;
     const uint32_t kdst = smem_u32(my_ring + stage * 2 * L::kTile);
 #pragma unroll
-    for (int x = lane; x < kSub * L::kChunks; x += 32) {
-      const int r = x / L::kChunks, c = x % L::kChunks;
+    for (int k = 0; k < kCopies; ++k) {
+      const int r = r_l + k * kRowStep;
       const bool valid = ok && vis.visible(t + r, seq_len);  // hidden slots are zero-filled, never read
-      const size_t src = valid ? ((static_cast<size_t>(phys) * p.block_size + off + r) * p.Hkv + kvh) * D + c * 8
-                               : 0;
-      const uint32_t dst = kdst + swz(r, c, L::kRowBytes);
+      const size_t src = valid ? base + static_cast<size_t>(k * kRowStep) * row_elems : 0;
+      const uint32_t dst = kdst + swz(r, c_l, L::kRowBytes);
+      cp_async_16(dst, p.k_cache + src, valid ? 16u : 0u);
+      cp_async_16(dst + L::kTile, p.v_cache + src, valid ? 16u : 0u);
+    }
+  };
+
+  // DYN: this warp's t-th tile is sub-block t % kDecGrainSubs of its
+  // (t / kDecGrainSubs)-th grain: the two fixed grains, then one taken from
+  // the counter per grain, two grains ahead of its use (lane 0 holds the
+  // pending ticket), with its block-table entries read one grain ahead. A
+  // grain at or past n_grains ends the warp's stream (the counter only grows,
+  // so every later one would too).
+  int grab = 0;
+  const bool may_grab = DYN && (*grain_ok != 0);
+  if (DYN && may_grab && lane == 0) grab = static_cast<int>(atomicAdd(grain_ctr, 1ull) & 0xffffffffull);
+  auto issue_dyn = [&](int t, int stage) {
+    const int off = t % kDecGrainSubs;
+    if (off == 0 && t > 0) {  // next grain
+      g_cur = g_nxt;
+      ph_a = ph_b;
+      const int taken = __shfl_sync(0xffffffffu, grab, 0);
+      g_nxt = (may_grab && g_cur < n_grains) ? 2 * n_fixed + taken : n_grains;
+      const int un = g_nxt * kDecGrainSubs + lane;
+      ph_b = (lane < kDecGrainSubs && g_nxt < n_grains && un < vis.nsb)
+                 ? __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks_per_seq + un * kSub / p.block_size)
+                 : -1;
+      if (may_grab && g_nxt < n_grains && lane == 0)
+        grab = static_cast<int>(atomicAdd(grain_ctr, 1ull) & 0xffffffffull);
+    }
+    const int u = g_cur * kDecGrainSubs + off;
+    const bool have = (g_cur < n_grains) && (u < vis.nsb);
+    if (lane == 0) dtok[warp * kStages + stage] = have ? u * kSub : -1;
+    if (!have) return;
+    const int t0 = u * kSub;
+    const int lblk = t0 / p.block_size;
+    const int boff = t0 - lblk * p.block_size;
+    const int phys = __shfl_sync(0xffffffffu, ph_a, off);
+    const bool ok = (phys >= 0) && (phys < p.num_blocks);
+    bad |= !ok;
+    const size_t base = ok ? (static_cast<size_t>(phys) * p.block_size + boff) * row_elems + lane_src : 0;
+    const uint32_t kdst = smem_u32(my_ring + stage * 2 * L::kTile);
+#pragma unroll
+    for (int k = 0; k < kCopies; ++k) {
+      const int r = r_l + k * kRowStep;
+      const bool valid = ok && (t0 + r < seq_len);
+      const size_t src = valid ? base + static_cast<size_t>(k * kRowStep) * row_elems : 0;
+      const uint32_t dst = kdst + swz(r, c_l, L::kRowBytes);
       cp_async_16(dst, p.k_cache + src, valid ? 16u : 0u);
       cp_async_16(dst + L::kTile, p.v_cache + src, valid ? 16u : 0u);
     }
@@ -403,7 +575,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
 
 #pragma unroll
   for (int j = 0; j < kStages - 1; ++j) {
-    if (j < n_my) issue(j, j);
+    if constexpr (DYN) {
+      issue_dyn(j, j);
+    } else {
+      if (j < n_my) issue(j, j);
+    }
     cp_async_commit();
   }
 
@@ -411,7 +587,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   uint32_t qf[D / 16][4];
   {
     const uint32_t qb = smem_u32(q_s);
-    const int r = lane & 15;
+    const int r = hw * 16 + (lane & 15);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const int c = kk * 2 + (lane >> 4);
@@ -428,28 +604,51 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
 
   const int g = lane >> 2, tq = lane & 3;
 
-  for (int j = 0; j < n_my; ++j) {
-    const int jn = j + kStages - 1;
-    if (jn < n_my) issue(jn, jn % kStages);
-    cp_async_commit();
-    cp_async_wait<kStages - 1>();
-    __syncwarp();
+  for (int j = 0; DYN || j < n_my; ++j) {
+    if constexpr (DYN) {
+      issue_dyn(j + kStages - 1, (j + kStages - 1) % kStages);
+      cp_async_commit();
+      cp_async_wait<kStages - 1>();
+      __syncwarp();
+      if (dtok[warp * kStages + j % kStages] < 0) break;  // no tile j: the stream has ended
+    } else if constexpr (HC == 1) {
+      const int jn = j + kStages - 1;
+      if (jn < n_my) issue(jn, jn % kStages);
+      cp_async_commit();
+      cp_async_wait<kStages - 1>();
+      __syncwarp();
+    } else {
+      // This thread's copies of tile j have landed; the pair barrier makes the
+      // partner's half visible and tells that the partner is done with tile
+      // j - 1, whose stage the next copy overwrites.
+      cp_async_wait<kStages - 2>();
+      asm volatile("bar.sync %0, %1;\n" ::"r"(1 + tg), "r"(32 * HC) : "memory");
+      const int jn = j + kStages - 1;
+      if (jn < n_my) issue(jn, jn % kStages);
+      cp_async_commit();
+    }
 
     const uint32_t kb = smem_u32(my_ring + (j % kStages) * 2 * L::kTile);
     const uint32_t vb = kb + L::kTile;
-    const int tok0 = vis.token0(u0 + warp + j * kDecWarps);
+    const int tok0 = DYN ? dtok[warp * kStages + j % kStages] : vis.token0(u0 + tg + j * kGroups);
 
-    // S = Q K^T for 16 tokens: two n-tiles of 8 tokens.
+    // S = Q K^T for 16 tokens: two n-tiles of 8 tokens, each summed in two
+    // independent accumulator chains (even and odd k steps).
     float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float s_odd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const int r = ((lane >> 4) << 3) + (lane & 7);
       const int c = kk * 2 + ((lane >> 3) & 1);
       uint32_t b00, b01, b10, b11;
       ldmatrix_x4(kb + swz(r, c, L::kRowBytes), b00, b01, b10, b11);
-      mma_bf16_16816(s[0], qf[kk], b00, b01);
-      mma_bf16_16816(s[1], qf[kk], b10, b11);
+      mma_bf16_16816((kk & 1) ? s_odd[0] : s[0], qf[kk], b00, b01);
+      mma_bf16_16816((kk & 1) ? s_odd[1] : s[1], qf[kk], b10, b11);
     }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[nt][e] += s_odd[nt][e];
     // scale into base 2, mask slots that are not visible
     float mx[2] = {neg_inf, neg_inf};
 #pragma unroll
@@ -467,14 +666,28 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
       mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
       mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
     }
-    // every listed sub-block holds a visible token, so mx is finite
-    float alpha[2];
+    // Every listed sub-block holds a visible token, so mx is finite. The
+    // maxima move (and the accumulators are rescaled) only when a row's new
+    // score exceeds its maximum by more than kDecRescaleLog2, always on the
+    // first sub-block (m_run = -inf); the test is warp-wide so that the
+    // rescaling stays one branch for the warp.
+    const bool grow = (mx[0] > m_run[0] + kDecRescaleLog2) || (mx[1] > m_run[1] + kDecRescaleLog2);
+    if (__any_sync(0xffffffffu, grow)) {
+      float alpha[2];
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      const float m_new = fmaxf(m_run[rr], mx[rr]);
-      alpha[rr] = fast_exp2(m_run[rr] - m_new);  // 0 on the first sub-block (m_run = -inf)
-      m_run[rr] = m_new;
-      l_run[rr] *= alpha[rr];
+      for (int rr = 0; rr < 2; ++rr) {
+        const float m_new = fmaxf(m_run[rr], mx[rr]);
+        alpha[rr] = fast_exp2(m_run[rr] - m_new);  // 0 on the first sub-block (m_run = -inf)
+        m_run[rr] = m_new;
+        l_run[rr] *= alpha[rr];
+      }
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) {
+        o_acc[n][0] *= alpha[0];
+        o_acc[n][1] *= alpha[0];
+        o_acc[n][2] *= alpha[1];
+        o_acc[n][3] *= alpha[1];
+      }
     }
     float pr[2][4];
 #pragma unroll
@@ -489,13 +702,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
     pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
     pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
     pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      o_acc[n][0] *= alpha[0];
-      o_acc[n][1] *= alpha[0];
-      o_acc[n][2] *= alpha[1];
-      o_acc[n][3] *= alpha[1];
-    }
     // O += P V: V rows are tokens (k), columns are the head dim (n) -> trans loads.
 #pragma unroll
     for (int n = 0; n < D / 8; n += 2) {
@@ -518,21 +724,24 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   if (bad) atomicOr(cta_bad, 1);
   __syncthreads();  // every warp is done with its ring: reuse it for the combine
 
-  // Combine the 4 warps: per warp m[16], l[16], O[16][D] (unnormalised, fp32).
+  // Combine the token groups: per group m[R], l[R], O[R][D] (unnormalised,
+  // fp32) for the CTA's R = 16 * HC query-head rows.
+  constexpr int R = Sh::kRows;
   float* wm = reinterpret_cast<float*>(ring);
-  float* wl = wm + kDecWarps * 16;
-  float* wo = wl + kDecWarps * 16;
+  float* wl = wm + kGroups * R;
+  float* wo = wl + kGroups * R;
+  const int r0 = tg * R + hw * 16 + g;  // this lane's first row in the combine area
   if (tq == 0) {
-    wm[warp * 16 + g] = m_run[0];
-    wm[warp * 16 + g + 8] = m_run[1];
-    wl[warp * 16 + g] = l_run[0];
-    wl[warp * 16 + g + 8] = l_run[1];
+    wm[r0] = m_run[0];
+    wm[r0 + 8] = m_run[1];
+    wl[r0] = l_run[0];
+    wl[r0 + 8] = l_run[1];
   }
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) {
     const int col = n * 8 + 2 * tq;
-    float* w0 = wo + (warp * 16 + g) * D + col;
-    float* w1 = wo + (warp * 16 + g + 8) * D + col;
+    float* w0 = wo + r0 * D + col;
+    float* w1 = wo + (r0 + 8) * D + col;
     w0[0] = o_acc[n][0];
     w0[1] = o_acc[n][1];
     w1[0] = o_acc[n][2];
@@ -542,25 +751,27 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
 
   const bool cta_is_bad = (*cta_bad != 0);
   if (cta_is_bad && threadIdx.x == 0) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
-  // 128 threads: thread -> (row = tid / 8, 8 threads per row, D / 8 columns each)
+  // thread -> (row = tid / 8, 8 threads per row, D / 8 columns each)
   {
     const int r = threadIdx.x >> 3;
     const int part = threadIdx.x & 7;
     if (r < rows) {
       float M = neg_inf;
 #pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, wm[w * 16 + r]);
-      float wsc[kDecWarps];
+      for (int w = 0; w < kGroups; ++w) M = fmaxf(M, wm[w * R + r]);
+      float wsc[kGroups];
       float Lsum = 0.f;
 #pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) {
-        wsc[w] = (wm[w * 16 + r] == neg_inf) ? 0.f : fast_exp2(wm[w * 16 + r] - M);
-        Lsum += wsc[w] * wl[w * 16 + r];
+      for (int w = 0; w < kGroups; ++w) {
+        wsc[w] = (wm[w * R + r] == neg_inf) ? 0.f : fast_exp2(wm[w * R + r] - M);
+        Lsum += wsc[w] * wl[w * R + r];
       }
-      float inv = 1.f / Lsum;
+      // a CTA that received no grain (DYN) leaves an empty partial: O = 0, LSE = -inf
+      float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
       if (direct) {
         bool bad_row = cta_is_bad;
-        const float lse_out = sink_fold(p.sinks, h0 + r, (M + __log2f(Lsum)) * kLn2, inv, bad_row);
+        const float lse_tok = (M + __log2f(Lsum)) * kLn2;
+        const float lse_out = p.sinks != nullptr ? sink_fold_value(sink_pre, lse_tok, inv, bad_row) : lse_tok;
         if (bad_row && part == 0 && !cta_is_bad) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
         __nv_bfloat16* dst = p.o + (static_cast<size_t>(b) * p.Hq + h0 + r) * D;
         for (int c = part * (D / 8); c < (part + 1) * (D / 8); c += 8) {
@@ -569,9 +780,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
           for (int e = 0; e < 8; e += 2) {
             float v0 = 0.f, v1 = 0.f;
 #pragma unroll
-            for (int w = 0; w < kDecWarps; ++w) {
-              v0 += wsc[w] * wo[(w * 16 + r) * D + c + e];
-              v1 += wsc[w] * wo[(w * 16 + r) * D + c + e + 1];
+            for (int w = 0; w < kGroups; ++w) {
+              v0 += wsc[w] * wo[(w * R + r) * D + c + e];
+              v1 += wsc[w] * wo[(w * R + r) * D + c + e + 1];
             }
             pk[e >> 1] = pack_bf16x2(bad_row ? NAN : v0 * inv, bad_row ? NAN : v1 * inv);
           }
@@ -588,12 +799,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
           for (int e = 0; e < 4; ++e) {
             float v = 0.f;
 #pragma unroll
-            for (int w = 0; w < kDecWarps; ++w) v += wsc[w] * wo[(w * 16 + r) * D + c + e];
+            for (int w = 0; w < kGroups; ++w) v += wsc[w] * wo[(w * R + r) * D + c + e];
             a[e] = cta_is_bad ? NAN : v * inv;
           }
           *reinterpret_cast<float4*>(dst + c) = acc;
         }
-        if (part == 0) p.lse_part[prow] = cta_is_bad ? NAN : (M + __log2f(Lsum)) * kLn2;
+        if (part == 0) p.lse_part[prow] = cta_is_bad ? NAN : (Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : -INFINITY);
       }
     }
   }
@@ -605,8 +816,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   // and the CTA finishing the last group merges the groups. Partial results
   // are published with a device-scope fence before the ticket and read after
   // one (through L2), so the merging CTA sees every other CTA's stores.
-  unsigned long long* counters =
-      p.counters + (static_cast<size_t>(b) * gridDim.y + blockIdx.y) * (1 + p.ngroups);
   const int G = p.group_slots;
   const int grp = split / G;
   const int gfirst = grp * G;
@@ -617,30 +826,32 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   // before thread 0's device-scope release fence and ticket; the thread that
   // takes the last ticket fences again (acquire) before the barrier that
   // releases the CTA into the merge.
+  // *last_flag and *tickets_ok hold the claims' outcomes (written before the
+  // barriers above); a CTA whose claim ran out takes no ticket.
   __syncthreads();  // also: the combine area was read above; the merge refills it
   if (threadIdx.x == 0) {
     fence_acq_rel_gpu();
-    const bool last = take_last_ticket(counters + 1 + grp, p.token, gcount, p.status);
+    const bool last = (*last_flag != 0) && take_ticket(counters + 1 + grp, gcount);
     if (last) fence_acq_rel_gpu();
     *last_flag = last ? 1 : 0;
   }
   __syncthreads();
   if (*last_flag == 0) return;
   if (ngroups == 1) {
-    merge_partials<D>(p, b, h0, rows, 0, ns, 1, true, stage, lse_s);
+    merge_partials<D, NT>(p, b, h0, rows, 0, ns, 1, true, stage, lse_s);
     return;
   }
-  merge_partials<D>(p, b, h0, rows, gfirst, gcount, 1, false, stage, lse_s);
+  merge_partials<D, NT>(p, b, h0, rows, gfirst, gcount, 1, false, stage, lse_s);
   __syncthreads();
   if (threadIdx.x == 0) {
     fence_acq_rel_gpu();
-    const bool last = take_last_ticket(counters, p.token, ngroups, p.status);
+    const bool last = (*tickets_ok != 0) && take_ticket(counters, ngroups);
     if (last) fence_acq_rel_gpu();
     *last_flag = last ? 1 : 0;
   }
   __syncthreads();
   if (*last_flag == 0) return;
-  merge_partials<D>(p, b, h0, rows, 0, ngroups, G, true, stage, lse_s);
+  merge_partials<D, NT>(p, b, h0, rows, 0, ngroups, G, true, stage, lse_s);
 }
 
 struct MergeParams {
@@ -652,6 +863,7 @@ struct MergeParams {
   float* lse;
   int32_t* status;
   int B, Hq, splits, chunk, max_seq_len, window, n_sink;
+  int all_splits;  // every split wrote a partial (run-time grains)
 };
 
 // Rows with fewer than 32 splits: one CTA of 8 warps per (sequence, query
@@ -688,7 +900,8 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_kernel(const Me
     return;
   }
   const int per_split = p.chunk / kSub;
-  const int ns = (VisibleList(seq_len, p.window, p.n_sink).nsb + per_split - 1) / per_split;
+  const int ns =
+      p.all_splits ? p.splits : (VisibleList(seq_len, p.window, p.n_sink).nsb + per_split - 1) / per_split;
   const float* lrow = p.lse_part + row * p.splits;
   // global max over the chunks
   float M = -INFINITY;
@@ -821,7 +1034,8 @@ __global__ void __launch_bounds__(kMergeWarps * 32) decode_merge_wide_kernel(con
     return;
   }
   const int per_split = p.chunk / kSub;
-  const int ns = (VisibleList(seq_len, p.window, p.n_sink).nsb + per_split - 1) / per_split;
+  const int ns =
+      p.all_splits ? p.splits : (VisibleList(seq_len, p.window, p.n_sink).nsb + per_split - 1) / per_split;
   const float* lrow = p.lse_part + row * p.splits;
   const float* obase = p.o_part + row * p.splits * D + c0;
   float M_run = -INFINITY, L_run = 0.f, acc_run = 0.f;  // acc_run: column `lane` (warp 0)
@@ -986,22 +1200,31 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
                                                  cudaSuccess)
     return cudaErrorUnknown;
-  p.early_dependents = (!p.merge_in_launch && ctas <= static_cast<long long>(kDecodeCtasPerSm) * sms) ? 1 : 0;
+  const long long resident = static_cast<long long>(kDecodeCtasPerSm) * sms * 16 / plan.cta_rows;
+  p.early_dependents = (!p.merge_in_launch && ctas <= resident) ? 1 : 0;
   p.window = window;
   p.n_sink = n_sink;
   p.token = token;
   p.scale_log2 = scale * kLog2e;
 
-  const int smem = DecSmem<D>::kTotal;
-  const auto kernel = window > 0 ? decode_split_kernel<D, true> : decode_split_kernel<D, false>;
+  const bool paired = plan.cta_rows == 32;
+  // run-time grains: one-wave plans of 16-head CTAs without a window (all the
+  // CTAs of a sequence run at once, so the faster ones can take over work)
+  p.dyn = (plan.dyn && !paired && window == 0 && plan.splits > 1 && ctas <= resident) ? 1 : 0;
+  const int smem = paired ? DecSmem<D, 2>::kTotal : DecSmem<D, 1>::kTotal;
+  const int threads = paired ? DecShape<2>::kThreads : DecShape<1>::kThreads;
+  const auto kernel =
+      paired ? (window > 0 ? decode_split_kernel<D, true, 2, false> : decode_split_kernel<D, false, 2, false>)
+             : (window > 0 ? decode_split_kernel<D, true, 1, false>
+                           : (p.dyn ? decode_split_kernel<D, false, 1, true> : decode_split_kernel<D, false, 1, false>));
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.splits, Hkv * plan.hchunks, B);
-  kernel<<<grid, kDecThreads, smem, stream>>>(p);
+  kernel<<<grid, threads, smem, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess || p.merge_in_launch) return e;
   return launch_decode_merge(p.o_part, p.lse_part, seq_lens, sinks, o, lse, B, Hq, D, plan.splits, plan.chunk,
-                             max_seq_len, window, n_sink, status, stream, p.early_dependents != 0);
+                             max_seq_len, window, n_sink, status, stream, p.early_dependents != 0, p.dyn != 0);
 }
 
 }  // namespace
@@ -1009,7 +1232,7 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
 cudaError_t launch_decode_merge(const float* o_part, const float* lse_part, const int32_t* seq_lens,
                                 const float* sinks, void* o, float* lse, int B, int Hq, int d, int splits, int chunk,
                                 int max_seq_len, int window, int n_sink, int32_t* status, cudaStream_t stream,
-                                bool after_split_grid) {
+                                bool after_split_grid, bool all_splits) {
   MergeParams m;
   m.o_part = o_part;
   m.lse_part = lse_part;
@@ -1025,9 +1248,9 @@ cudaError_t launch_decode_merge(const float* o_part, const float* lse_part, cons
   m.max_seq_len = max_seq_len;
   m.window = window;
   m.n_sink = n_sink;
-  // rows with many splits: 32 columns per CTA, so a single long sequence still
-  // spreads its merge over many SMs
-  // rows with many splits: 32 columns per CTA, one split per thread per round
+  m.all_splits = all_splits ? 1 : 0;
+  // rows with many splits: 32 columns per CTA, one split per thread per round,
+  // so that a single long sequence still spreads its merge over many SMs
   const bool wide = splits >= 32;
   const unsigned rows = static_cast<unsigned>(B) * static_cast<unsigned>(Hq);
   const dim3 grid(rows, wide ? static_cast<unsigned>(d / 32) : 1u);
@@ -1068,7 +1291,7 @@ DecodeWorkspace decode_workspace_layout(int B, int Hq, int Hkv, int d, const Dec
   w.lse_part_offset = rows * d * sizeof(float);
   w.counters_offset = (w.lse_part_offset + rows * sizeof(float) + 15) / 16 * 16;
   const size_t units = static_cast<size_t>(B) * Hkv * plan.hchunks;
-  w.bytes = w.counters_offset + units * (1 + plan.ngroups) * sizeof(unsigned long long);
+  w.bytes = w.counters_offset + units * (2 + plan.ngroups) * sizeof(unsigned long long);
   return w;
 }
 
@@ -1088,11 +1311,13 @@ int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_seq_len <= 0 || num_sms <= 0 || out == nullptr)
     return ATTN_ERR_INVALID_ARG;
   const int group = Hq / Hkv;
-  const int hchunks = (group + 15) / 16;
-  const int rows = group < 16 ? group : 16;
+  // more than 16 query heads per K/V head: CTAs of 32 heads (warp pairs), one per SM
+  const int cta_rows = group > 16 ? 32 : 16;
+  const int hchunks = (group + cta_rows - 1) / cta_rows;
+  const int rows = group < cta_rows ? group : cta_rows;
   const long long units = static_cast<long long>(B) * Hkv * hchunks;  // (sequence, K/V head, head chunk)
   const long long subs = (static_cast<long long>(max_seq_len) + 15) / 16;
-  const long long slots = static_cast<long long>(kDecodeCtasPerSm) * num_sms;  // CTAs resident at once
+  const long long slots = static_cast<long long>(kDecodeCtasPerSm) * num_sms * 16 / cta_rows;  // CTAs resident at once
   const long long cap = kDecodeMergeSlots / rows;  // partials one merge stages at a time
   long long splits;
   if (units >= slots) {
@@ -1113,7 +1338,9 @@ int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan
   const long long chunk_subs = (subs + splits - 1) / splits;
   out->chunk = static_cast<int>(16 * chunk_subs);
   out->splits = static_cast<int>((subs + chunk_subs - 1) / chunk_subs);
+  out->cta_rows = cta_rows;
   out->hchunks = hchunks;
+  out->dyn = units < slots ? 1 : 0;
   // first-level merge groups: all splits in one group when one staging holds
   // them, else near-equal groups of at most cap splits
   const long long s = out->splits;

@@ -27,13 +27,16 @@ void* tensor_map_encode_fn();
 struct DecodePlan {
   int chunk;        // tokens per split (multiple of 16, at most 16 * kDecodeMaxChunkSubs)
   int splits;       // ceil(planning length / chunk)
-  int hchunks;      // query-head chunks of <= 16 per K/V head
+  int cta_rows;     // query heads a split CTA covers: 16, or 32 (warp pairs) when 16 < Hq / Hkv
+  int hchunks;      // split CTAs per (sequence, K/V head, split): ceil(Hq / Hkv / cta_rows)
   int group_slots;  // splits per first-level merge group
   int ngroups;      // ceil(splits / group_slots)
+  int dyn;          // 1: few (sequence, K/V head) units, whole waves: grains handed out at run time
 };
-// Split plan constants: resident decode CTAs per SM (two fit in shared memory
-// at d = 128), the most 16-token sub-blocks per split, and the partials one
-// merge staging holds for one query-head row (divided by the rows merged).
+// Split plan constants: resident decode CTAs of 16 query heads per SM (two
+// fit in shared memory at d = 128; one CTA of 32 heads takes both places), the
+// most 16-token sub-blocks per split, and the partials one merge staging holds
+// for one query-head row (divided by the rows merged).
 constexpr int kDecodeCtasPerSm = 2;
 constexpr int kDecodeMaxChunkSubs = 256;
 constexpr int kDecodeMergeSlots = 192;
@@ -43,8 +46,8 @@ int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan
 // most tokens a windowed query's visible sub-block list can span.
 int decode_plan_length(int max_seq_len, int window, int n_sink);
 // Workspace: partial outputs [B, Hq, splits, d] fp32, partial LSEs
-// [B, Hq, splits] fp32, then (16-byte aligned) the merge's ticket counters,
-// 1 + ngroups uint64 per (sequence, K/V head, head chunk).
+// [B, Hq, splits] fp32, then (16-byte aligned) the merge's ticket counters and
+// the grain counter, 2 + ngroups uint64 per (sequence, K/V head, head chunk).
 struct DecodeWorkspace {
   size_t o_part_offset, lse_part_offset, counters_offset, bytes;
 };
@@ -81,11 +84,13 @@ int launch_mla_decode(const void* q, const void* cache, const int32_t* block_tab
                       cudaStream_t stream);
 // The split-merge kernel of the paged decode, for head widths 64, 128 and 512.
 // after_split_grid: launched right after a decode split grid that let its
-// dependents launch early (programmatic dependent launch).
+// dependents launch early (programmatic dependent launch). all_splits: every
+// split wrote a partial (the decode's run-time grains), not just the splits
+// that hold the sequence's sub-blocks.
 cudaError_t launch_decode_merge(const float* o_part, const float* lse_part, const int32_t* seq_lens,
                                 const float* sinks, void* o, float* lse, int B, int Hq, int d, int splits, int chunk,
                                 int max_seq_len, int window, int n_sink, int32_t* status, cudaStream_t stream,
-                                bool after_split_grid = false);
+                                bool after_split_grid = false, bool all_splits = false);
 
 // Backward pass (backward_sm100.cu): workspace = D = rowsum(dO * O), fp32 [B, Hq, N].
 size_t backward_workspace_bytes(int B, int Hq, int N);

@@ -157,11 +157,12 @@ ATTN_API int attn_prefill_paged(const void* q, const void* k_cache, const void* 
  * GPU needed). Long sequences are cut into chunks of *chunk_tokens tokens
  * (a multiple of 16); each (sequence, K/V head, chunk) is one unit of work
  * ("Inference attention" post, "FlashDecoding": split keys along the
- * sequence so that small batches fill the GPU). With at least two (sequence,
- * K/V head, 16-head chunk) units per SM the chunks are 2048 tokens; with fewer
- * (a single long sequence, a small batch) the chunk count fills whole waves
- * of two resident CTAs per SM, each chunk at most 4096 tokens. num_sms is the
- * device's SM count. Returns ATTN_OK or ATTN_ERR_INVALID_ARG.
+ * sequence so that small batches fill the GPU). A unit covers 16 query
+ * heads of a K/V head, or 32 when Hq / Hkv is above 16 (one such CTA takes
+ * the place of two). With at least two units per SM the chunks are 2048
+ * tokens; with fewer (a single long sequence, a small batch) the chunk count
+ * fills whole waves of resident CTAs, each chunk at most 4096 tokens. num_sms
+ * is the device's SM count. Returns ATTN_OK or ATTN_ERR_INVALID_ARG.
  */
 ATTN_API int attn_decode_plan(int B, int Hq, int Hkv, int max_seq_len, int num_sms, int* chunk_tokens, int* num_splits);
 
@@ -169,7 +170,8 @@ ATTN_API int attn_decode_plan(int B, int Hq, int Hkv, int max_seq_len, int num_s
  * attn_decode_workspace_bytes - bytes of device workspace attn_decode_paged
  * needs for these sizes on the current device (partial outputs fp32
  * [B, Hq, splits, d], partial log-sum-exp fp32 [B, Hq, splits], then the
- * split merge's ticket counters, a few uint64 per (sequence, K/V head)).
+ * split merge's ticket counters and a work counter, a few uint64 per
+ * (sequence, K/V head)).
  * Returns 0 for invalid sizes.
  */
 ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int max_seq_len, int block_size);
@@ -185,7 +187,15 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int m
  * cached tokens, its own K/V already appended ("USAAIO Lesson 90", part 2), so
  * no mask applies. Split partials are merged with the online softmax's
  * rescaling ("Inference attention" post, "FlashDecoding"), inside the same
- * single launch: the last CTA to finish a sequence's splits merges them.
+ * single launch: the last CTA to finish a sequence's splits merges them (a
+ * second, dependent launch merges when a sequence has more partials than one
+ * CTA stages at once).
+ *
+ * Reproducibility: a plan with fixed chunks gives bit-identical results on
+ * every call. A plan whose CTAs all fit on the GPU at once (few sequences,
+ * no window, at most 16 query heads per K/V head) hands the chunks' 32-token
+ * grains to whichever CTA is free at run time, so repeated calls agree to the
+ * rounding of a different summation order.
  *
  *   q            [B, Hq, d] bf16                            read
  *   k_cache,
@@ -200,10 +210,10 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int m
  *   max_seq_len  <= max_blocks_per_seq * block_size
  *   workspace    device scratch of at least attn_decode_workspace_bytes(...)
  *                bytes, 16-byte aligned; contents on entry are irrelevant
- *                (the merge's counters carry a 32-bit tag that changes with
- *                every call; a counter without this call's tag counts as
- *                zero). Calls whose kernels overlap on the GPU must not share
- *                a workspace.
+ *                (the counters carry a 32-bit tag that changes with every
+ *                call; a counter without this call's tag is taken as zero).
+ *                Calls whose kernels overlap on the GPU must not share a
+ *                workspace.
  *   status       device int32 or NULL.
  *
  * A referenced block-table entry outside [0, num_blocks) or a seq_len outside

@@ -65,6 +65,30 @@ def test_head_groups(hq, hkv):
     _check(x, what=f"{hq}/{hkv}")
 
 
+# More than 16 query heads per K/V head: CTAs of 32 heads whose warp pairs
+# share one ring (20 and 24 heads leave padding rows; 64 heads take two CTAs
+# per split), on both head sizes, both split-plan branches (a batch of 160
+# sequences fills the GPU with one CTA per sequence and split) and one long
+# sequence whose splits go to the merge kernel.
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("hq,hkv", [(32, 1), (64, 2), (24, 1), (64, 1)])
+def test_paired_head_groups(d, hq, hkv):
+    x = workloads.paged_decode_inputs(3, hq, hkv, d, seq_lens=[1, 75, 9000], block_size=16, seed=31,
+                                      extra_blocks=3)
+    _check(x, what=f"paired {hq}/{hkv} d={d}")
+
+
+def test_paired_batch_fills_gpu():
+    lens = [1 + (37 * i) % 2100 for i in range(160)]
+    x = workloads.paged_decode_inputs(160, 32, 1, 128, seq_lens=lens, block_size=16, seed=32)
+    _check(x, seqs=[0, 1, 57, 158, 159], poison=False, what="paired batch")
+
+
+def test_paired_single_sequence_merge_kernel():
+    x = workloads.paged_decode_inputs(1, 32, 1, 128, seq_lens=[65536 + 13], block_size=16, seed=33)
+    _check(x, poison=False, what="paired merge kernel")
+
+
 @pytest.mark.parametrize("bs", [32, 64])
 def test_block_sizes(bs):
     x = workloads.paged_decode_inputs(3, 8, 1, 128, seq_lens=[5, 1000, 777], block_size=bs, seed=3,
@@ -89,7 +113,10 @@ def test_permutation_invariance():
     vc2[perm] = vc
     bt2 = torch.where(bt >= 0, perm[bt.clamp(min=0).long()].int(), bt)
     o2, l2 = decode_paged(q, kc2, vc2, bt2, sl, x.max_seq_len)
-    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    # a one-wave plan hands out its work at run time: equal up to the rounding
+    # of the summation order
+    assert (o1.float() - o2.float()).abs().max().item() <= 2e-3
+    assert (l1 - l2).abs().max().item() <= 1e-4
 
 
 def test_gather_bit_exact():
@@ -189,6 +216,27 @@ def test_full_size_sampled(name):
 # workspace; two-level merges; a result that does not depend on which CTA
 # finished last
 # --------------------------------------------------------------------------
+def test_fixed_split_plan_is_bit_reproducible():
+    """A batch that fills the GPU takes 2048-token splits fixed by the plan:
+    repeated calls are bit-identical."""
+    lens = [1 + (911 * i) % 9000 for i in range(80)]
+    x = workloads.paged_decode_inputs(80, 8, 4, 128, seq_lens=lens, block_size=16, seed=25)
+    t = _to_cuda(x)
+    o1, l1 = decode_paged(*t, x.max_seq_len)
+    o2, l2 = decode_paged(*t, x.max_seq_len)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_run_time_grains_cover_every_token():
+    """One-wave plans hand out grains of two sub-blocks at run time: short and
+    long sequences of one batch (most CTAs of the short ones receive no
+    grain), the last grain partial, lengths around grain edges."""
+    x = workloads.paged_decode_inputs(4, 16, 4, 128, seq_lens=[1, 31, 33, 50001], block_size=16, seed=26,
+                                      extra_blocks=2)
+    _check(x, what="run-time grains")
+
+
 def test_two_level_merge_single_sequence():
     """16 query heads on one K/V head: 139 splits merged as 12 groups (the
     last one partial), then the groups."""
@@ -198,8 +246,11 @@ def test_two_level_merge_single_sequence():
 
 def test_workspace_reused_with_garbage_and_other_plans():
     """The workspace is never cleared by the caller: random bytes, then the
-    leftovers of a call with another plan, must not change any result, and
-    repeated calls are bit-identical."""
+    leftovers of a call with another plan, must not change any result.
+    Repeated calls of a plan with fixed splits (here the 32-head CTAs) are
+    bit-identical; a one-wave plan of 16-head CTAs hands out its work at run
+    time, so its repeats agree to the rounding of a different summation
+    order (both match the oracle)."""
     xa = workloads.paged_decode_inputs(2, 16, 4, 128, seq_lens=[30000, 7000], block_size=16, seed=22)
     xb = workloads.paged_decode_inputs(3, 32, 1, 64, seq_lens=[9000, 100, 25000], block_size=16, seed=23)
     from exact_softmax_attention_causal_b200 import decode_workspace_bytes
@@ -215,9 +266,10 @@ def test_workspace_reused_with_garbage_and_other_plans():
             t[0].shape[0], t[0].shape[1], t[1].shape[2], t[0].shape[2], x.max_seq_len, 16)])
         outs.append((o.clone(), lse.clone()))
     torch.cuda.synchronize()
-    assert torch.equal(outs[0][0], outs[2][0]) and torch.equal(outs[0][1], outs[2][1])
+    assert (outs[0][0].float() - outs[2][0].float()).abs().max().item() <= 2e-3
+    assert (outs[0][1] - outs[2][1]).abs().max().item() <= 1e-4
     assert torch.equal(outs[1][0], outs[3][0]) and torch.equal(outs[1][1], outs[3][1])
-    for x, (o, lse) in ((xa, outs[0]), (xb, outs[1])):
+    for x, (o, lse) in ((xa, outs[0]), (xb, outs[1]), (xa, outs[2]), (xb, outs[3])):
         d = x.q.shape[-1]
         for bi in range(x.q.shape[0]):
             heads = [0, x.q.shape[1] - 1]

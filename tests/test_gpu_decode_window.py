@@ -84,6 +84,14 @@ def test_block_sizes(bs):
     _check(x, 100, 4, x.sinks, what=f"bs={bs}")
 
 
+@pytest.mark.parametrize("window,n_sink,with_sinks", [(128, 0, True), (100, 4, True), (1000, 16, False)])
+def test_paired_heads(window, n_sink, with_sinks):
+    """32 query heads on one K/V head: the warp-pair CTAs with a window."""
+    x = workloads.paged_decode_inputs(4, 32, 1, 128, seq_lens=[1, 130, 1200, 7000], block_size=16, seed=17,
+                                      learned_sinks=with_sinks)
+    _check(x, window, n_sink, x.sinks if with_sinks else None, what=f"paired w={window}")
+
+
 def test_gptoss_shape_window128_with_sinks():
     """gpt-oss local layer: 64 query heads over 8 K/V heads, head_dim 64,
     window 128, one learned sink per head."""
@@ -92,13 +100,17 @@ def test_gptoss_shape_window128_with_sinks():
     _check(x, 128, 0, x.sinks, what="gpt-oss")
 
 
-def test_window_covering_everything_equals_plain_decode_bitwise():
+def test_window_covering_everything_equals_plain_decode():
+    """A window at least as long as every sequence hides nothing: the same
+    kernel as the plain decode runs (this one-wave plan hands out its work at
+    run time, so the results agree up to the rounding of the summation order)."""
     x = workloads.paged_decode_inputs(3, 8, 2, 128, seq_lens=[7, 300, 2000], block_size=16, seed=12)
     q, kc, vc, bt, sl = (t.cuda() for t in (x.q, x.k_cache, x.v_cache, x.block_table, x.seq_lens))
     o_ref, l_ref = decode_paged(q, kc, vc, bt, sl, x.max_seq_len)
     for window, n_sink in ((0, 0), (x.max_seq_len, 0), (x.max_seq_len + 5, 3)):
         o, lse = decode_paged_window(q, kc, vc, bt, sl, x.max_seq_len, window=window, n_sink=n_sink)
-        assert torch.equal(o, o_ref) and torch.equal(lse, l_ref), (window, n_sink)
+        assert (o.float() - o_ref.float()).abs().max().item() <= 2e-3, (window, n_sink)
+        assert (lse - l_ref).abs().max().item() <= 1e-4, (window, n_sink)
 
 
 def test_evicted_middle_blocks_are_never_read():
