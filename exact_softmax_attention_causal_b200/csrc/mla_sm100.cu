@@ -364,6 +364,32 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     for (int c = 0; c < 32; ++c) l_part[c] = 0.f;
     float m_lane = -INFINITY;  // lane c: the max head column 32 hh + c's exponentials use (base 2)
     named_sync(1 + hh, 128);
+    if (hb * kNH + hh * 32 >= p.H) {
+      // A column half with no head of this block (H < 64 or a partial last block):
+      // its P^T columns are zero for every tile, written once the score MMAs have
+      // read the tile's positional chunk; nothing else is computed or stored.
+      bool idle_ok = true;
+      for (int i = 0; i < ntiles; ++i) {
+        const int sb = i % kSlots;
+        if (idle_ok)
+          idle_ok =
+              __all_sync(0xffffffffu, mbar_wait_bounded(bar(kMbSFull + sb), (i / kSlots) & 1, budget, abort_flag));
+        if (!idle_ok) continue;
+        if (lane == 0) mbar_arrive(bar(kMbSFree + sb));
+        if (lane < 16) {
+          uint8_t* pslot = smem + kKOff + sb * kTileBytes + kPSlot * kKChunkBytes;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = hh * 4 + q;
+            *reinterpret_cast<uint4*>(pslot + tok * 128 + ((chunk ^ (tok & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kMbPFull + sb));
+      }
+      if (!idle_ok) mla_abort(abort_flag, p.status);
+    } else {
     // Every softmax warp takes part in every named barrier of every tile, also
     // after a wait gave up (ok == false: it then skips its TMEM and mbarrier
     // work), so no warp can be left waiting at a barrier the others skipped.
@@ -482,6 +508,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
           p.o_part[((static_cast<size_t>(b) * p.H + head0 + c) * p.splits + split) * kDc + m * 128 + r] =
               out_ok ? __uint_as_float(ov[c]) * inv : NAN;
       }
+    }
     }
   }
 
