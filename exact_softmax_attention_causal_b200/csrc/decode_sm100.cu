@@ -22,9 +22,11 @@
 // and its log-sum-exp per (sequence, head, chunk). The CTA that finishes last among
 // the chunks of a (sequence, K/V head, head chunk) combines them with the
 // online softmax's rescaling and writes the output, in the same launch (a
-// ticket counter in the workspace tells each CTA whether it is the last).
-// Many chunks are combined in two levels: groups of chunks first, then the
-// groups.
+// ticket counter in the workspace tells each CTA whether it is the last);
+// more chunks than one CTA stages at once are combined by a merge kernel that
+// spreads the rows over the GPU. When every CTA of a sequence is resident at
+// once (few sequences, 16-head CTAs, no window) the chunks' 32-token grains
+// are handed out at run time, so that SMs served faster by HBM take more.
 //
 // The kernel is HBM-bound: each K/V byte of a (sequence, K/V head) is read
 // once and shared by the whole query-head group.
@@ -90,9 +92,8 @@ struct DecodeParams {
   const int32_t* seq_lens;
   float* o_part;    // [B, Hq, splits, D]
   float* lse_part;  // [B, Hq, splits]
-  // Counters, (2 + ngroups) per (sequence, K/V head, head chunk): [0] counts
-  // the merged groups, [1 + g] the finished chunks of group g, [1 + ngroups]
-  // hands out grains (DYN kernels).
+  // Counters, two per (sequence, K/V head, head chunk): [0] counts the
+  // finished chunks (the merge in the launch), [1] hands out grains (DYN).
   unsigned long long* counters;
   // Sequences whose visible sub-blocks fit one split are written directly by
   // that split's CTA (normalised, learned sink folded in); the others by the
@@ -104,7 +105,6 @@ struct DecodeParams {
   int B, Hq, Hkv, group, hchunks;
   int num_blocks, block_size, max_blocks_per_seq, max_seq_len;
   int chunk, splits;
-  int group_slots, ngroups;  // chunks per first-level merge group; groups per row at most
   int merge_in_launch;       // 1: the last CTA merges; 0: every CTA leaves its partial to a merge kernel
   int early_dependents;      // 1: let the merge kernel's CTAs launch now (they wait for this grid to finish)
   int window, n_sink;  // window 0: every cached token is visible (n_sink is then 0)
@@ -233,18 +233,17 @@ __device__ __forceinline__ bool claim_counter(unsigned long long* c, uint32_t to
   return false;
 }
 
-// Merge `count` partial results (slots first, first + stride, ...) of `rows`
-// query-head rows into one: lse = log sum_s exp(lse_s), O = sum_s
+// Merge the `count` partial results (slots 0 .. count - 1) of `rows`
+// query-head rows into the output: lse = log sum_s exp(lse_s), O = sum_s
 // exp(lse_s - lse) O_s ("Inference attention" post, "FlashDecoding"). The
 // partials are staged in shared memory with cp.async (L2 only: they were
-// written by other CTAs of this launch), kMergeFloats / (rows * D) slots at a
-// time, and combined with the online softmax's rescaling between stagings.
-// With `to_output` the row is normalised, the learned sink folded in and O
-// (bf16) and LSE written; otherwise the merged partial goes back into slot
-// `first`. Called by all NT threads of the CTA.
+// written by other CTAs of this launch), kDecodeMergeSlots / rows slots at a
+// time, and combined with the online softmax's rescaling between stagings;
+// the row is then normalised, the learned sink folded in and O (bf16) and LSE
+// written. Called by all NT threads of the CTA.
 template <int D, int NT>
-__device__ void merge_partials(const DecodeParams& p, int b, int h0, int rows, int first, int count, int stride,
-                               bool to_output, float* stage, float* lse_s) {
+__device__ void merge_partials(const DecodeParams& p, int b, int h0, int rows, int count, float* stage,
+                               float* lse_s) {
   constexpr int kMaxCpt = D / 8;
   int tpr = D / 4;  // threads per row: a power of two, at least 8
   while (tpr * rows > NT) tpr >>= 1;
@@ -269,7 +268,7 @@ __device__ void merge_partials(const DecodeParams& p, int b, int h0, int rows, i
     // one warp per (slot, row): the row's D floats are contiguous in the workspace
     for (int pi = warp; pi < n * rows; pi += NT / 32) {
       const int sl = pi / rows, rr = pi - sl * rows;
-      const size_t src_row = (static_cast<size_t>(b) * p.Hq + h0 + rr) * p.splits + first + (c0 + sl) * stride;
+      const size_t src_row = (static_cast<size_t>(b) * p.Hq + h0 + rr) * p.splits + c0 + sl;
       const float* src = p.o_part + src_row * D;
       const uint32_t dst = smem_u32(stage + pi * D);
 #pragma unroll
@@ -279,8 +278,7 @@ __device__ void merge_partials(const DecodeParams& p, int b, int h0, int rows, i
     // the log-sum-exps: independent loads, one or two per thread, all in flight together
     for (int i = threadIdx.x; i < n * rows; i += NT) {
       const int sl = i / rows, rr = i - sl * rows;
-      lse_s[i] = __ldcg(p.lse_part + (static_cast<size_t>(b) * p.Hq + h0 + rr) * p.splits + first +
-                        (c0 + sl) * stride);
+      lse_s[i] = __ldcg(p.lse_part + (static_cast<size_t>(b) * p.Hq + h0 + rr) * p.splits + c0 + sl);
     }
     cp_async_wait<0>();
     __syncthreads();
@@ -319,32 +317,17 @@ __device__ void merge_partials(const DecodeParams& p, int b, int h0, int rows, i
   if (!active) return;
   float inv = 1.f / L;
   const float lse_tok = M + __logf(L);
-  if (to_output) {
-    bool bad = nan_seen;
-    bool bad_sink = false;
-    const float lse_out = sink_fold(p.sinks, h0 + r, lse_tok, inv, bad_sink);
-    if (bad_sink && part == 0) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
-    bad |= bad_sink;
-    __nv_bfloat16* dst = p.o + rowg * D + col0;
+  bool bad = nan_seen;
+  bool bad_sink = false;
+  const float lse_out = sink_fold(p.sinks, h0 + r, lse_tok, inv, bad_sink);
+  if (bad_sink && part == 0) flag_status(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
+  bad |= bad_sink;
+  __nv_bfloat16* dst = p.o + rowg * D + col0;
 #pragma unroll
-    for (int e = 0; e < kMaxCpt; e += 2)
-      if (e < cpt)
-        *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(bad ? NAN : acc[e] * inv, bad ? NAN : acc[e + 1] * inv);
-    if (part == 0 && p.lse != nullptr) p.lse[rowg] = bad ? NAN : lse_out;
-  } else {
-    float* dst = p.o_part + (rowg * p.splits + first) * D + col0;
-#pragma unroll
-    for (int e = 0; e < kMaxCpt; e += 4)
-      if (e < cpt) {
-        float4 v;
-        v.x = nan_seen ? NAN : acc[e] * inv;
-        v.y = nan_seen ? NAN : acc[e + 1] * inv;
-        v.z = nan_seen ? NAN : acc[e + 2] * inv;
-        v.w = nan_seen ? NAN : acc[e + 3] * inv;
-        *reinterpret_cast<float4*>(dst + e) = v;
-      }
-    if (part == 0) p.lse_part[rowg * p.splits + first] = nan_seen ? NAN : lse_tok;
-  }
+  for (int e = 0; e < kMaxCpt; e += 2)
+    if (e < cpt)
+      *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(bad ? NAN : acc[e] * inv, bad ? NAN : acc[e + 1] * inv);
+  if (part == 0 && p.lse != nullptr) p.lse[rowg] = bad ? NAN : lse_out;
 }
 
 // WIN: the sequence is read through the visible-sub-block list (sliding window,
@@ -367,7 +350,6 @@ __global__ void __launch_bounds__(DecShape<HC>::kThreads) decode_split_kernel(co
   int* cta_bad = reinterpret_cast<int*>(smem + L::kFlagOff);
   int* last_flag = cta_bad + 1;
   int* grain_ok = cta_bad + 2;
-  int* tickets_ok = cta_bad + 3;
   int* dtok = reinterpret_cast<int*>(smem + L::kPhysOff);  // DYN: first token per (warp, stage), -1: no tile
 
   // One wave followed by the merge kernel: its CTAs may take the SMs' spare
@@ -417,7 +399,7 @@ __global__ void __launch_bounds__(DecShape<HC>::kThreads) decode_split_kernel(co
     const int ua = g_cur * kDecGrainSubs + lane, ub = g_nxt * kDecGrainSubs + lane;
     if (lane < kDecGrainSubs && ua < subs_max) ph_a = __ldg(trow + ua * kSub / p.block_size);
     if (lane < kDecGrainSubs && ub < subs_max) ph_b = __ldg(trow + ub * kSub / p.block_size);
-    grain_ctr = p.counters + (static_cast<size_t>(b) * gridDim.y + blockIdx.y) * (2 + p.ngroups) + 1 + p.ngroups;
+    grain_ctr = p.counters + (static_cast<size_t>(b) * gridDim.y + blockIdx.y) * 2 + 1;
     if (threadIdx.x == 64) *grain_ok = claim_counter(grain_ctr, p.token, p.status) ? 1 : 0;
   } else if constexpr (!WIN) {
     const int subs_max = (p.max_seq_len + kSub - 1) / kSub;
@@ -430,14 +412,10 @@ __global__ void __launch_bounds__(DecShape<HC>::kThreads) decode_split_kernel(co
     }
   }
 
-  // The in-launch merge's ticket counters (this split's group, and the
-  // groups' counter when there are several), claimed by two other warps while
-  // the loads above are in flight.
-  unsigned long long* counters = p.counters + (static_cast<size_t>(b) * gridDim.y + blockIdx.y) * (2 + p.ngroups);
-  if (p.merge_in_launch) {
-    if (threadIdx.x == 0) *last_flag = claim_counter(counters + 1 + split / p.group_slots, p.token, p.status) ? 1 : 0;
-    if (threadIdx.x == 32) *tickets_ok = (p.ngroups == 1 || claim_counter(counters, p.token, p.status)) ? 1 : 0;
-  }
+  // The in-launch merge's ticket counter, claimed while the loads above are
+  // in flight.
+  unsigned long long* tickets = p.counters + (static_cast<size_t>(b) * gridDim.y + blockIdx.y) * 2;
+  if (p.merge_in_launch && threadIdx.x == 0) *last_flag = claim_counter(tickets, p.token, p.status) ? 1 : 0;
 
   const int seq_len = p.seq_lens[b];
   if (seq_len < 1 || seq_len > p.max_seq_len) {
@@ -810,48 +788,26 @@ __global__ void __launch_bounds__(DecShape<HC>::kThreads) decode_split_kernel(co
   }
   if (direct || !p.merge_in_launch) return;
 
-  // Split-KV merge in this launch. The chunks of the sequence are merged in
-  // groups of group_slots; the CTA finishing a group last merges it (into the
-  // group's first slot, or straight into the output when there is one group),
-  // and the CTA finishing the last group merges the groups. Partial results
-  // are published with a device-scope fence before the ticket and read after
-  // one (through L2), so the merging CTA sees every other CTA's stores.
-  const int G = p.group_slots;
-  const int grp = split / G;
-  const int gfirst = grp * G;
-  const int gcount = min(G, ns - gfirst);
-  const int ngroups = (ns + G - 1) / G;
+  // Split-KV merge in this launch (the plan leaves it to the merge kernel when
+  // a sequence has more partials than one staging holds). Partial results are
+  // published with a device-scope fence before the ticket and read after one
+  // (through L2), so the merging CTA sees every other CTA's stores: the
+  // barrier orders every thread's partial stores before thread 0's release
+  // fence and ticket; the thread that takes the last ticket fences again
+  // (acquire) before the barrier that releases the CTA into the merge.
+  // *last_flag holds the counter claim's outcome (written before the barriers
+  // above); a CTA whose claim ran out takes no ticket.
   float* stage = reinterpret_cast<float*>(ring);
-  // Publish, then count: the barrier orders every thread's partial stores
-  // before thread 0's device-scope release fence and ticket; the thread that
-  // takes the last ticket fences again (acquire) before the barrier that
-  // releases the CTA into the merge.
-  // *last_flag and *tickets_ok hold the claims' outcomes (written before the
-  // barriers above); a CTA whose claim ran out takes no ticket.
   __syncthreads();  // also: the combine area was read above; the merge refills it
   if (threadIdx.x == 0) {
     fence_acq_rel_gpu();
-    const bool last = (*last_flag != 0) && take_ticket(counters + 1 + grp, gcount);
+    const bool last = (*last_flag != 0) && take_ticket(tickets, ns);
     if (last) fence_acq_rel_gpu();
     *last_flag = last ? 1 : 0;
   }
   __syncthreads();
   if (*last_flag == 0) return;
-  if (ngroups == 1) {
-    merge_partials<D, NT>(p, b, h0, rows, 0, ns, 1, true, stage, lse_s);
-    return;
-  }
-  merge_partials<D, NT>(p, b, h0, rows, gfirst, gcount, 1, false, stage, lse_s);
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    fence_acq_rel_gpu();
-    const bool last = (*tickets_ok != 0) && take_ticket(counters, ngroups);
-    if (last) fence_acq_rel_gpu();
-    *last_flag = last ? 1 : 0;
-  }
-  __syncthreads();
-  if (*last_flag == 0) return;
-  merge_partials<D, NT>(p, b, h0, rows, 0, ngroups, G, true, stage, lse_s);
+  merge_partials<D, NT>(p, b, h0, rows, ns, stage, lse_s);
 }
 
 struct MergeParams {
@@ -1189,12 +1145,10 @@ cudaError_t launch_decode_t(const void* q, const void* k_cache, const void* v_ca
   p.max_seq_len = max_seq_len;
   p.chunk = plan.chunk;
   p.splits = plan.splits;
-  p.group_slots = plan.group_slots;
-  p.ngroups = plan.ngroups;
-  // One merge level: the last CTA of a (sequence, head) merges in this launch.
-  // More partials than one staging holds: a separate merge kernel spreads the
-  // rows over the whole GPU, which costs less than two in-launch levels.
-  p.merge_in_launch = plan.ngroups == 1 ? 1 : 0;
+  // The last CTA of a (sequence, head chunk) merges in this launch when one
+  // staging holds all its partials; otherwise a separate merge kernel spreads
+  // the rows over the whole GPU, which costs less than two in-launch levels.
+  p.merge_in_launch = plan.merge_in_launch;
   const long long ctas = static_cast<long long>(plan.splits) * Hkv * plan.hchunks * B;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
@@ -1291,7 +1245,7 @@ DecodeWorkspace decode_workspace_layout(int B, int Hq, int Hkv, int d, const Dec
   w.lse_part_offset = rows * d * sizeof(float);
   w.counters_offset = (w.lse_part_offset + rows * sizeof(float) + 15) / 16 * 16;
   const size_t units = static_cast<size_t>(B) * Hkv * plan.hchunks;
-  w.bytes = w.counters_offset + units * (2 + plan.ngroups) * sizeof(unsigned long long);
+  w.bytes = w.counters_offset + units * 2 * sizeof(unsigned long long);
   return w;
 }
 
@@ -1341,12 +1295,8 @@ int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan
   out->cta_rows = cta_rows;
   out->hchunks = hchunks;
   out->dyn = units < slots ? 1 : 0;
-  // first-level merge groups: all splits in one group when one staging holds
-  // them, else near-equal groups of at most cap splits
-  const long long s = out->splits;
-  const long long nstage = (s + cap - 1) / cap;
-  out->group_slots = static_cast<int>((s + nstage - 1) / nstage);
-  out->ngroups = static_cast<int>((s + out->group_slots - 1) / out->group_slots);
+  // the merge in the launch stages every partial of a row at once
+  out->merge_in_launch = out->splits <= cap ? 1 : 0;
   return ATTN_OK;
 }
 

@@ -29,8 +29,7 @@ struct DecodePlan {
   int splits;       // ceil(planning length / chunk)
   int cta_rows;     // query heads a split CTA covers: 16, or 32 (warp pairs) when 16 < Hq / Hkv
   int hchunks;      // split CTAs per (sequence, K/V head, split): ceil(Hq / Hkv / cta_rows)
-  int group_slots;  // splits per first-level merge group
-  int ngroups;      // ceil(splits / group_slots)
+  int merge_in_launch;  // 1: every partial of a row fits one CTA's staging (the last CTA merges)
   int dyn;          // 1: few (sequence, K/V head) units, whole waves: grains handed out at run time
 };
 // Split plan constants: resident decode CTAs of 16 query heads per SM (two
@@ -46,8 +45,8 @@ int plan_decode(int B, int Hq, int Hkv, int max_seq_len, int num_sms, DecodePlan
 // most tokens a windowed query's visible sub-block list can span.
 int decode_plan_length(int max_seq_len, int window, int n_sink);
 // Workspace: partial outputs [B, Hq, splits, d] fp32, partial LSEs
-// [B, Hq, splits] fp32, then (16-byte aligned) the merge's ticket counters and
-// the grain counter, 2 + ngroups uint64 per (sequence, K/V head, head chunk).
+// [B, Hq, splits] fp32, then (16-byte aligned) the merge's ticket counter and
+// the grain counter, two uint64 per (sequence, K/V head, head chunk).
 struct DecodeWorkspace {
   size_t o_part_offset, lse_part_offset, counters_offset, bytes;
 };

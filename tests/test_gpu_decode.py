@@ -213,7 +213,7 @@ def test_full_size_sampled(name):
 
 # --------------------------------------------------------------------------
 # the in-launch split merge: ticket counters in a reused, never-cleared
-# workspace; two-level merges; a result that does not depend on which CTA
+# workspace; the merge kernel; a result that does not depend on which CTA
 # finished last
 # --------------------------------------------------------------------------
 def test_fixed_split_plan_is_bit_reproducible():
@@ -237,11 +237,13 @@ def test_run_time_grains_cover_every_token():
     _check(x, what="run-time grains")
 
 
-def test_two_level_merge_single_sequence():
-    """16 query heads on one K/V head: 139 splits merged as 12 groups (the
-    last one partial), then the groups."""
+def test_merge_kernel_single_sequence():
+    """16 query heads on one K/V head: more splits than one CTA stages at once
+    (192 / 16 rows), so the split grid leaves its partials to the merge kernel
+    (launched as a programmatic dependent of the one-wave split grid, with
+    run-time grains in the split kernel)."""
     x = workloads.paged_decode_inputs(1, 16, 1, 128, seq_lens=[40000], block_size=16, seed=21)
-    _check(x, poison=False, what="two-level merge")
+    _check(x, poison=False, what="merge kernel")
 
 
 def test_workspace_reused_with_garbage_and_other_plans():
