@@ -296,6 +296,27 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       // test), so the parity tests are unambiguous.
       int ns = 0, npv = 0;
       long long idle_since = clock64();
+      // O^T += V^T . P^T of tile npv when its P^T has been written (the softmax
+      // rescaled O^T first where its max moved); its commit frees the tile's slot.
+      auto try_pv = [&]() -> bool {
+        if (npv >= ns) return false;
+        const int sl = npv % kSlots;
+        if (!mbar_test_wait(bar(kMbPFull + sl), (npv / kSlots) & 1)) return false;
+        tc_fence_after();
+        for (int m = 0; m < 4; ++m) {
+#pragma unroll
+          for (int kk = 0; kk < kTok / 16; ++kk) {
+            const uint64_t a =
+                dv + sl * kTileUnits + static_cast<uint64_t>((2 * m * kKChunkBytes + kk * 2048) >> 4);
+            const uint64_t bp = dp + sl * kTileUnits + static_cast<uint64_t>((kk * 2048) >> 4);
+            tc_mma_ss(tmem + kColO + 64u * m, a, bp, kIdescOut, (npv > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(bar(kMbKEmpty + sl));
+        tc_commit(bar(kMbOReady));
+        ++npv;
+        return true;
+      };
       while (ok && npv < ntiles) {
         bool progressed = false;
         if (ns < ntiles && ns < npv + kSlots) {
@@ -303,7 +324,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
           if (mbar_test_wait(bar(kMbKFull + sl), (ns / kSlots) & 1) &&
               (ns < kSlots || mbar_test_wait(bar(kMbSFree + sl), ((ns - kSlots) / kSlots) & 1))) {
             tc_fence_after();
-            // S^T = K . Q^T over the nine chunks, 4 steps of 16 columns each
+            // S^T = K . Q^T over the nine chunks, 4 steps of 16 columns each. Issuing
+            // MMAs blocks while the tensor pipe is busy, so between chunks a tile whose
+            // P^T is ready gets its output MMAs first: they free its slot for the next
+            // copy instead of waiting behind the whole score product.
             for (int j = 0; j < kChunks; ++j) {
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
@@ -311,32 +335,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 const uint64_t bq = dq + static_cast<uint64_t>((j * kQChunkBytes + kk * 32) >> 4);
                 tc_mma_ss(tmem + kColS + 64u * sl, a, bq, kIdescScore, (j | kk) != 0 ? 1u : 0u);
               }
+              try_pv();
             }
             tc_commit(bar(kMbSFull + sl));
             ++ns;
             progressed = true;
           }
         }
-        if (!progressed && npv < ns) {
-          const int sl = npv % kSlots;
-          if (mbar_test_wait(bar(kMbPFull + sl), (npv / kSlots) & 1)) {
-            tc_fence_after();
-            // O^T += V^T . P^T (the softmax rescaled O^T first where its max moved)
-            for (int m = 0; m < 4; ++m) {
-#pragma unroll
-              for (int kk = 0; kk < kTok / 16; ++kk) {
-                const uint64_t a =
-                    dv + sl * kTileUnits + static_cast<uint64_t>((2 * m * kKChunkBytes + kk * 2048) >> 4);
-                const uint64_t bp = dp + sl * kTileUnits + static_cast<uint64_t>((kk * 2048) >> 4);
-                tc_mma_ss(tmem + kColO + 64u * m, a, bp, kIdescOut, (npv > 0 || kk > 0) ? 1u : 0u);
-              }
-            }
-            tc_commit(bar(kMbKEmpty + sl));
-            tc_commit(bar(kMbOReady));
-            ++npv;
-            progressed = true;
-          }
-        }
+        if (!progressed) progressed = try_pv();
         if (progressed) {
           idle_since = clock64();
         } else if (*abort_flag || clock64() - idle_since > budget) {
