@@ -57,6 +57,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <type_traits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -118,6 +119,7 @@ constexpr uint32_t idesc_mla(int M, int N, int a_mn, int b_mn) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 constexpr uint32_t kIdescScore = idesc_mla(kTok, kNH, 0, 0);  // S^T = K . Q^T, both K-major
+constexpr uint32_t kIdescScore16 = idesc_mla(kTok, 16, 0, 0);  // the same for a block of <= 16 heads
 constexpr uint32_t kIdescOut = idesc_mla(128, kNH, 1, 1);     // O^T += V^T . P^T, both MN-major
 
 struct MlaParams {
@@ -136,12 +138,13 @@ __device__ __forceinline__ void mla_abort(volatile int* abort_flag, int32_t* sta
   if (status != nullptr) atomicOr(status, ATTN_STATUS_BIT_TIMEOUT);
 }
 
-// Warp reduce-scatter of 32 columns: on entry lane l holds v[c] for its token
-// row; on exit lane l holds the max (or sum) of column l over the 32 rows.
-template <bool kMax>
-__device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32], int lane) {
+// Warp reduce-scatter of NC columns (16 or 32): on entry lane l holds v[c] for
+// its token row; on exit lane l holds the max (or sum) of column l % NC over
+// the 32 rows.
+template <int NC, bool kMax>
+__device__ __forceinline__ float warp_reduce_scatter(float (&v)[NC], int lane) {
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
+  for (int o = NC / 2; o >= 1; o >>= 1) {
     const bool upper = (lane & o) != 0;
 #pragma unroll
     for (int k = 0; k < o; ++k) {
@@ -150,6 +153,11 @@ __device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32], int lane)
       const float recv = __shfl_xor_sync(0xffffffffu, send, o);
       v[k] = kMax ? fmaxf(keep, recv) : keep + recv;
     }
+  }
+#pragma unroll
+  for (int o = NC; o < 32; o <<= 1) {  // the lane groups that held different rows
+    const float recv = __shfl_xor_sync(0xffffffffu, v[0], o);
+    v[0] = kMax ? fmaxf(v[0], recv) : v[0] + recv;
   }
   return v[0];
 }
@@ -174,6 +182,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   if (t0 >= seq_len) return;  // nothing cached in this split: the merge never reads it
   const int t1 = min(t0 + p.chunk, seq_len);
   const int ntiles = (t1 - t0 + kTok - 1) / kTok;
+  // this block holds at most 16 heads (H = 16, or a last block of at most 16)
+  const bool narrow = p.H - hb * kNH <= 16;
 
   const uint32_t bars = sbase + kBarOff;
   auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
@@ -296,6 +306,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       // test), so the parity tests are unambiguous.
       int ns = 0, npv = 0;
       long long idle_since = clock64();
+      // a block of at most 16 heads scores only its first 16 query columns
+      const uint32_t idesc_s = narrow ? kIdescScore16 : kIdescScore;
       // O^T += V^T . P^T of tile npv when its P^T has been written (the softmax
       // rescaled O^T first where its max moved); its commit frees the tile's slot.
       auto try_pv = [&]() -> bool {
@@ -333,7 +345,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t a = dk + sl * kTileUnits + static_cast<uint64_t>((j * kKChunkBytes + kk * 32) >> 4);
                 const uint64_t bq = dq + static_cast<uint64_t>((j * kQChunkBytes + kk * 32) >> 4);
-                tc_mma_ss(tmem + kColS + 64u * sl, a, bq, kIdescScore, (j | kk) != 0 ? 1u : 0u);
+                tc_mma_ss(tmem + kColS + 64u * sl, a, bq, idesc_s, (j | kk) != 0 ? 1u : 0u);
               }
               try_pv();
             }
@@ -399,6 +411,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // Every softmax warp takes part in every named barrier of every tile, also
     // after a wait gave up (ok == false: it then skips its TMEM and mbarrier
     // work), so no warp can be left waiting at a barrier the others skipped.
+    // NC: the head columns this warp scores (32, or 16 in a block of at most 16
+    // heads, whose remaining columns of P^T are written as zeros).
+    auto run = [&](auto nc_tag) {
+    constexpr int NC = decltype(nc_tag)::value;
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
       const int sb = i % kSlots;
@@ -410,13 +426,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       float wmax = -INFINITY;
       if (ok) {
         tc_fence_after();
-        uint32_t raw[32];
-        tmem_ld_32x32b_x32(col_s, raw);
+        uint32_t raw[NC];
+        if constexpr (NC == 32) tmem_ld_32x32b_x32(col_s, raw);
+        else tmem_ld_32x32b_x16(col_s, raw);
         tc_wait_ld();
-        float v[32];
+        float v[NC];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) v[c] = valid ? __uint_as_float(raw[c]) * sl2 : -INFINITY;
-        wmax = warp_reduce_scatter32<true>(v, lane);  // lane c: column c over this warp's 16 tokens
+        for (int c = 0; c < NC; ++c) v[c] = valid ? __uint_as_float(raw[c]) * sl2 : -INFINITY;
+        wmax = warp_reduce_scatter<NC, true>(v, lane);  // lane c: column c % NC over this warp's 16 tokens
       }
       // tile max of every head column across the 4 warps; running max update
       red[sp * 32 + lane] = wmax;
@@ -431,7 +448,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       if (!ok) continue;
       if (__any_sync(0xffffffffu, moved)) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) l_part[c] *= __shfl_sync(0xffffffffu, a_lane, c);
+        for (int c = 0; c < NC; ++c) l_part[c] *= __shfl_sync(0xffffffffu, a_lane, c);
         if (i > 0) {
           // the previous tile's output MMAs must be complete before O^T is rescaled
           ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kMbOReady), (i - 1) & 1, budget, abort_flag));
@@ -454,8 +471,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       // probabilities from a second read of the scores (fewer live registers);
       // P^T row tok (lanes 0-15), head columns 32 hh .. + 31 -> 64 bytes of the
       // 128-byte swizzled row: 16-byte chunk q lands at chunk q ^ (tok & 7)
-      uint32_t raw[32];
-      tmem_ld_32x32b_x32(col_s, raw);
+      uint32_t raw[NC];
+      if constexpr (NC == 32) tmem_ld_32x32b_x32(col_s, raw);
+      else tmem_ld_32x32b_x16(col_s, raw);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -463,13 +481,17 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       uint32_t pk[16];
 #pragma unroll
       for (int c = 0; c < 32; c += 2) {
-        const float x0 = valid ? __uint_as_float(raw[c]) * sl2 : -INFINITY;
-        const float x1 = valid ? __uint_as_float(raw[c + 1]) * sl2 : -INFINITY;
-        const float p0 = fast_exp2(x0 - __shfl_sync(0xffffffffu, m_lane, c));
-        const float p1 = fast_exp2(x1 - __shfl_sync(0xffffffffu, m_lane, c + 1));
-        l_part[c] += p0;
-        l_part[c + 1] += p1;
-        pk[c >> 1] = pack_bf16x2(p0, p1);
+        if (c < NC) {
+          const float x0 = valid ? __uint_as_float(raw[c]) * sl2 : -INFINITY;
+          const float x1 = valid ? __uint_as_float(raw[c + 1]) * sl2 : -INFINITY;
+          const float p0 = fast_exp2(x0 - __shfl_sync(0xffffffffu, m_lane, c));
+          const float p1 = fast_exp2(x1 - __shfl_sync(0xffffffffu, m_lane, c + 1));
+          l_part[c] += p0;
+          l_part[c + 1] += p1;
+          pk[c >> 1] = pack_bf16x2(p0, p1);
+        } else {
+          pk[c >> 1] = 0u;  // heads past the block's 16
+        }
       }
       if (lane < 16) {
         uint8_t* pslot = smem + kKOff + sb * kTileBytes + kPSlot * kKChunkBytes;
@@ -491,7 +513,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     if (!ok) mla_abort(abort_flag, p.status);
     tc_fence_after();
     // column sums of the probabilities over all 64 token rows
-    const float wsum = warp_reduce_scatter32<false>(l_part, lane);
+    float l_nc[NC];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) l_nc[c] = l_part[c];
+    const float wsum = warp_reduce_scatter<NC, false>(l_nc, lane);
     red[sp * 32 + lane] = wsum;
     named_sync(1 + hh, 128);
     const float csum = (red[lane] + red[32 + lane]) + (red[64 + lane] + red[96 + lane]);
@@ -499,7 +524,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     if (threadIdx.x == 0 && *bad_flag != 0 && p.status != nullptr) atomicOr(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
     const float inv_lane = 1.f / csum;
     const int head0 = hb * kNH + hh * 32;
-    if (sp == 0 && head0 + lane < p.H)  // one warp per column half writes the partial log-sum-exps
+    if (sp == 0 && lane < NC && head0 + lane < p.H)  // one warp per column half writes the partial log-sum-exps
       p.lse_part[(static_cast<size_t>(b) * p.H + head0 + lane) * p.splits + split] =
           out_ok ? (m_lane + __log2f(csum)) * kLn2 : NAN;
 #pragma unroll 1
@@ -510,11 +535,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         const float inv = __shfl_sync(0xffffffffu, inv_lane, c);
-        if (head0 + c < p.H)
+        if (c < NC && head0 + c < p.H)
           p.o_part[((static_cast<size_t>(b) * p.H + head0 + c) * p.splits + split) * kDc + m * 128 + r] =
               out_ok ? __uint_as_float(ov[c]) * inv : NAN;
       }
     }
+    };
+    if (narrow) run(std::integral_constant<int, 16>{});
+    else run(std::integral_constant<int, 32>{});
     }
   }
 
