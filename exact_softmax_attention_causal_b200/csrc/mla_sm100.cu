@@ -382,10 +382,16 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     for (int c = 0; c < 32; ++c) l_part[c] = 0.f;
     float m_lane = -INFINITY;  // lane c: the max head column 32 hh + c's exponentials use (base 2)
     named_sync(1 + hh, 128);
-    if (hb * kNH + hh * 32 >= p.H) {
-      // A column half with no head of this block (H < 64 or a partial last block):
-      // its P^T columns are zero for every tile, written once the score MMAs have
-      // read the tile's positional chunk; nothing else is computed or stored.
+    // This half's head columns: 32 hh .. 32 hh + 31, or in a block of at most
+    // 16 heads 8 hh .. 8 hh + 7. Each half writes its own 16-byte chunks of
+    // every P^T row: its data chunk (4 hh .. 4 hh + 3, or hh) and, in a narrow
+    // block, three of the six zero chunks 2 .. 7.
+    const int cb = narrow ? 8 * hh : 32 * hh;
+    auto chunk_of = [&](int q) { return narrow ? (q == 0 ? hh : 1 + 3 * hh + q) : 4 * hh + q; };
+    if (hb * kNH + cb >= p.H) {
+      // A column half with no head of this block: its P^T chunks are zero for
+      // every tile, written once the score MMAs have read the tile's positional
+      // chunk; nothing else is computed or stored.
       bool idle_ok = true;
       for (int i = 0; i < ntiles; ++i) {
         const int sb = i % kSlots;
@@ -398,7 +404,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
           uint8_t* pslot = smem + kKOff + sb * kTileBytes + kPSlot * kKChunkBytes;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const int chunk = hh * 4 + q;
+            const int chunk = chunk_of(q);
             *reinterpret_cast<uint4*>(pslot + tok * 128 + ((chunk ^ (tok & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
           }
         }
@@ -411,14 +417,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // Every softmax warp takes part in every named barrier of every tile, also
     // after a wait gave up (ok == false: it then skips its TMEM and mbarrier
     // work), so no warp can be left waiting at a barrier the others skipped.
-    // NC: the head columns this warp scores (32, or 16 in a block of at most 16
+    // NC: the head columns this warp scores (32, or 8 in a block of at most 16
     // heads, whose remaining columns of P^T are written as zeros).
     auto run = [&](auto nc_tag) {
     constexpr int NC = decltype(nc_tag)::value;
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
       const int sb = i % kSlots;
-      const uint32_t col_s = lane_base + kColS + 64u * sb + 32u * hh;
+      const uint32_t col_s = lane_base + kColS + 64u * sb + static_cast<uint32_t>(cb);
       if (ok)
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kMbSFull + sb), (i / kSlots) & 1, budget, abort_flag));
       // lanes 16-31 of the sub-partition hold no score of an M = 64 tile
@@ -428,7 +434,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         tc_fence_after();
         uint32_t raw[NC];
         if constexpr (NC == 32) tmem_ld_32x32b_x32(col_s, raw);
-        else tmem_ld_32x32b_x16(col_s, raw);
+        else tmem_ld_32x32b_x8(col_s, raw);
         tc_wait_ld();
         float v[NC];
 #pragma unroll
@@ -456,14 +462,16 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
           tc_fence_after();
 #pragma unroll 1
           for (int m = 0; m < 4; ++m) {
-            uint32_t ov[32];
-            const uint32_t col = lane_base + kColO + 64u * m + 32u * hh;
-            tmem_ld_32x32b_x32(col, ov);
+            uint32_t ov[NC];  // only this half's columns: a narrow block's halves share a 32-column window
+            const uint32_t col = lane_base + kColO + 64u * m + static_cast<uint32_t>(cb);
+            if constexpr (NC == 32) tmem_ld_32x32b_x32(col, ov);
+            else tmem_ld_32x32b_x8(col, ov);
             tc_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
+            for (int c = 0; c < NC; ++c)
               ov[c] = __float_as_uint(__uint_as_float(ov[c]) * __shfl_sync(0xffffffffu, a_lane, c));
-            tmem_st_32x32b_x32(col, ov);
+            if constexpr (NC == 32) tmem_st_32x32b_x32(col, ov);
+            else tmem_st_32x32b_x8(col, ov);
           }
           tc_wait_st();
         }
@@ -473,7 +481,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       // 128-byte swizzled row: 16-byte chunk q lands at chunk q ^ (tok & 7)
       uint32_t raw[NC];
       if constexpr (NC == 32) tmem_ld_32x32b_x32(col_s, raw);
-      else tmem_ld_32x32b_x16(col_s, raw);
+      else tmem_ld_32x32b_x8(col_s, raw);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -490,14 +498,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
           l_part[c + 1] += p1;
           pk[c >> 1] = pack_bf16x2(p0, p1);
         } else {
-          pk[c >> 1] = 0u;  // heads past the block's 16
+          pk[c >> 1] = 0u;  // the zero chunks of a narrow block
         }
       }
       if (lane < 16) {
         uint8_t* pslot = smem + kKOff + sb * kTileBytes + kPSlot * kKChunkBytes;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int chunk = hh * 4 + q;
+          const int chunk = chunk_of(q);
           *reinterpret_cast<uint4*>(pslot + tok * 128 + ((chunk ^ (tok & 7)) << 4)) =
               make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
         }
@@ -523,14 +531,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     const bool out_ok = ok && (*bad_flag == 0);
     if (threadIdx.x == 0 && *bad_flag != 0 && p.status != nullptr) atomicOr(p.status, ATTN_STATUS_BIT_DEVICE_CHECK);
     const float inv_lane = 1.f / csum;
-    const int head0 = hb * kNH + hh * 32;
+    const int head0 = hb * kNH + cb;
     if (sp == 0 && lane < NC && head0 + lane < p.H)  // one warp per column half writes the partial log-sum-exps
       p.lse_part[(static_cast<size_t>(b) * p.H + head0 + lane) * p.splits + split] =
           out_ok ? (m_lane + __log2f(csum)) * kLn2 : NAN;
 #pragma unroll 1
     for (int m = 0; m < 4; ++m) {
       uint32_t ov[32];
-      tmem_ld_32x32b_x32(lane_base + kColO + 64u * m + 32u * hh, ov);
+      tmem_ld_32x32b_x32(lane_base + kColO + 64u * m + static_cast<uint32_t>(cb), ov);
       tc_wait_ld();
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
@@ -541,7 +549,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       }
     }
     };
-    if (narrow) run(std::integral_constant<int, 16>{});
+    if (narrow) run(std::integral_constant<int, 8>{});
     else run(std::integral_constant<int, 32>{});
     }
   }
