@@ -46,7 +46,7 @@ def _check(x, seqs=None, heads=None, poison=True, what=""):
     return o, lse
 
 
-@pytest.mark.parametrize("H", [128, 64, 16, 100, 32, 20, 96, 80, 8])
+@pytest.mark.parametrize("H", [128, 64, 16, 100, 32, 20, 96, 80, 8, 12, 72])
 def test_mixed_lengths(H):
     # one token, a ragged tile, several tiles, and enough tokens for several splits
     x = workloads.mla_decode_inputs(4, H, 512, 64, seq_lens=[1, 130, 700, 9000], block_size=16, seed=H,
