@@ -60,8 +60,9 @@ def test_block_sizes(bs):
     _check(x, what=f"bs={bs}")
 
 
-def test_deterministic_and_permutation_invariant():
-    x = workloads.mla_decode_inputs(2, 64, 512, 64, seq_lens=[300, 2000], block_size=16, seed=5, extra_blocks=4)
+@pytest.mark.parametrize("H", [64, 16])
+def test_deterministic_and_permutation_invariant(H):
+    x = workloads.mla_decode_inputs(2, H, 512, 64, seq_lens=[300, 2000], block_size=16, seed=5, extra_blocks=4)
     o1, l1 = _run(x)
     o2, l2 = _run(x)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
@@ -75,15 +76,16 @@ def test_deterministic_and_permutation_invariant():
     assert torch.equal(o3.cpu(), o1) and torch.equal(l3.cpu(), l1)
 
 
-def test_bad_entry_and_seq_len_are_flagged():
-    x = workloads.mla_decode_inputs(3, 128, 512, 64, seq_lens=[200, 200, 200], block_size=16, seed=6)
+@pytest.mark.parametrize("H", [128, 16])
+def test_bad_entry_and_seq_len_are_flagged(H):
+    x = workloads.mla_decode_inputs(3, H, 512, 64, seq_lens=[200, 200, 200], block_size=16, seed=6)
     x.block_table[1, 5] = 10 ** 6
     x.seq_lens[2] = 0
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     o, lse = _run(x, status)
     assert int(status.item()) & 0x1
     assert torch.isnan(o[1].float()).all() and torch.isnan(o[2].float()).all()
-    o_ref, l_ref = oracle.mla_decode_rows_ref(x.q, x.cache, x.block_table, x.seq_lens, 0, range(128), 512, SCALE)
+    o_ref, l_ref = oracle.mla_decode_rows_ref(x.q, x.cache, x.block_table, x.seq_lens, 0, range(H), 512, SCALE)
     assert_parity(o[0], o_ref, lse[0], l_ref)
 
 
